@@ -1,0 +1,9 @@
+"""Oracle (test infrastructure): fp64 CPU restatement of the decode step.
+
+Importable only from tests/, __graft_entry__.smoke() and bench.py's CPU-baseline legs.
+"""
+from .retrieval_attention import (  # noqa: F401
+    attend, attention_mass, bf16_to_f64, candidate_set, decode_head, decode_step,
+    dense_decode, dense_head, merge_partials, partial_state, scores, select_topk,
+    softmax_weights, static_set, threshold_set,
+)

@@ -1,0 +1,199 @@
+"""Oracle for one decode step of RetrievalAttention with exact top-k retrieval (fp64, CPU).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.  The
+product (``top_retrieval_attention_b200``) never imports it and has no CPU fallback.
+
+It is a plain, slow restatement of what the method computes, written from the slides
+"RetrievalAttention: Accelerating Long-Context LLM Inference via Vector Retrieval"
+(arXiv 2409.10516v3 paper discussion).  Library primitives used as single steps: a
+matrix-vector product, a lexicographic sort, ``exp``.  No blocking, fusion or reordering.
+
+Notation follows the slides: query q_t, keys k_i, values v_i, head dimension d, scores
+z_i, static set W (first sink tokens plus the last window), dynamic set Omega (the
+retrieved top-k), partial softmax state (m_S, Z_S, N_S, o_S) and merge weights gamma_S.
+
+Inputs are bf16 bit patterns (uint16 arrays), decoded exactly to float64.
+  q : [B, Hq, d]        K, V : [B, Hkv, N, d]        query head h reads KV head h // G.
+
+Readings of points the slides leave open (each is listed with its reason in the design
+notes of the repository):
+  * W and Omega are disjoint ("The GPU keeps 640 fixed positions": "W and Omega are
+    disjoint"), so the top-k runs over the candidates C = [0, N) minus W only.
+  * Ties in z go to the lower position; k larger than |C| is clamped to |C|.
+  * W = [0, min(n_sink, N)) union [max(0, N - n_window), N); the two may overlap.
+  * The output is the exact softmax over U = W union Omega in fp64 ("Two local softmax
+    outputs need global weights": the merge equals softmax over the selected union).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# ------------------------------------------------------------------------------------
+# inputs
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit pattern -> float64 (exact: bf16 is the top half of an IEEE float)."""
+    u = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+# ------------------------------------------------------------------------------------
+# Eq. (1): scaled dot-product scores and the softmax over the history
+
+
+def scores(q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """z_i = q_t k_i^T / sqrt(d) for every cached key (slide "Sparse attention
+    renormalizes selected tokens", Eq. (1)).  q [d] float64, K [N, d] float64."""
+    d = q.shape[-1]
+    return (K @ q) / math.sqrt(d)
+
+
+def softmax_weights(z: np.ndarray) -> np.ndarray:
+    """a_{t,i} = e^{z_i} / sum_j e^{z_j} over the whole history (Eq. (1)), computed with
+    the max subtracted (the identity e^{z-m}/sum e^{z-m} = e^z/sum e^z)."""
+    m = np.max(z)
+    e = np.exp(z - m)
+    return e / np.sum(e)
+
+
+def threshold_set(z: np.ndarray, eps: float) -> np.ndarray:
+    """I_{t,eps} = {i : a_{t,i} > eps} (Eq. (2)), ascending positions."""
+    return np.nonzero(softmax_weights(z) > eps)[0]
+
+
+def attention_mass(z: np.ndarray, U: np.ndarray) -> float:
+    """Share of the full softmax mass that the positions U recover (the statistic of
+    slide "The active tokens are sparse and dynamic", Fig. 2)."""
+    return float(np.sum(softmax_weights(z)[np.asarray(U, dtype=np.int64)]))
+
+
+# ------------------------------------------------------------------------------------
+# the static set W and the candidates C ("The GPU keeps 640 fixed positions")
+
+
+def static_set(N: int, n_sink: int, n_window: int) -> np.ndarray:
+    """W: the first n_sink tokens plus the last n_window tokens, ascending, no repeats."""
+    sink = np.arange(0, min(n_sink, N), dtype=np.int64)
+    window = np.arange(max(0, N - n_window), N, dtype=np.int64)
+    return np.union1d(sink, window)
+
+
+def candidate_set(N: int, n_sink: int, n_window: int) -> np.ndarray:
+    """C = [0, N) minus W: the positions the dynamic retrieval may return."""
+    return np.setdiff1d(np.arange(N, dtype=np.int64), static_set(N, n_sink, n_window))
+
+
+def select_topk(z: np.ndarray, C: np.ndarray, k: int) -> np.ndarray:
+    """Omega: the min(k, |C|) candidates with the largest z (slide "Sparse attention
+    renormalizes selected tokens": a fixed top-k budget rather than a threshold).
+    Full sort by (z descending, position ascending), then take the head of the order."""
+    C = np.asarray(C, dtype=np.int64)
+    k_eff = min(max(k, 0), C.size)
+    order = np.lexsort((C, -z[C]))
+    return C[order[:k_eff]]
+
+
+# ------------------------------------------------------------------------------------
+# softmax over a selected set, partial states and their merge
+# (slide "Two local softmax outputs need global weights", Eqs. (3)-(5), and the backup
+#  slide "The normalization identity", Appendix B)
+
+
+def attend(z: np.ndarray, V: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """o = sum_{i in U} e^{z_i} v_i / sum_{j in U} e^{z_j} (Eq. (2)'s renormalised sum
+    over the selected set), evaluated with the max over U subtracted."""
+    U = np.asarray(U, dtype=np.int64)
+    zu = z[U]
+    m = np.max(zu)
+    w = np.exp(zu - m)
+    return (w @ V[U]) / np.sum(w)
+
+
+def partial_state(z: np.ndarray, V: np.ndarray, S: np.ndarray):
+    """(m_S, Z_S, N_S) of one subset S: m_S = max z, Z_S = sum e^{z-m_S},
+    N_S = sum e^{z-m_S} v (backup slide, Appendix B).  o_S = N_S / Z_S."""
+    S = np.asarray(S, dtype=np.int64)
+    zs = z[S]
+    m = float(np.max(zs))
+    w = np.exp(zs - m)
+    return m, float(np.sum(w)), w @ V[S]
+
+
+def merge_partials(parts) -> np.ndarray:
+    """o = sum_S gamma_S o_S with gamma_S = e^{m_S-m} Z_S / sum_T e^{m_T-m} Z_T and
+    m = max_S m_S (Eqs. (3)-(5), generalised from the two parts W, Omega to any number of
+    disjoint parts)."""
+    m = max(p[0] for p in parts)
+    den = sum(math.exp(mS - m) * ZS for mS, ZS, _ in parts)
+    o = 0.0
+    for mS, ZS, NS in parts:
+        gamma = math.exp(mS - m) * ZS / den
+        o = o + gamma * (NS / ZS)
+    return np.asarray(o, dtype=np.float64)
+
+
+# ------------------------------------------------------------------------------------
+# the decode step
+
+
+def decode_head(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray, k: int,
+                n_sink: int, n_window: int):
+    """One query head: returns (o [d], Omega, z).  q [d], K/V [N, d] as bf16 bits."""
+    q = bf16_to_f64(q_bits)
+    K = bf16_to_f64(K_bits)
+    V = bf16_to_f64(V_bits)
+    N = K.shape[0]
+    if N == 0:
+        raise ValueError("empty cache")
+    z = scores(q, K)
+    W = static_set(N, n_sink, n_window)
+    C = candidate_set(N, n_sink, n_window)
+    omega = select_topk(z, C, k)
+    U = np.concatenate([W, omega])
+    if U.size == 0:
+        raise ValueError("empty selected union")
+    return attend(z, V, U), omega, z
+
+
+def decode_step(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray, k: int,
+                n_sink: int, n_window: int):
+    """All (b, h): out [B, Hq, d] float64 and Omega per (b, h) (list of lists).
+
+    GQA: query head h reads KV head h // G with its own selection (slide "The GPU keeps
+    640 fixed positions": GQA heads get separate indices but share KV storage)."""
+    B, Hq, d = q_bits.shape
+    Hkv = K_bits.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    omegas = [[None] * Hq for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            o, om, _ = decode_head(q_bits[b, h], K_bits[b, h // G], V_bits[b, h // G], k,
+                                   n_sink, n_window)
+            out[b, h] = o
+            omegas[b][h] = om
+    return out, omegas
+
+
+def dense_head(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray) -> np.ndarray:
+    """Full attention of one query head over all N cached tokens (Eq. (1))."""
+    q = bf16_to_f64(q_bits)
+    K = bf16_to_f64(K_bits)
+    V = bf16_to_f64(V_bits)
+    z = scores(q, K)
+    return attend(z, V, np.arange(K.shape[0]))
+
+
+def dense_decode(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray) -> np.ndarray:
+    B, Hq, d = q_bits.shape
+    G = Hq // K_bits.shape[1]
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            out[b, h] = dense_head(q_bits[b, h], K_bits[b, h // G], V_bits[b, h // G])
+    return out

@@ -1,0 +1,83 @@
+"""Planted mistakes in the oracle (CPU only): each must make at least one pin fail.
+
+The mistakes are planted by monkeypatching the oracle module for the duration of a test;
+the oracle's files are never modified.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.retrieval_attention as ra
+import test_oracle_pins as pins
+
+
+def _patch(monkeypatch, name, fn):
+    monkeypatch.setattr(ra, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_wrong_score_scale_is_caught(monkeypatch):
+    _patch(monkeypatch, "scores", lambda q, K: (K @ q) / q.shape[-1])
+    assert _fails(pins.test_scores_match_exact_rationals, 64)
+
+
+def test_transposed_or_dropped_term_is_caught(monkeypatch):
+    _patch(monkeypatch, "scores", lambda q, K: (K[:, 1:] @ q[1:]) / math.sqrt(q.shape[-1]))
+    assert _fails(pins.test_scores_match_exact_rationals, 128)
+
+
+def test_ascending_selection_is_caught(monkeypatch):
+    def bad(z, C, k):
+        C = np.asarray(C, dtype=np.int64)
+        order = np.lexsort((C, z[C]))
+        return C[order[:min(k, C.size)]]
+    _patch(monkeypatch, "select_topk", bad)
+    assert _fails(pins.test_topk_brute_force_with_ties, 0)
+
+
+def test_ties_to_higher_position_are_caught(monkeypatch):
+    def bad(z, C, k):
+        C = np.asarray(C, dtype=np.int64)
+        order = np.lexsort((-C, -z[C]))
+        return C[order[:min(k, C.size)]]
+    _patch(monkeypatch, "select_topk", bad)
+    assert any(_fails(pins.test_topk_brute_force_with_ties, t) for t in range(10))
+
+
+def test_overlapping_static_and_dynamic_sets_are_caught(monkeypatch):
+    _patch(monkeypatch, "candidate_set", lambda N, s, w: np.arange(N, dtype=np.int64))
+    assert _fails(pins.test_topk_brute_force_with_ties, 1)
+
+
+def test_window_off_by_one_is_caught(monkeypatch):
+    def bad(N, n_sink, n_window):
+        return np.union1d(np.arange(0, min(n_sink, N)), np.arange(max(0, N - n_window - 1), N))
+    _patch(monkeypatch, "static_set", bad)
+    assert _fails(pins.test_static_set_and_candidates)
+
+
+def test_merge_without_rescale_is_caught(monkeypatch):
+    def bad(parts):
+        den = sum(ZS for _, ZS, _ in parts)
+        return sum((ZS / den) * (NS / ZS) for _, ZS, NS in parts)
+    _patch(monkeypatch, "merge_partials", bad)
+    assert _fails(pins.test_merge_of_disjoint_parts_equals_union_softmax, 3)
+
+
+def test_unnormalised_attention_is_caught(monkeypatch):
+    def bad(z, V, U):
+        U = np.asarray(U, dtype=np.int64)
+        w = np.exp(z[U] - np.max(z[U]))
+        return w @ V[U]
+    _patch(monkeypatch, "attend", bad)
+    assert _fails(pins.test_dense_matches_torch_sdpa_fp64, 7, 128)

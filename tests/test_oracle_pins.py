@@ -1,0 +1,377 @@
+"""Pins of the fp64 oracle to facts outside itself (CPU only).
+
+Each test checks the oracle against something it does not compute the same way: exact
+rational arithmetic, a closed form, an independent library routine (torch's
+scaled-dot-product attention in float64), brute-force enumeration on tiny inputs, or an
+identity the slides state.  A plausible mistake (wrong scale, dropped term, transposed
+operand, wrong sort direction or tie rule, W and Omega overlapping, a missing rescale in
+the merge) fails at least one of them.
+"""
+import itertools
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import oracle
+from synth import gen
+
+RNG = np.random.default_rng(1234)
+
+
+def rand_bf16(shape, scale=1.0, rng=RNG):
+    return gen.f64_to_bf16_bits(rng.standard_normal(shape) * scale)
+
+
+# ---------------------------------------------------------------- bf16 decode
+
+
+def test_bf16_decode_known_patterns():
+    bits = np.array([0x3F80, 0xBF80, 0x4000, 0x3F00, 0x0000, 0x8000, 0x4049, 0x7F7F],
+                    dtype=np.uint16)
+    want = [1.0, -1.0, 2.0, 0.5, 0.0, -0.0, 3.140625, 3.3895313892515355e38]
+    got = oracle.bf16_to_f64(bits)
+    assert list(got) == want
+
+
+# ---------------------------------------------------------------- Eq. (1) scores
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_scores_match_exact_rationals(d):
+    """z_i = q k_i / sqrt(d): the dot product of bf16 values is a dyadic rational that
+    Fraction computes exactly; the oracle must agree to fp64 rounding."""
+    q = rand_bf16(d)
+    K = rand_bf16((17, d))
+    z = oracle.scores(oracle.bf16_to_f64(q), oracle.bf16_to_f64(K))
+    qf = [Fraction(float(x)) for x in oracle.bf16_to_f64(q)]
+    for i in range(K.shape[0]):
+        kf = [Fraction(float(x)) for x in oracle.bf16_to_f64(K[i])]
+        dot = sum(a * b for a, b in zip(qf, kf))
+        if d == 64:
+            exact = float(dot / 8)          # sqrt(64) = 8 exactly
+            assert abs(z[i] - exact) <= 4e-16 * max(1.0, abs(exact)) * d
+        else:
+            exact = float(dot) / math.sqrt(d)
+            assert abs(z[i] - exact) <= 1e-14 * max(1.0, abs(exact))
+
+
+def test_scores_unit_query_reads_one_channel():
+    d = 128
+    K = rand_bf16((9, d))
+    Kf = oracle.bf16_to_f64(K)
+    for j in (0, 5, 127):
+        q = np.zeros(d)
+        q[j] = 2.0
+        z = oracle.scores(q, Kf)
+        assert np.array_equal(z, 2.0 * Kf[:, j] / math.sqrt(d))
+
+
+# ---------------------------------------------------------------- static set W
+
+
+def test_static_set_and_candidates():
+    W = oracle.static_set(1000, 4, 64)
+    assert list(W) == list(range(4)) + list(range(936, 1000))
+    C = oracle.candidate_set(1000, 4, 64)
+    assert list(C) == list(range(4, 936))
+    # overlap: N < n_sink + n_window -> W is everything, C empty
+    assert list(oracle.static_set(50, 32, 32)) == list(range(50))
+    assert oracle.candidate_set(50, 32, 32).size == 0
+    # no static set at all
+    assert oracle.static_set(10, 0, 0).size == 0
+    assert list(oracle.candidate_set(10, 0, 0)) == list(range(10))
+    # N smaller than the sink count
+    assert list(oracle.static_set(3, 128, 0)) == [0, 1, 2]
+
+
+# ---------------------------------------------------------------- selection
+
+
+def _dominates(za, a, zb, b):
+    return za > zb or (za == zb and a < b)
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_topk_brute_force_with_ties(trial):
+    """For N <= 12 enumerate every k-subset of C; exactly one dominates all the rest
+    pairwise (higher z, ties to the lower position): it must be the oracle's Omega."""
+    rng = np.random.default_rng(trial)
+    N = int(rng.integers(1, 13))
+    n_sink = int(rng.integers(0, 3))
+    n_window = int(rng.integers(0, 3))
+    z = rng.integers(-3, 4, size=N).astype(np.float64) * 0.5   # many exact ties
+    C = oracle.candidate_set(N, n_sink, n_window)
+    for k in range(0, C.size + 2):
+        om = oracle.select_topk(z, C, k)
+        k_eff = min(k, C.size)
+        winners = []
+        for S in itertools.combinations(C.tolist(), k_eff):
+            rest = [b for b in C.tolist() if b not in S]
+            if all(_dominates(z[a], a, z[b], b) for a in S for b in rest):
+                winners.append(set(S))
+        assert len(winners) == 1
+        assert set(om.tolist()) == winners[0]
+        assert om.size == k_eff
+        assert not set(om.tolist()) & set(oracle.static_set(N, n_sink, n_window).tolist())
+
+
+def test_topk_order_is_by_score_then_position():
+    z = np.array([1.0, 3.0, 3.0, 2.0, 3.0, -1.0])
+    om = oracle.select_topk(z, np.arange(6), 4)
+    assert list(om) == [1, 2, 4, 3]
+
+
+def test_eq2_threshold_set_is_a_topk_set():
+    """Eq. (2): I_eps = {i : a_i > eps}.  Softmax is monotone, so I_eps is the top-|I_eps|
+    set of z (no static set, distinct scores)."""
+    rng = np.random.default_rng(7)
+    for _ in range(20):
+        z = rng.standard_normal(300) * 2.0
+        C = np.arange(300)
+        for eps in (1e-1, 1e-2, 3e-3, 1e-3, 1e-4):
+            I = oracle.threshold_set(z, eps)
+            om = oracle.select_topk(z, C, I.size)
+            assert set(I.tolist()) == set(om.tolist())
+
+
+def test_topk_permutation_equivariant():
+    rng = np.random.default_rng(3)
+    N, d = 200, 64
+    q = rand_bf16(d, rng=rng)
+    K = rand_bf16((N, d), rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    o1, om1, _ = oracle.decode_head(q, K, V, 20, 4, 8)
+    perm = np.arange(N)
+    mid = rng.permutation(np.arange(4, N - 8))
+    perm[4:N - 8] = mid
+    o2, om2, _ = oracle.decode_head(q, K[perm], V[perm], 20, 4, 8)
+    assert set(perm[om2].tolist()) == set(om1.tolist())
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+
+
+def test_planted_needles_are_retrieved():
+    """Needles whose score clears every other candidate by 1 must all be in Omega."""
+    rng = np.random.default_rng(11)
+    N, d, G = 4096, 128, 4
+    q = rand_bf16((G, d), rng=rng)
+    K = rand_bf16((N, d), rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    Kf = oracle.bf16_to_f64(K)
+    n_sink, n_window, k = 16, 64, 40
+    pos = rng.choice(np.arange(n_sink, N - n_window), size=8 * G, replace=False)
+    for h in range(G):
+        qf = oracle.bf16_to_f64(q[h])
+        top = np.max(Kf @ qf / math.sqrt(d))
+        lam = (top + 1.0) * math.sqrt(d) / np.linalg.norm(qf) * 1.05
+        for j in range(8):
+            K[pos[h * 8 + j]] = gen.needle_row(q[h], lam)
+    for h in range(G):
+        _, om, _ = oracle.decode_head(q[h], K, V, k, n_sink, n_window)
+        mine = set(pos[h * 8:(h + 1) * 8].tolist())
+        assert mine <= set(om.tolist())
+
+
+# ---------------------------------------------------------------- attention
+
+
+def _sdpa(z_q, K, V):
+    """torch scaled_dot_product_attention in float64: an independent softmax attention."""
+    q = torch.from_numpy(z_q)[None, None, None, :]
+    k = torch.from_numpy(K)[None, None]
+    v = torch.from_numpy(V)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v)[0, 0, 0].numpy()
+
+
+@pytest.mark.parametrize("N,d", [(1, 64), (7, 128), (640, 128), (4097, 64)])
+def test_dense_matches_torch_sdpa_fp64(N, d):
+    rng = np.random.default_rng(N)
+    q = rand_bf16(d, rng=rng)
+    K = rand_bf16((N, d), 2.0, rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    o = oracle.dense_head(q, K, V)
+    ref = _sdpa(oracle.bf16_to_f64(q), oracle.bf16_to_f64(K), oracle.bf16_to_f64(V))
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_union_matches_torch_sdpa_on_the_selected_rows():
+    rng = np.random.default_rng(5)
+    N, d = 3000, 128
+    q = rand_bf16(d, rng=rng)
+    K = rand_bf16((N, d), 2.0, rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    o, om, _ = oracle.decode_head(q, K, V, 100, 4, 64)
+    U = np.concatenate([oracle.static_set(N, 4, 64), om])
+    ref = _sdpa(oracle.bf16_to_f64(q), oracle.bf16_to_f64(K)[U], oracle.bf16_to_f64(V)[U])
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_two_keys_closed_form_logistic():
+    """Two keys: o = v2 + sigmoid(z1 - z2) (v1 - v2)."""
+    rng = np.random.default_rng(9)
+    for _ in range(20):
+        z = rng.standard_normal(2) * 3
+        V = rng.standard_normal((2, 16))
+        o = oracle.attend(z, V, np.array([0, 1]))
+        ref = V[1] + expit(z[0] - z[1]) * (V[0] - V[1])
+        np.testing.assert_allclose(o, ref, rtol=0, atol=1e-14)
+
+
+def test_attention_is_a_convex_combination():
+    rng = np.random.default_rng(10)
+    z = rng.standard_normal(50) * 4
+    U = np.arange(50)
+    V = np.tile(rng.standard_normal(8), (50, 1))
+    np.testing.assert_allclose(oracle.attend(z, V, U), V[0], rtol=0, atol=1e-14)
+    # affine equivariance in V
+    V = rng.standard_normal((50, 8))
+    A = rng.standard_normal((8, 8))
+    c = rng.standard_normal(8)
+    np.testing.assert_allclose(oracle.attend(z, V @ A + c, U), oracle.attend(z, V, U) @ A + c,
+                               rtol=0, atol=1e-12)
+    # shift of every score (equivalently one vector added to every key) changes nothing
+    np.testing.assert_allclose(oracle.attend(z + 123.25, V, U), oracle.attend(z, V, U),
+                               rtol=0, atol=1e-13)
+
+
+def test_identical_keys_give_the_mean_of_values():
+    rng = np.random.default_rng(12)
+    N, d = 33, 64
+    q = rand_bf16(d, rng=rng)
+    K = np.tile(rand_bf16(d, rng=rng), (N, 1))
+    V = rand_bf16((N, d), rng=rng)
+    o = oracle.dense_head(q, K, V)
+    np.testing.assert_allclose(o, oracle.bf16_to_f64(V).mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_one_dominant_key_limit():
+    """A score gap g bounds |o - v_top| by (N-1) e^{-g} max|v - v_top|."""
+    rng = np.random.default_rng(13)
+    z = rng.standard_normal(100)
+    z[17] = 40.0
+    V = rng.standard_normal((100, 4))
+    o = oracle.attend(z, V, np.arange(100))
+    gap = 40.0 - np.max(np.delete(z, 17))
+    bound = 99 * math.exp(-gap) * np.max(np.abs(V - V[17]))
+    assert np.max(np.abs(o - V[17])) <= bound
+
+
+# ---------------------------------------------------------------- merge (Eqs. 3-5)
+
+
+@pytest.mark.parametrize("parts", [2, 3, 7])
+def test_merge_of_disjoint_parts_equals_union_softmax(parts):
+    """The slides' identity: merging partial states of disjoint subsets with gamma_S is the
+    exact softmax over their union."""
+    rng = np.random.default_rng(parts)
+    z = rng.standard_normal(400) * 5 + 30     # large scores: needs the max subtraction
+    V = rng.standard_normal((400, 16))
+    U = rng.permutation(400)[:257]
+    cuts = np.sort(rng.choice(np.arange(1, U.size), size=parts - 1, replace=False))
+    subsets = np.split(U, cuts)
+    states = [oracle.partial_state(z, V, S) for S in subsets]
+    np.testing.assert_allclose(oracle.merge_partials(states), oracle.attend(z, V, U),
+                               rtol=0, atol=1e-12)
+
+
+def test_merge_of_static_and_dynamic_parts():
+    rng = np.random.default_rng(21)
+    N, d = 2000, 64
+    q = rand_bf16(d, rng=rng)
+    K = rand_bf16((N, d), 2.0, rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    o, om, z = oracle.decode_head(q, K, V, 50, 8, 32)
+    W = oracle.static_set(N, 8, 32)
+    Vf = oracle.bf16_to_f64(V)
+    merged = oracle.merge_partials([oracle.partial_state(z, Vf, W),
+                                    oracle.partial_state(z, Vf, om)])
+    np.testing.assert_allclose(merged, o, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- decode-step invariants
+
+
+@pytest.mark.parametrize("N,n_sink,n_window", [(500, 4, 64), (70, 64, 64), (33, 0, 0)])
+def test_k_at_least_candidates_equals_dense(N, n_sink, n_window):
+    """k >= |C| selects every candidate, so the step is full attention."""
+    rng = np.random.default_rng(N)
+    q = rand_bf16((1, 2, 64), rng=rng)
+    K = rand_bf16((1, 1, N, 64), 2.0, rng=rng)
+    V = rand_bf16((1, 1, N, 64), rng=rng)
+    out, _ = oracle.decode_step(q, K, V, N, n_sink, n_window)
+    dense = oracle.dense_decode(q, K, V)
+    np.testing.assert_allclose(out, dense, rtol=0, atol=1e-13)
+
+
+def test_k_zero_is_static_attention_only():
+    """k = 0: the step attends to W only (the sink-plus-window special case)."""
+    rng = np.random.default_rng(4)
+    N, d = 300, 64
+    q = rand_bf16(d, rng=rng)
+    K = rand_bf16((N, d), rng=rng)
+    V = rand_bf16((N, d), rng=rng)
+    o, om, _ = oracle.decode_head(q, K, V, 0, 4, 16)
+    assert om.size == 0
+    W = oracle.static_set(N, 4, 16)
+    ref = _sdpa(oracle.bf16_to_f64(q), oracle.bf16_to_f64(K)[W], oracle.bf16_to_f64(V)[W])
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-13)
+
+
+def test_gqa_heads_select_separately_but_share_kv():
+    rng = np.random.default_rng(8)
+    B, Hq, Hkv, N, d = 2, 4, 2, 256, 64
+    q = rand_bf16((B, Hq, d), rng=rng)
+    K = rand_bf16((B, Hkv, N, d), rng=rng)
+    V = rand_bf16((B, Hkv, N, d), rng=rng)
+    out, oms = oracle.decode_step(q, K, V, 10, 2, 4)
+    for b in range(B):
+        for h in range(Hq):
+            o, om, _ = oracle.decode_head(q[b, h], K[b, h // 2], V[b, h // 2], 10, 2, 4)
+            np.testing.assert_array_equal(out[b, h], o)
+            assert set(om.tolist()) == set(oms[b][h].tolist())
+    # heads of one group generally pick different sets
+    assert set(oms[0][0].tolist()) != set(oms[0][1].tolist())
+
+
+def test_empty_cache_is_an_error():
+    with pytest.raises(ValueError):
+        oracle.decode_head(np.zeros(64, np.uint16), np.zeros((0, 64), np.uint16),
+                           np.zeros((0, 64), np.uint16), 1, 0, 0)
+
+
+# ---------------------------------------------------------------- attention-mass statistic
+
+
+def test_topk_maximises_recovered_mass():
+    """Fig. 2's statistic: the top-k set recovers at least the mass of any k-subset."""
+    rng = np.random.default_rng(14)
+    z = rng.standard_normal(9) * 2
+    C = np.arange(9)
+    assert abs(oracle.attention_mass(z, C) - 1.0) < 1e-15
+    for k in range(1, 9):
+        best = oracle.attention_mass(z, oracle.select_topk(z, C, k))
+        for S in itertools.combinations(range(9), k):
+            assert oracle.attention_mass(z, np.array(S)) <= best + 1e-15
+
+
+# ---------------------------------------------------------------- sizes (Table 1)
+
+
+def test_kv_capacity_table1():
+    """Bytes per token of a Llama-3-8B cache (2 x 32 layers x 8 KV heads x 128 x 2 B) against
+    the printed Table 1 capacities, whose prompt labels count thousands of tokens
+    (1M = 1024 thousand) and whose unit is 2^30 bytes."""
+    per_token = 2 * 32 * 8 * 128 * 2
+    assert per_token == 131072
+    w = gen.workload("l8b_1m_32layer")
+    assert w.kv_bytes() == per_token * (1 << 20)
+    path = os.path.join(os.path.dirname(__file__), "golden", "kv_capacity_table1.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    thousands = {"128K": 128, "256K": 256, "512K": 512, "1M": 1024}
+    for label, gb in rows:
+        cap = thousands[label] * 1000 * per_token / 2**30
+        assert abs(cap - float(gb)) <= 0.06, (label, cap, gb)
