@@ -1,0 +1,152 @@
+/*
+ * ra.h -- C ABI of libra: exact top-k retrieval attention for one decode step on B200.
+ *
+ * The operation is the decode step of RetrievalAttention ("RetrievalAttention:
+ * Accelerating Long-Context LLM Inference via Vector Retrieval", arXiv 2409.10516v3 slides):
+ *
+ *   z_i = q_t k_i^T / sqrt(d)                          slide "Sparse attention renormalizes
+ *                                                       selected tokens", Eq. (1)
+ *   W   = first n_sink tokens + last n_window tokens    slide "The GPU keeps 640 fixed
+ *                                                       positions" (128 + 512 there)
+ *   C   = [0, N) \ W;  Omega = the k largest z in C     same slide: W and Omega disjoint,
+ *                                                       a fixed top-k budget, one index
+ *                                                       per query head under GQA
+ *   o   = softmax over U = W u Omega of z, times v      Eq. (2) renormalised over U, computed
+ *                                                       as split partial states merged by
+ *                                                       Eqs. (3)-(5) (slide "Two local softmax
+ *                                                       outputs need global weights")
+ *
+ * Retrieval here is exact (a full scan of K in HBM), not the slides' CPU-side ANN index.
+ *
+ * Conventions shared by every entry point:
+ *   - Ownership: the caller owns every buffer (device memory unless stated).  The library
+ *     allocates nothing and keeps no state between calls.
+ *   - Ordering: all work is enqueued on `stream` (a cudaStream_t, may be NULL for the legacy
+ *     default stream); no call synchronises the host.  Results are valid once the stream
+ *     reaches that point.
+ *   - Errors: arguments are validated on the host before anything is enqueued; on any error
+ *     status nothing has been enqueued, except RA_ERR_CUDA, which reports a failed launch.
+ *     No C++ exception crosses this interface.
+ *   - Layouts are dense row-major.  bf16 is IEEE bfloat16 (raw 16-bit patterns).
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef RA_H
+#define RA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t is `struct CUstream_st *`; declared here so the header needs no CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st *ra_stream_t;
+
+typedef enum {
+  RA_OK = 0,
+  RA_ERR_ARG = 1,        /* null or misaligned pointer, negative size or budget            */
+  RA_ERR_SHAPE = 2,      /* unsupported shape: d not 64/128, Hq % Hkv != 0, G > 8, N > cap */
+  RA_ERR_CAPACITY = 3,   /* append would exceed the cache capacity                         */
+  RA_ERR_WORKSPACE = 4,  /* ws is NULL or ws_bytes is below the required size              */
+  RA_ERR_CUDA = 5,       /* a CUDA call or kernel launch failed                            */
+  RA_ERR_EMPTY = 6       /* N == 0: nothing to attend to                                   */
+} ra_status;
+
+/*
+ * A per-layer KV cache resident in device memory.
+ *   K, V : bf16 [B, Hkv, cap, d], device, caller-owned.  Row (b, g, i) holds key/value i of
+ *          KV head g of sequence b.
+ *   B    : sequences (batch), >= 1.       Hkv : KV heads, >= 1.
+ *   d    : head dimension, 64 or 128.     cap : rows allocated per (b, g), >= N.
+ *   N    : tokens currently cached (host-side; ra_append_kv advances it).
+ */
+typedef struct {
+  void *K;
+  void *V;
+  int32_t B, Hkv, d, cap;
+  int64_t N;
+} ra_kv;
+
+/* Human-readable name of a status (static string). */
+const char *ra_status_str(ra_status s);
+
+/* Library version string (static). */
+const char *ra_version(void);
+
+/* Detail of the last RA_ERR_CUDA on the calling thread (static thread-local string). */
+const char *ra_last_error(void);
+
+/*
+ * Append T new tokens: K[b, g, N + t, :] = k_new[b, g, t, :] (same for V), then kv->N += T.
+ * Eq. (1)'s sum runs over j <= t, so the current token is appended before the decode step.
+ *   k_new, v_new : bf16 [B, Hkv, T, d], device.   T >= 0 (T == 0 is a no-op).
+ * Errors: RA_ERR_ARG (null kv/pointers, T < 0), RA_ERR_CAPACITY (N + T > cap; kv unchanged).
+ */
+ra_status ra_append_kv(ra_kv *kv, const void *k_new, const void *v_new, int32_t T,
+                       ra_stream_t stream);
+
+/*
+ * Workspace bytes that ra_decode_step (and its three phases) need for this shape.
+ * Returns 0 for an invalid shape.  The size grows with B*Hq*N (scores and candidates).
+ */
+size_t ra_decode_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, int32_t k,
+                                 int32_t n_sink, int32_t n_window);
+
+/*
+ * One decode step of exact top-k retrieval attention (all four parts above).
+ *   kv       : cache of this layer (N >= 1).
+ *   q        : bf16 [B, Hq, d], device.  Query head h reads KV head h / (Hq / Hkv).
+ *   Hq       : query heads; Hq % Hkv == 0 and G = Hq / Hkv <= 8.
+ *   k        : retrieval budget per query head (>= 0); clamped to |C|, so k >= N is legal
+ *              and makes the step full attention.
+ *   n_sink   : leading tokens always attended (>= 0).
+ *   n_window : trailing tokens always attended (>= 0).  The two ranges may overlap.
+ *   out      : float32 [B, Hq, d], device: the attention output.
+ *   idx      : int32 [B, Hq, k], device (may be NULL only when k == 0): Omega, the retrieved
+ *              positions of each query head, in unspecified order (a set); entries past
+ *              min(k, |C|) are -1.  Ties in score go to the lower position.
+ *   ws       : device workspace of at least ra_decode_workspace_bytes(...) bytes, 256-byte
+ *              aligned; contents need no initialisation and are clobbered.
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_EMPTY (N == 0), RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ * Calls that share one workspace must not overlap on the device.
+ */
+ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                         ra_stream_t stream);
+
+/*
+ * The three phases of ra_decode_step, exposed so a caller can time or interleave them.
+ * Run in this order with the same arguments and workspace, they are ra_decode_step.
+ *   ra_score_gqa   : z for every (query head, position) into ws, plus the per-head score
+ *                    histogram of the candidates (one pass over K per KV head).
+ *   ra_topk_select : Omega into idx from the scores in ws (radix select + bitonic finish).
+ *   ra_sparse_attn : out from the scores in ws, V rows of U = W u Omega, and the merge.
+ */
+ra_status ra_score_gqa(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
+                       int32_t n_window, void *ws, size_t ws_bytes, ra_stream_t stream);
+ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
+                         ra_stream_t stream);
+ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, const int32_t *idx, float *out, void *ws,
+                         size_t ws_bytes, ra_stream_t stream);
+
+/* Workspace bytes for ra_dense_decode (split partial states).  0 for an invalid shape. */
+size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d);
+
+/*
+ * Full attention over all N cached tokens (Eq. (1)): the dense flash-decode comparison path.
+ *   q : bf16 [B, Hq, d], device.   out : float32 [B, Hq, d], device.
+ *   ws: at least ra_dense_workspace_bytes(...) bytes, 256-byte aligned.
+ * Errors: as ra_decode_step.
+ */
+ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out, void *ws,
+                          size_t ws_bytes, ra_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RA_H */

@@ -1,0 +1,148 @@
+"""The C ABI without a GPU: the libraries load, export what the headers declare, and reject
+bad arguments on the host before anything is enqueued."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import top_retrieval_attention_b200 as ra  # noqa: E402
+from synth import device as sdev  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from top_retrieval_attention_b200 import build
+    build.build_all()
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b((?:ra|synth)_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared("ra.h")
+    assert set(names) == set(ra.EXPORTS)
+    L = ctypes.CDLL(ra.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    S = ctypes.CDLL(sdev.LIB_PATH)
+    for n in _declared("ra_synth.h"):
+        assert hasattr(S, n), n
+
+
+def test_library_needs_no_driver_at_load_time():
+    out = subprocess.run(["ldd", ra.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+    assert "libtorch" not in out
+
+
+def test_status_strings_and_version():
+    assert ra.ra_status_str(ra.RA_OK) == "RA_OK"
+    assert ra.ra_status_str(ra.RA_ERR_WORKSPACE) == "RA_ERR_WORKSPACE"
+    assert "sm_100a" in ra.ra_version()
+
+
+FAKE = 1 << 20   # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def _kv(B=1, Hkv=2, d=128, cap=100, N=50, K=FAKE, V=FAKE):
+    return ra.ra_kv(K, V, B, Hkv, d, cap, N)
+
+
+def test_workspace_bytes():
+    n = ra.ra_decode_workspace_bytes(1, 32, 131072, 128, 1310, 128, 512)
+    # scores (32 x 131072 fp32) + histograms + counters + candidates + partial states
+    assert n >= 32 * 131072 * 4 * 2
+    assert n % 256 == 0
+    assert ra.ra_decode_workspace_bytes(1, 32, 131072, 96, 10, 0, 0) == 0     # d
+    assert ra.ra_decode_workspace_bytes(0, 32, 131072, 128, 10, 0, 0) == 0    # B
+    assert ra.ra_decode_workspace_bytes(1, 32, 131072, 128, -1, 0, 0) == 0    # k
+    assert ra.ra_dense_workspace_bytes(1, 32, 131072, 128) > 0
+    assert ra.ra_dense_workspace_bytes(1, 32, 131072, 80) == 0
+
+
+@pytest.mark.parametrize("mut,status", [
+    (dict(K=0), ra.RA_ERR_ARG),
+    (dict(V=FAKE + 8), ra.RA_ERR_ARG),
+    (dict(d=96), ra.RA_ERR_SHAPE),
+    (dict(N=101), ra.RA_ERR_SHAPE),
+    (dict(B=0), ra.RA_ERR_ARG),
+    (dict(N=0), ra.RA_ERR_EMPTY),
+])
+def test_decode_rejects_bad_cache(mut, status):
+    kv = _kv(**mut)
+    ws_bytes = 1 << 30
+    s = ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, FAKE, FAKE, FAKE, ws_bytes, None)
+    assert s == status
+
+
+def test_decode_rejects_bad_arguments():
+    kv = _kv()
+    big = 1 << 30
+    assert ra.ra_decode_step(kv, FAKE, 3, 10, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_SHAPE
+    assert ra.ra_decode_step(kv, FAKE, 18, 10, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_SHAPE
+    assert ra.ra_decode_step(kv, FAKE, 4, -1, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, -4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step(kv, 0, 4, 10, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, 0, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, FAKE, 0, FAKE, big, None) == ra.RA_ERR_ARG
+    # workspace: null, misaligned, too small
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, FAKE, FAKE, 0, big, None) == ra.RA_ERR_WORKSPACE
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, FAKE, FAKE, FAKE + 16, big, None) == ra.RA_ERR_WORKSPACE
+    need = ra.ra_decode_workspace_bytes(1, 4, 50, 128, 10, 4, 8)
+    assert ra.ra_decode_step(kv, FAKE, 4, 10, 4, 8, FAKE, FAKE, FAKE, need - 1, None) == ra.RA_ERR_WORKSPACE
+    # empty selected union: no static set and k = 0
+    assert ra.ra_decode_step(kv, FAKE, 4, 0, 0, 0, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_EMPTY
+
+
+def test_phases_validate_like_the_step():
+    kv = _kv()
+    big = 1 << 30
+    assert ra.ra_score_gqa(kv, 0, 4, 10, 4, 8, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_topk_select(kv, 4, 10, 4, 8, 0, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_sparse_attn(kv, 4, 10, 4, 8, FAKE, 0, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_sparse_attn(kv, 4, 10, 4, 8, FAKE, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
+
+
+def test_dense_rejects_bad_arguments():
+    kv = _kv()
+    big = 1 << 30
+    assert ra.ra_dense_decode(kv, FAKE, 3, FAKE, FAKE, big, None) == ra.RA_ERR_SHAPE
+    assert ra.ra_dense_decode(_kv(N=0), FAKE, 4, FAKE, FAKE, big, None) == ra.RA_ERR_EMPTY
+    assert ra.ra_dense_decode(kv, FAKE, 4, FAKE, FAKE, 16, None) == ra.RA_ERR_WORKSPACE
+
+
+def test_append_capacity_and_arguments():
+    kv = _kv(cap=100, N=98)
+    assert ra.ra_append_kv(kv, FAKE, FAKE, 3, None) == ra.RA_ERR_CAPACITY
+    assert kv.N == 98
+    assert ra.ra_append_kv(kv, FAKE, FAKE, -1, None) == ra.RA_ERR_ARG
+    assert ra.ra_append_kv(kv, 0, FAKE, 1, None) == ra.RA_ERR_ARG
+    assert ra.ra_append_kv(kv, FAKE, FAKE, 0, None) == ra.RA_OK
+    assert kv.N == 98
+
+
+def test_synth_constants_match_host_generator():
+    from synth import gen
+    a, b = sdev.constants()
+    assert a == gen.IH_SCALE == math.sqrt(3) / 65536
+    assert b == gen.OFF_STD == math.sqrt(2)
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "top_retrieval_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
+                assert "oracle/" not in text, f

@@ -1,0 +1,37 @@
+// Append T new tokens to a layer's KV cache: K[b, g, N + t, :] = k_new[b, g, t, :], same for
+// V.  The decode step attends over j <= t including the current token (RetrievalAttention
+// slides, Eq. (1)), so a step appends before it scores.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ra {
+
+__global__ void __launch_bounds__(256) append_kv_kernel(const AppendParams p) {
+  // one 16-byte unit per thread: units per row = d / 8
+  const int upr = p.d / 8;
+  const long long units = static_cast<long long>(p.B) * p.Hkv * p.T * upr;
+  for (long long u = blockIdx.x * 256LL + threadIdx.x; u < 2 * units;
+       u += static_cast<long long>(gridDim.x) * 256) {
+    const bool is_v = u >= units;
+    const long long w = is_v ? u - units : u;
+    const int c = static_cast<int>(w % upr);
+    const long long rt = w / upr;               // (b*Hkv + g) * T + t
+    const long long t = rt % p.T;
+    const long long bg = rt / p.T;
+    const uint4 *src = reinterpret_cast<const uint4 *>(is_v ? p.v_new : p.k_new) + w;
+    __nv_bfloat16 *dst_base = is_v ? p.V : p.K;
+    uint4 *dst = reinterpret_cast<uint4 *>(dst_base + (bg * p.cap + p.N + t) * p.d) + c;
+    *dst = __ldg(src);
+  }
+}
+
+cudaError_t launch_append(const AppendParams &p, cudaStream_t s) {
+  const long long units = 2LL * p.B * p.Hkv * p.T * (p.d / 8);
+  long long blocks = (units + 255) / 256;
+  if (blocks > 4LL * num_sms()) blocks = 4LL * num_sms();
+  if (blocks < 1) blocks = 1;
+  append_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace ra

@@ -1,0 +1,112 @@
+// Shared device helpers for libra (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ra {
+
+constexpr int kHistBits = 11;                 // first radix digit: top 11 bits of the key
+constexpr int kHistBins = 1 << kHistBits;     // 2048 bins per query head
+constexpr int kMaxGroup = 8;                  // query heads per KV head (one n8 MMA tile)
+constexpr int kMetaWords = 8;                 // per-row counters in the workspace
+
+// per-row counters (uint32) in the workspace's meta block
+enum MetaSlot { kSelCount = 0, kCandCount = 1, kThreshBin = 2, kAbove = 3, kDone = 4,
+                kDenseDone = 5, kError = 6 };
+
+// ------------------------------------------------------------------ order-preserving keys
+
+// Maps a float to a uint32 whose unsigned order equals the float order (-0 sorts below +0;
+// scores are canonicalised so that zero is always +0).
+__device__ __forceinline__ uint32_t order_key(float z) {
+  uint32_t u = __float_as_uint(z);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float canon_zero(float z) { return z == 0.0f ? 0.0f : z; }
+
+// ------------------------------------------------------------------ async copies
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global -> shared copy; src_bytes == 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// ------------------------------------------------------------------ tensor-core fragments
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                            uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Swizzled byte offset of 16-byte chunk `c` of row `r` in a tile whose rows are `row_bytes`
+// long (128 or 256): the low three chunk bits are XORed with the row's low three bits, so
+// eight consecutive rows at one logical chunk hit eight distinct bank groups.
+__device__ __forceinline__ uint32_t swz(int r, int c, int row_bytes) {
+  return static_cast<uint32_t>(r * row_bytes + ((c ^ (r & 7)) << 4));
+}
+
+// ------------------------------------------------------------------ bf16 pairs
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ------------------------------------------------------------------ warp reductions
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Warp-aggregated append: every lane with `pred` gets a distinct slot from *counter.
+__device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t *counter, bool &ok) {
+  const uint32_t mask = __ballot_sync(0xffffffffu, pred);
+  ok = pred;
+  if (mask == 0) return 0;
+  const int leader = __ffs(mask) - 1;
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(mask)));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  return base + __popc(mask & lanemask_lt());
+}
+
+}  // namespace ra

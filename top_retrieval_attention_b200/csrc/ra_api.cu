@@ -1,0 +1,325 @@
+// C ABI of libra: argument validation, workspace layout and kernel sequencing.
+// Every check runs on the host before anything is enqueued; the library allocates nothing.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <algorithm>
+
+#include "../../include/ra.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ra {
+
+static thread_local char g_last_error[256] = "";
+
+static ra_status cuda_fail(cudaError_t e, const char *where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
+           static_cast<int>(e));
+  return RA_ERR_CUDA;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+static constexpr size_t kAlign = 256;
+static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+static long long round4(long long x) { return (x + 3) / 4 * 4; }
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Derived sizes of one decode step (positions follow the slide "The GPU keeps 640 fixed
+// positions": W = [0, s1) u [w0, N), candidates C = [s1, w0)).
+struct Step {
+  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit;
+  long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC;
+  size_t off_S, off_hist, off_meta, off_cand, off_part, total;
+};
+
+static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
+                            int n_window, Step &st) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 0 || k < 0 || n_sink < 0 || n_window < 0) return RA_ERR_ARG;
+  if (d != 64 && d != 128) return RA_ERR_SHAPE;
+  if (Hq % Hkv != 0 || Hq / Hkv > kMaxGroup) return RA_ERR_SHAPE;
+  if (N >= (1LL << 31) - 1) return RA_ERR_SHAPE;
+  if (static_cast<long long>(B) * Hq > 65535) return RA_ERR_SHAPE;
+  st.B = B; st.Hq = Hq; st.Hkv = Hkv; st.G = Hq / Hkv; st.d = d; st.k = k;
+  st.n_sink = n_sink; st.n_window = n_window; st.N = N;
+  st.R = B * Hq;
+  st.s1 = std::min<long long>(n_sink, N);
+  st.w0 = std::max<long long>(st.s1, N - n_window);
+  st.nW = st.s1 + (N - st.w0);
+  st.nC = st.w0 - st.s1;
+  st.k_eff = std::min<long long>(k, st.nC);
+  st.ldS = round4(std::max<long long>(N, 1));
+  st.ldC = round4(std::max<long long>(st.nC, 1));
+  const long long nU = st.nW + st.k_eff;
+  st.nsplit = static_cast<int>(std::max<long long>(1, (nU + kAttnChunk - 1) / kAttnChunk));
+  size_t off = 0;
+  st.off_S = off;    off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
+  st.off_hist = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
+  st.off_meta = off; off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
+  st.off_cand = off; off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 4);
+  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit * (d + 2) * 4);
+  st.total = off;
+  return RA_OK;
+}
+
+static ra_status check_kv(const ra_kv *kv) {
+  if (!kv || !kv->K || !kv->V) return RA_ERR_ARG;
+  if (!aligned16(kv->K) || !aligned16(kv->V)) return RA_ERR_ARG;
+  if (kv->B < 1 || kv->Hkv < 1 || kv->cap < 0 || kv->N < 0) return RA_ERR_ARG;
+  if (kv->d != 64 && kv->d != 128) return RA_ERR_SHAPE;
+  if (kv->N > kv->cap) return RA_ERR_SHAPE;
+  return RA_OK;
+}
+
+// Validation common to the decode step and its phases.
+static ra_status plan_step(const ra_kv *kv, int Hq, int k, int n_sink, int n_window, void *ws,
+                           size_t ws_bytes, Step &st) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  s = plan_shape(kv->B, Hq, kv->Hkv, kv->N, kv->d, k, n_sink, n_window, st);
+  if (s != RA_OK) return s;
+  st.cap = kv->cap;
+  if (kv->N == 0 || st.nW + st.k_eff == 0) return RA_ERR_EMPTY;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return RA_ERR_WORKSPACE;
+  if (ws_bytes < st.total) return RA_ERR_WORKSPACE;
+  return RA_OK;
+}
+
+static uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
+
+static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void *ws,
+                           cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(at(ws, st.off_hist), 0, st.off_cand - st.off_hist, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  ScoreParams p{};
+  p.K = static_cast<const __nv_bfloat16 *>(kv->K);
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.S = reinterpret_cast<float *>(at(ws, st.off_S));
+  p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
+  p.N = st.N; p.cap = st.cap; p.ldS = st.ldS;
+  p.cand_lo = st.s1; p.cand_hi = st.w0;
+  p.tiles_per_head = (st.N + kScoreTile - 1) / kScoreTile;
+  p.total_tiles = p.tiles_per_head * st.B * st.Hkv;
+  p.B = st.B; p.Hkv = st.Hkv; p.G = st.G; p.Hq = st.Hq;
+  p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
+  p.do_hist = st.k_eff > 0 && st.k_eff < st.nC;
+  e = launch_score(p, st.d, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
+}
+
+static ra_status run_topk(const Step &st, int32_t *idx, void *ws, cudaStream_t stream) {
+  if (st.k == 0) return RA_OK;
+  TopkParams p{};
+  p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
+  p.hist = reinterpret_cast<const uint32_t *>(at(ws, st.off_hist));
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
+  p.cand = reinterpret_cast<uint32_t *>(at(ws, st.off_cand));
+  p.idx = idx;
+  p.ldS = st.ldS; p.ldC = st.ldC; p.N = st.N;
+  p.cand_lo = st.s1; p.cand_hi = st.w0; p.nC = st.nC; p.k_eff = st.k_eff;
+  p.chunk = kCollectChunk;
+  p.k = st.k; p.R = st.R;
+  cudaError_t e = launch_topk(p, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "topk");
+}
+
+static ra_status run_attn(const ra_kv *kv, const Step &st, const int32_t *idx, float *out,
+                          void *ws, cudaStream_t stream) {
+  AttnParams p{};
+  p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
+  p.V = static_cast<const __nv_bfloat16 *>(kv->V);
+  p.idx = idx;
+  p.part = reinterpret_cast<float *>(at(ws, st.off_part));
+  p.out = out;
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
+  p.ldS = st.ldS; p.cap = st.cap; p.N = st.N;
+  p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.k_eff = st.k_eff;
+  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.nsplit = st.nsplit; p.R = st.R;
+  cudaError_t e = launch_sparse_attn(p, st.d, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "sparse_attn");
+}
+
+// Dense flash-decode split plan: as many splits per KV head as keep the grid close to a
+// whole number of waves of one CTA per SM, at most kDenseMaxSplit.
+static constexpr int kDenseMaxSplit = 256;
+
+static int dense_nsplit_cap(long long N) {
+  const long long tiles = std::max<long long>(1, (N + kDenseTile - 1) / kDenseTile);
+  return static_cast<int>(std::min<long long>(tiles, kDenseMaxSplit));
+}
+
+static size_t dense_bytes(int R, int nsplit_cap, int d, size_t *off_meta) {
+  size_t off = align_up(static_cast<size_t>(R) * nsplit_cap * (d + 2) * 4);
+  if (off_meta) *off_meta = off;
+  return align_up(off + static_cast<size_t>(R) * kMetaWords * 4);
+}
+
+}  // namespace ra
+
+using namespace ra;
+
+extern "C" {
+
+const char *ra_status_str(ra_status s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_ARG: return "RA_ERR_ARG";
+    case RA_ERR_SHAPE: return "RA_ERR_SHAPE";
+    case RA_ERR_CAPACITY: return "RA_ERR_CAPACITY";
+    case RA_ERR_WORKSPACE: return "RA_ERR_WORKSPACE";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA";
+    case RA_ERR_EMPTY: return "RA_ERR_EMPTY";
+  }
+  return "RA_ERR_UNKNOWN";
+}
+
+const char *ra_version(void) { return "libra 0.1 (sm_100a)"; }
+
+const char *ra_last_error(void) { return g_last_error; }
+
+ra_status ra_append_kv(ra_kv *kv, const void *k_new, const void *v_new, int32_t T,
+                       ra_stream_t stream) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (T < 0) return RA_ERR_ARG;
+  if (T == 0) return RA_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return RA_ERR_ARG;
+  if (kv->N + T > kv->cap) return RA_ERR_CAPACITY;
+  AppendParams p{};
+  p.K = static_cast<__nv_bfloat16 *>(kv->K);
+  p.V = static_cast<__nv_bfloat16 *>(kv->V);
+  p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+  p.cap = kv->cap; p.N = kv->N; p.B = kv->B; p.Hkv = kv->Hkv; p.d = kv->d; p.T = T;
+  cudaError_t e = launch_append(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append");
+  kv->N += T;
+  return RA_OK;
+}
+
+size_t ra_decode_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, int32_t k,
+                                 int32_t n_sink, int32_t n_window) {
+  Step st{};
+  // the layout does not depend on the KV head count: plan it with one query head per KV head
+  if (plan_shape(B, Hq, Hq, N, d, k, n_sink, n_window, st) != RA_OK) return 0;
+  return st.total;
+}
+
+ra_status ra_score_gqa(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
+                       int32_t n_window, void *ws, size_t ws_bytes, ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q)) return RA_ERR_ARG;
+  return run_score(kv, q, st, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
+                         ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  return run_topk(st, idx, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, const int32_t *idx, float *out, void *ws,
+                         size_t ws_bytes, ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if ((k > 0 && (!idx || !aligned16(idx))) || !out || !aligned16(out)) return RA_ERR_ARG;
+  return run_attn(kv, st, idx, out, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
+                         int32_t n_window, float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                         ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  s = run_score(kv, q, st, ws, cs);
+  if (s != RA_OK) return s;
+  s = run_topk(st, idx, ws, cs);
+  if (s != RA_OK) return s;
+  return run_attn(kv, st, idx, out, ws, cs);
+}
+
+size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d) {
+  if (B < 1 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
+  if (N >= (1LL << 31) - 1) return 0;
+  return dense_bytes(B * Hq, dense_nsplit_cap(N), d, nullptr);
+}
+
+ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out, void *ws,
+                          size_t ws_bytes, ra_stream_t stream) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (Hq < 1 || Hq % kv->Hkv != 0 || Hq / kv->Hkv > kMaxGroup) return RA_ERR_SHAPE;
+  if (kv->N >= (1LL << 31) - 1 || static_cast<long long>(kv->B) * Hq > 65535) return RA_ERR_SHAPE;
+  if (kv->N == 0) return RA_ERR_EMPTY;
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  const int R = kv->B * Hq;
+  const int cap_split = dense_nsplit_cap(kv->N);
+  size_t off_meta = 0;
+  const size_t need = dense_bytes(R, cap_split, kv->d, &off_meta);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < need)
+    return RA_ERR_WORKSPACE;
+
+  // splits: the smallest whole number of waves (one CTA per SM) that is >= 95% full
+  const long long tiles = (kv->N + kDenseTile - 1) / kDenseTile;
+  const int BH = kv->B * kv->Hkv;
+  const int sms = num_sms();
+  int best = 1;
+  double best_eff = -1.0;
+  for (int w = 1; w <= 8; ++w) {
+    int ns = std::max(1, (sms * w) / BH);
+    ns = static_cast<int>(std::min<long long>(ns, std::min<long long>(tiles, cap_split)));
+    const long long ctas = static_cast<long long>(BH) * ns;
+    const long long waves = (ctas + sms - 1) / sms;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+    if (eff >= 0.95) break;
+  }
+  const long long kps = (tiles + best - 1) / best * kDenseTile;
+  const int nsplit = static_cast<int>((kv->N + kps - 1) / kps);
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(at(ws, off_meta), 0, static_cast<size_t>(R) * kMetaWords * 4, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  DenseParams p{};
+  p.K = static_cast<const __nv_bfloat16 *>(kv->K);
+  p.V = static_cast<const __nv_bfloat16 *>(kv->V);
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.part = static_cast<float *>(ws);
+  p.out = out;
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, off_meta));
+  p.N = kv->N; p.cap = kv->cap; p.keys_per_split = kps;
+  p.B = kv->B; p.Hkv = kv->Hkv; p.G = Hq / kv->Hkv; p.Hq = Hq; p.nsplit = nsplit;
+  p.scale = 1.0f / sqrtf(static_cast<float>(kv->d));
+  e = launch_dense(p, kv->d, cs);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "dense_decode");
+}
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+"""ctypes binding of libra (include/ra.h): argument marshalling only.
+
+The raw entry points keep the C names (``ra_decode_step`` ...) and take integer device
+pointers; the small helpers below them (``KVCache``, ``decode_step`` ...) allocate outputs and
+workspaces with torch and pass tensor pointers and the current torch stream.  Every step of the
+computation runs in libra's CUDA kernels; there is no other implementation behind this module.
+Loading fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import c_char_p, c_int32, c_int64, c_size_t, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libra.so")
+
+RA_OK, RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_CAPACITY, RA_ERR_WORKSPACE, RA_ERR_CUDA, RA_ERR_EMPTY = range(7)
+
+#: every symbol include/ra.h declares
+EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
+           "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
+           "ra_sparse_attn", "ra_dense_workspace_bytes", "ra_dense_decode")
+
+
+class ra_kv(ctypes.Structure):
+    _fields_ = [("K", c_void_p), ("V", c_void_p), ("B", c_int32), ("Hkv", c_int32),
+                ("d", c_int32), ("cap", c_int32), ("N", c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libra.so is not built ({LIB_PATH}); run "
+                               "`python -m top_retrieval_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(ra_kv)
+        sig = {
+            "ra_status_str": (c_char_p, [c_int32]),
+            "ra_version": (c_char_p, []),
+            "ra_last_error": (c_char_p, []),
+            "ra_append_kv": (c_int32, [P, c_void_p, c_void_p, c_int32, c_void_p]),
+            "ra_decode_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32, c_int32,
+                                                     c_int32, c_int32]),
+            "ra_decode_step": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32,
+                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+            "ra_score_gqa": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32, c_void_p,
+                                       c_size_t, c_void_p]),
+            "ra_topk_select": (c_int32, [P, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                         c_size_t, c_void_p]),
+            "ra_sparse_attn": (c_int32, [P, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                         c_void_p, c_size_t, c_void_p]),
+            "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
+            "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
+                                          c_void_p]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------ raw entry points
+
+
+def ra_status_str(s: int) -> str:
+    return lib().ra_status_str(s).decode()
+
+
+def ra_version() -> str:
+    return lib().ra_version().decode()
+
+
+def ra_last_error() -> str:
+    return lib().ra_last_error().decode()
+
+
+def ra_append_kv(kv, k_new, v_new, T, stream):
+    return lib().ra_append_kv(ctypes.byref(kv), k_new, v_new, T, stream)
+
+
+def ra_decode_workspace_bytes(B, Hq, N, d, k, n_sink, n_window) -> int:
+    return lib().ra_decode_workspace_bytes(B, Hq, N, d, k, n_sink, n_window)
+
+
+def ra_decode_step(kv, q, Hq, k, n_sink, n_window, out, idx, ws, ws_bytes, stream):
+    return lib().ra_decode_step(ctypes.byref(kv), q, Hq, k, n_sink, n_window, out, idx, ws,
+                                ws_bytes, stream)
+
+
+def ra_score_gqa(kv, q, Hq, k, n_sink, n_window, ws, ws_bytes, stream):
+    return lib().ra_score_gqa(ctypes.byref(kv), q, Hq, k, n_sink, n_window, ws, ws_bytes, stream)
+
+
+def ra_topk_select(kv, Hq, k, n_sink, n_window, idx, ws, ws_bytes, stream):
+    return lib().ra_topk_select(ctypes.byref(kv), Hq, k, n_sink, n_window, idx, ws, ws_bytes,
+                                stream)
+
+
+def ra_sparse_attn(kv, Hq, k, n_sink, n_window, idx, out, ws, ws_bytes, stream):
+    return lib().ra_sparse_attn(ctypes.byref(kv), Hq, k, n_sink, n_window, idx, out, ws,
+                                ws_bytes, stream)
+
+
+def ra_dense_workspace_bytes(B, Hq, N, d) -> int:
+    return lib().ra_dense_workspace_bytes(B, Hq, N, d)
+
+
+def ra_dense_decode(kv, q, Hq, out, ws, ws_bytes, stream):
+    return lib().ra_dense_decode(ctypes.byref(kv), q, Hq, out, ws, ws_bytes, stream)
+
+
+# ------------------------------------------------------------------ torch-facing helpers
+
+
+class RaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {ra_status_str(status)}"
+        if status == RA_ERR_CUDA:
+            msg += f" ({ra_last_error()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def check(status: int, where: str) -> None:
+    if status != RA_OK:
+        raise RaError(status, where)
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return c_void_p(s.cuda_stream)
+
+
+class KVCache:
+    """A layer's K and V caches ([B, Hkv, cap, d] bf16 torch tensors) and their ra_kv."""
+
+    def __init__(self, B: int, Hkv: int, d: int, cap: int, device="cuda", K=None, V=None):
+        import torch
+        shape = (B, Hkv, cap, d)
+        self.K = torch.empty(shape, dtype=torch.bfloat16, device=device) if K is None else K
+        self.V = torch.empty(shape, dtype=torch.bfloat16, device=device) if V is None else V
+        assert tuple(self.K.shape) == shape and self.K.is_contiguous() and self.V.is_contiguous()
+        self.kv = ra_kv(self.K.data_ptr(), self.V.data_ptr(), B, Hkv, d, cap, 0)
+
+    @property
+    def N(self) -> int:
+        return int(self.kv.N)
+
+    @N.setter
+    def N(self, n: int) -> None:
+        self.kv.N = n
+
+    B = property(lambda self: self.kv.B)
+    Hkv = property(lambda self: self.kv.Hkv)
+    d = property(lambda self: self.kv.d)
+    cap = property(lambda self: self.kv.cap)
+
+
+def append_kv(cache: KVCache, k_new, v_new, stream=None) -> None:
+    T = int(k_new.shape[2])
+    check(ra_append_kv(cache.kv, k_new.data_ptr(), v_new.data_ptr(), T, _stream(stream)),
+          "ra_append_kv")
+
+
+def decode_workspace(cache: KVCache, Hq: int, k: int, n_sink: int, n_window: int):
+    import torch
+    n = ra_decode_workspace_bytes(cache.B, Hq, cache.N, cache.d, k, n_sink, n_window)
+    if n == 0:
+        raise RaError(RA_ERR_SHAPE, "ra_decode_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=cache.K.device)
+
+
+def decode_step(cache: KVCache, q, k: int, n_sink: int, n_window: int, out=None, idx=None,
+                ws=None, stream=None):
+    """Exact top-k retrieval attention for one decode step.  Returns (out fp32, idx int32)."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = decode_workspace(cache, Hq, k, n_sink, n_window)
+    check(ra_decode_step(cache.kv, q.data_ptr(), Hq, k, n_sink, n_window, out.data_ptr(),
+                         idx.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+          "ra_decode_step")
+    return out, idx[..., :k]
+
+
+def dense_workspace(cache: KVCache, Hq: int):
+    import torch
+    n = ra_dense_workspace_bytes(cache.B, Hq, cache.N, cache.d)
+    if n == 0:
+        raise RaError(RA_ERR_SHAPE, "ra_dense_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=cache.K.device)
+
+
+def dense_decode(cache: KVCache, q, out=None, ws=None, stream=None):
+    """Full attention over all N cached tokens.  Returns out fp32 [B, Hq, d]."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = dense_workspace(cache, Hq)
+    check(ra_dense_decode(cache.kv, q.data_ptr(), Hq, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                          _stream(stream)), "ra_dense_decode")
+    return out
