@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of exact top-k retrieval attention on B200.
+
+A step is one pass of the whole hot path for every layer of the workload: append the new
+token's K/V row (ra_append_kv), score all positions (ra_score_gqa), select the top-k per query
+head (ra_topk_select), and attend over sinks + window + top-k (ra_sparse_attn).  The cache
+holds N-1 tokens; each step appends the N-th and decodes over N, then the next step re-appends
+into the same slot, so every step has identical work.  Each step uses its own query.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Rank 0 prints one JSON line.  `value` is whole-job decode steps/s with the caches resident in
+HBM; `e2e` is the same metric through the public Python API with the step's inputs (query,
+new K/V row) copied from pinned host memory and the outputs (out, idx) copied back and waited
+for inside the timed region; `roofline` is the score kernel (the K scan, the dominant kernel)
+against the measured HBM copy bandwidth; `cpu_baseline` is the fp64 oracle on a bounded sample
+timed on the host cores.  `--impl reference` times only the oracle (the reference arm).
+Under torchrun each rank runs an independent replica (the step does not shard across GPUs).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode steps/s & K-scan HBM GB/s (frac of peak) at 128K–1M ctx, top-k sparse attn"
+DEFAULT_WORKLOAD = "l8b_128k_k1pct"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one score-kernel launch, from an ncu capture,
+# keyed by the sha256 of the score kernel's sources it was taken on (so a changed kernel
+# reports null until it is captured again).  Values are per launch of the named workload.
+TRAFFIC = {}
+
+
+def score_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("score.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "top_retrieval_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default: ~1 s of work)")
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def dist_init(world, use_cuda):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group("nccl" if use_cuda else "gloo",
+                            timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks during timing
+
+
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * max(mx or [1])] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            v = float(json.load(fh)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline legs)
+
+
+def _blas_threads() -> int:
+    from threadpoolctl import threadpool_info
+    cores = 1
+    for info in threadpool_info():
+        if info.get("user_api") == "blas":
+            cores = max(cores, int(info.get("num_threads", 1)))
+    return cores
+
+
+def _oracle_group_seconds(w, qh, K, V, k_s) -> float:
+    """Wall time of the oracle's decode of the G query heads that share KV head 0."""
+    import oracle
+    t0 = time.perf_counter()
+    for h in range(w.G):
+        oracle.decode_head(qh[0, h], K, V, k_s, w.n_sink, w.n_window)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(w, seconds: float):
+    """The fp64 oracle on one KV head group (G query heads) of layer 0 at full N, repeated for
+    about `seconds`; returns (steps/s, cores, description) scaled to one whole step."""
+    from synth import gen
+    qh = gen.gen_q(w.seed, w.B, w.Hq, w.d)
+    K, V = gen.host_head(w, 0, 0, 0, w.N)
+    times = []
+    t_end = time.perf_counter() + seconds
+    while not times or time.perf_counter() < t_end:
+        times.append(_oracle_group_seconds(w, qh, K, V, w.k))
+    scale = w.Hkv * w.B * w.layers
+    step_s = statistics.median(times) * scale
+    desc = (f"oracle decode of the {w.G} query heads of KV head 0 (layer 0, b 0) over all "
+            f"{w.N} keys, median of {len(times)} runs, x{scale} for the whole step")
+    return 1.0 / step_s, _blas_threads(), desc
+
+
+def run_reference(args, w, rank, world):
+    """The reference arm: the oracle as it stands, on the host cores.  Each step times the
+    oracle on a bounded sample of the workload (the G query heads of one KV head over a
+    contiguous slice of the keys, with k scaled to the slice), sized so the whole run takes
+    about 100 s, and scales it to one whole step (the oracle's cost is linear in N apart from
+    the sort's log factor, so this slightly flatters the CPU at large N)."""
+    if rank != 0:
+        return
+    from synth import gen
+    steps = args.steps if args.steps is not None else 5
+    warm = args.warmup
+    budget = max(0.005, 100.0 / max(1, steps + warm))
+    qh = gen.gen_q(w.seed, w.B, w.Hq, w.d)
+    n_cal = min(w.N, 8192)
+    K, V = gen.host_head(w, 0, 0, 0, n_cal)
+    t_cal = min(_oracle_group_seconds(w, qh, K, V, max(1, w.k * n_cal // w.N)) for _ in range(3))
+    n_keys = int(min(w.N, max(1024, n_cal * budget / max(t_cal, 1e-9))))
+    K, V = gen.host_head(w, 0, 0, 0, n_keys)
+    k_s = w.k if n_keys == w.N else max(1, int(round(w.k * n_keys / w.N)))
+    scale = (w.N / n_keys) * w.Hkv * w.B * w.layers
+    vals = []
+    for i in range(warm + steps):
+        t = _oracle_group_seconds(w, qh, K, V, k_s)
+        if i >= warm:
+            vals.append(1.0 / (t * scale))
+    value = statistics.median(vals)
+    desc = (f"per step: oracle decode of the {w.G} query heads of KV head 0 (layer 0, b 0) over "
+            f"keys [0, {n_keys}) of {w.N} with k={k_s}, scaled x{scale:.1f} to one whole step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s",
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": 1000.0 / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": _blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N,
+            "k": w.k, "n_sink": w.n_sink, "n_window": w.n_window, "layers": w.layers,
+            "needles_per_kv_head": w.n_needle, "parallelism": "replicas",
+            "l2": "inputs larger than L2 (whole K scanned every step); a distinct query per step"}
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def run_ours(args, w, rank, local_rank, world, dist):
+    import ctypes
+
+    import torch
+
+    import top_retrieval_attention_b200 as ra
+    from synth import device as sdev
+    from synth import gen
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    ra.lib()
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    L, B, Hq, Hkv, d, N, k = w.layers, w.B, w.Hq, w.Hkv, w.d, w.N, w.k
+
+    # caches: rows [0, N) filled by the generator; the last row is the token each step appends
+    caches, knew, vnew = [], [], []
+    for layer in range(L):
+        c = ra.KVCache(B, Hkv, d, N, device=dev)
+        sdev.device_layer(w, layer, c.K, c.V)
+        knew.append(c.K[:, :, N - 1:N].clone())
+        vnew.append(c.V[:, :, N - 1:N].clone())
+        c.N = N - 1
+        caches.append(c)
+    P = 16
+    qpool = torch.empty((P, L, B, Hq, d), dtype=torch.bfloat16, device=dev)
+    for s in range(P):
+        for layer in range(L):
+            sdev.fill_q(qpool[s, layer], w.seed + 7919 * s + 104729 * layer)
+    ws_bytes = ra.ra_decode_workspace_bytes(B, Hq, N, d, k, w.n_sink, w.n_window)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
+    idxs = [torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=dev) for _ in range(L)]
+    torch.cuda.synchronize()
+
+    def phases(layer, qptr, ev=None):
+        c = caches[layer]
+        kv = c.kv
+        if ev is not None:
+            ev[0].record(stream)
+        ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
+        if ev is not None:
+            ev[1].record(stream)
+        ra.check(ra.ra_score_gqa(kv, qptr, Hq, k, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
+        if ev is not None:
+            ev[2].record(stream)
+        ra.check(ra.ra_topk_select(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+                                   ws.data_ptr(), ws_bytes, sp), "topk")
+        if ev is not None:
+            ev[3].record(stream)
+        ra.check(ra.ra_sparse_attn(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+                                   outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "attn")
+        if ev is not None:
+            ev[4].record(stream)
+        c.N = N - 1
+
+    def step(s, evs=None):
+        for layer in range(L):
+            phases(layer, qpool[s % P, layer].data_ptr(), None if evs is None else evs[layer])
+
+    # warm-up, then (for short timed regions) an untimed soak so clocks reach steady state
+    for s in range(max(3, args.warmup)):
+        step(s)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for s in range(5):
+        step(s)
+    torch.cuda.synchronize()
+    est = max((time.perf_counter() - t0) / 5, 1e-6)
+    steps = args.steps if args.steps is not None else max(10, min(20000, int(1.0 / est)))
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(L)]
+           for _ in range(steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    clk = Clocks(uuid)
+    clk.start()
+    soak_end = time.perf_counter() + 0.4
+    s = 0
+    while time.perf_counter() < soak_end:
+        step(s)
+        s += 1
+        if s % 64 == 0:
+            torch.cuda.synchronize()
+    barrier(dist, local_rank)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for s in range(steps):
+        step(s, evs[s])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, local_rank)
+    clocks = clk.stop()
+    elapsed_ms = t_start.elapsed_time(t_stop)
+    elapsed_ms = max_over_ranks(dist, elapsed_ms, dev)
+
+    ph = {"append": [], "score": [], "topk": [], "attn": []}
+    busy = 0.0
+    for s in range(steps):
+        for layer in range(L):
+            e = evs[s][layer]
+            ph["append"].append(e[0].elapsed_time(e[1]))
+            ph["score"].append(e[1].elapsed_time(e[2]))
+            ph["topk"].append(e[2].elapsed_time(e[3]))
+            ph["attn"].append(e[3].elapsed_time(e[4]))
+            busy += e[0].elapsed_time(e[4])
+    ph_us = {kk: 1000.0 * statistics.mean(v) for kk, v in ph.items()}
+    ms_per_step = elapsed_ms / steps
+    value = world * steps / (elapsed_ms / 1000.0)
+
+    # algorithmic bytes: K once per KV head, plus the V rows of U per query head
+    s1 = min(w.n_sink, N)
+    w0 = max(s1, N - w.n_window)
+    n_w = s1 + (N - w0)
+    k_eff = min(k, w0 - s1)
+    k_bytes = B * Hkv * N * 2 * d
+    v_bytes = B * Hq * (n_w + k_eff) * 2 * d
+    peak, peak_kind = measured_hbm_peak()
+    score_s = ph_us["score"] / 1e6
+    kscan_gbs = k_bytes / score_s / 1e9
+    step_gbs = L * (k_bytes + v_bytes) / (ms_per_step / 1000.0) / 1e9
+    src_hash = score_source_hash()
+    traffic = TRAFFIC.get((src_hash, w.name))
+    roofline = {"kernel": "score_gqa_kernel (K scan)", "bound": "hbm", "achieved": kscan_gbs,
+                "peak": peak, "unit": "GB/s", "frac": kscan_gbs / peak,
+                "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                "algorithmic_bytes_per_launch": k_bytes,
+                "frac_of_nominal_8tbs": kscan_gbs / NOMINAL_HBM_GBS,
+                "score_kernel_sha": src_hash}
+    launches_per_layer = 2 + (1 if k_eff > 0 else 0) + (1 if k > 0 else 0) + 1
+    result = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 / Irwin-Hall normals, Llama-3-8B-shaped caches)",
+        "config": workload_config(w),
+        "roofline": roofline,
+        "kscan_hbm_gbs": kscan_gbs,
+        "step_algorithmic_gbs": step_gbs,
+        "step_frac_of_peak": step_gbs / peak,
+        "step_frac_of_nominal_8tbs": step_gbs / NOMINAL_HBM_GBS,
+        "phases_us": ph_us,
+        "device_busy_frac": busy / elapsed_ms,
+        "gpu_launches": launches_per_layer * L * steps,
+        "clocks": clocks,
+    }
+
+    # dense flash-decode on the same cache (decode part only is compared)
+    if not args.no_dense:
+        for c in caches:
+            c.N = N
+        dws = torch.zeros(max(ra.ra_dense_workspace_bytes(B, Hq, N, d), 256), dtype=torch.uint8, device=dev)
+        dsteps = max(5, min(steps, 2000))
+        for s in range(5):
+            for layer in range(L):
+                ra.check(ra.ra_dense_decode(caches[layer].kv, qpool[s % P, layer].data_ptr(), Hq,
+                                            outs[layer].data_ptr(), dws.data_ptr(), dws.numel(), sp), "dense")
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for s in range(dsteps):
+            for layer in range(L):
+                ra.check(ra.ra_dense_decode(caches[layer].kv, qpool[s % P, layer].data_ptr(), Hq,
+                                            outs[layer].data_ptr(), dws.data_ptr(), dws.numel(), sp), "dense")
+        b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = max_over_ranks(dist, a.elapsed_time(b) / dsteps, dev)
+        sparse_decode_ms = L * (ph_us["score"] + ph_us["topk"] + ph_us["attn"]) / 1000.0
+        result["dense"] = {"ms_per_step": dense_ms, "steps": dsteps,
+                           "hbm_gbs": L * 2 * k_bytes / (dense_ms / 1000.0) / 1e9,
+                           "speedup_of_sparse_decode": dense_ms / sparse_decode_ms}
+        for c in caches:
+            c.N = N - 1
+        del dws
+
+    # end to end through the public Python API, inputs from pinned host memory
+    if not args.no_e2e:
+        esteps = max(5, min(steps, 1000))
+        hq = torch.empty((P, L, B, Hq, d), dtype=torch.bfloat16).pin_memory()
+        hq.copy_(qpool.cpu())
+        hk = [t.cpu().pin_memory() for t in knew]
+        hv = [t.cpu().pin_memory() for t in vnew]
+        dq = torch.empty((L, B, Hq, d), dtype=torch.bfloat16, device=dev)
+        dk = [torch.empty_like(t) for t in knew]
+        dv = [torch.empty_like(t) for t in vnew]
+        ho = torch.empty((L, B, Hq, d), dtype=torch.float32).pin_memory()
+        hi = torch.empty((L, B, Hq, max(k, 1)), dtype=torch.int32).pin_memory()
+
+        def e2e_step(s):
+            dq.copy_(hq[s % P], non_blocking=True)
+            for layer in range(L):
+                dk[layer].copy_(hk[layer], non_blocking=True)
+                dv[layer].copy_(hv[layer], non_blocking=True)
+                ra.append_kv(caches[layer], dk[layer], dv[layer])
+                ra.decode_step(caches[layer], dq[layer], k, w.n_sink, w.n_window,
+                               out=outs[layer], idx=idxs[layer], ws=ws)
+                caches[layer].N = N - 1
+                ho[layer].copy_(outs[layer], non_blocking=True)
+                hi[layer].copy_(idxs[layer], non_blocking=True)
+            stream.synchronize()
+
+        for s in range(3):
+            e2e_step(s)
+        barrier(dist, local_rank)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for s in range(esteps):
+            e2e_step(s)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(dist, a.elapsed_time(b) / esteps, dev)
+        h2d = L * (B * Hq * d * 2 + 2 * B * Hkv * d * 2)
+        d2h = L * (B * Hq * d * 4 + B * Hq * max(k, 1) * 4)
+        result["e2e"] = {"value": world * 1000.0 / e2e_ms, "unit": "steps/s",
+                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": esteps,
+                         "ms_per_step": e2e_ms,
+                         "note": "public API (append_kv + decode_step), host sync every step"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc = oracle_sample(w, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                                  "sample": desc}
+    return result
+
+
+def main():
+    args = parse()
+    rank, local_rank, world = dist_info()
+    from synth import gen
+    w = gen.workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product has no CPU path)")
+    dist = dist_init(world, True)
+    try:
+        res = run_ours(args, w, rank, local_rank, world, dist)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

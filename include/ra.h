@@ -20,7 +20,8 @@
  *
  * Conventions shared by every entry point:
  *   - Ownership: the caller owns every buffer (device memory unless stated).  The library
- *     allocates nothing and keeps no state between calls.
+ *     allocates nothing; the only state carried between calls is the zeroed counter block at
+ *     the front of a workspace (see ra_decode_step).
  *   - Ordering: all work is enqueued on `stream` (a cudaStream_t, may be NULL for the legacy
  *     default stream); no call synchronises the host.  Results are valid once the stream
  *     reaches that point.
@@ -108,7 +109,11 @@ size_t ra_decode_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, in
  *              positions of each query head, in unspecified order (a set); entries past
  *              min(k, |C|) are -1.  Ties in score go to the lower position.
  *   ws       : device workspace of at least ra_decode_workspace_bytes(...) bytes, 256-byte
- *              aligned; contents need no initialisation and are clobbered.
+ *              aligned, zero-filled once before its first use (cudaMemsetAsync(ws, 0, n)).
+ *              It starts with a counter block (per query head: a 2048-bin histogram and 8
+ *              counters) whose place depends on B*Hq only; every completed call leaves that
+ *              block zero again, so one workspace serves any later call with the same B*Hq
+ *              (N may grow; the dense path's workspace follows the same rule).
  * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_EMPTY (N == 0), RA_ERR_WORKSPACE, RA_ERR_CUDA.
  * Calls that share one workspace must not overlap on the device.
  */
@@ -118,7 +123,8 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
 
 /*
  * The three phases of ra_decode_step, exposed so a caller can time or interleave them.
- * Run in this order with the same arguments and workspace, they are ra_decode_step.
+ * Run in this order with the same arguments and workspace, they are ra_decode_step; run them
+ * only as that complete sequence (ra_topk_select re-zeroes what ra_score_gqa counted).
  *   ra_score_gqa   : z for every (query head, position) into ws, plus the per-head score
  *                    histogram of the candidates (one pass over K per KV head).
  *   ra_topk_select : Omega into idx from the scores in ws (radix select + bitonic finish).
@@ -139,7 +145,8 @@ size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d);
 /*
  * Full attention over all N cached tokens (Eq. (1)): the dense flash-decode comparison path.
  *   q : bf16 [B, Hq, d], device.   out : float32 [B, Hq, d], device.
- *   ws: at least ra_dense_workspace_bytes(...) bytes, 256-byte aligned.
+ *   ws: at least ra_dense_workspace_bytes(...) bytes, 256-byte aligned, zero-filled once
+ *       before first use (same counter-block rule as ra_decode_step).
  * Errors: as ra_decode_step.
  */
 ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out, void *ws,

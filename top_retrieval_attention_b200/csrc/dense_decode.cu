@@ -238,9 +238,9 @@ template <int D>
 static cudaError_t launch_dense_t(const DenseParams &p, cudaStream_t s) {
   using C = DenseCfg<D>;
   const size_t smem = C::smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(dense_decode_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static bool done[64] = {};
+  const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(dense_decode_kernel<D>),
+                                          static_cast<int>(smem), done);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.B * p.Hkv));
   dense_decode_kernel<D><<<grid, C::kThreads, smem, s>>>(p);

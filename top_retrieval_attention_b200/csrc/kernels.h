@@ -71,7 +71,10 @@ constexpr int kCollectChunk = 4096; // positions per collect CTA
 constexpr int kDenseTile = 128;
 
 int num_sms();
-int max_smem_optin();
+
+// Raises a kernel's dynamic shared-memory limit once per device (so that later launches,
+// including launches inside a stream capture, make no attribute call).
+cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]);
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);

@@ -33,6 +33,16 @@ int num_sms() {
   return cache[dev];
 }
 
+cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
 static constexpr size_t kAlign = 256;
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 static long long round4(long long x) { return (x + 3) / 4 * 4; }
@@ -65,10 +75,11 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.ldC = round4(std::max<long long>(st.nC, 1));
   const long long nU = st.nW + st.k_eff;
   st.nsplit = static_cast<int>(std::max<long long>(1, (nU + kAttnChunk - 1) / kAttnChunk));
+  // counter block first (its offsets depend on B*Hq only), then the per-call arrays
   size_t off = 0;
-  st.off_S = off;    off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
   st.off_hist = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_meta = off; off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
+  st.off_S = off;    off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
   st.off_cand = off; off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 4);
   st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit * (d + 2) * 4);
   st.total = off;
@@ -102,8 +113,6 @@ static uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + o
 
 static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void *ws,
                            cudaStream_t stream) {
-  cudaError_t e = cudaMemsetAsync(at(ws, st.off_hist), 0, st.off_cand - st.off_hist, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "memset");
   ScoreParams p{};
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -116,7 +125,7 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   p.B = st.B; p.Hkv = st.Hkv; p.G = st.G; p.Hq = st.Hq;
   p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
   p.do_hist = st.k_eff > 0 && st.k_eff < st.nC;
-  e = launch_score(p, st.d, stream);
+  const cudaError_t e = launch_score(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
 
@@ -161,10 +170,19 @@ static int dense_nsplit_cap(long long N) {
   return static_cast<int>(std::min<long long>(tiles, kDenseMaxSplit));
 }
 
-static size_t dense_bytes(int R, int nsplit_cap, int d, size_t *off_meta) {
-  size_t off = align_up(static_cast<size_t>(R) * nsplit_cap * (d + 2) * 4);
-  if (off_meta) *off_meta = off;
-  return align_up(off + static_cast<size_t>(R) * kMetaWords * 4);
+// Counter block: per-row histograms then per-row counters, at the front of every workspace.
+// Kernels leave it zero when they finish, so a workspace zero-filled once stays usable by
+// later calls with the same B * Hq (whatever N), sparse and dense alike.
+static size_t counter_bytes(int R, size_t *off_meta) {
+  const size_t m = align_up(static_cast<size_t>(R) * kHistBins * 4);
+  if (off_meta) *off_meta = m;
+  return align_up(m + static_cast<size_t>(R) * kMetaWords * 4);
+}
+
+static size_t dense_bytes(int R, int nsplit_cap, int d, size_t *off_meta, size_t *off_part) {
+  const size_t c = counter_bytes(R, off_meta);
+  if (off_part) *off_part = c;
+  return align_up(c + static_cast<size_t>(R) * nsplit_cap * (d + 2) * 4);
 }
 
 }  // namespace ra
@@ -266,7 +284,7 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d) {
   if (B < 1 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
   if (N >= (1LL << 31) - 1) return 0;
-  return dense_bytes(B * Hq, dense_nsplit_cap(N), d, nullptr);
+  return dense_bytes(B * Hq, dense_nsplit_cap(N), d, nullptr, nullptr);
 }
 
 ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out, void *ws,
@@ -279,8 +297,8 @@ ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out
   if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
   const int R = kv->B * Hq;
   const int cap_split = dense_nsplit_cap(kv->N);
-  size_t off_meta = 0;
-  const size_t need = dense_bytes(R, cap_split, kv->d, &off_meta);
+  size_t off_meta = 0, off_part = 0;
+  const size_t need = dense_bytes(R, cap_split, kv->d, &off_meta, &off_part);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < need)
     return RA_ERR_WORKSPACE;
 
@@ -306,19 +324,17 @@ ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out
   const int nsplit = static_cast<int>((kv->N + kps - 1) / kps);
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(at(ws, off_meta), 0, static_cast<size_t>(R) * kMetaWords * 4, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "memset");
   DenseParams p{};
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.q = static_cast<const __nv_bfloat16 *>(q);
-  p.part = static_cast<float *>(ws);
+  p.part = reinterpret_cast<float *>(at(ws, off_part));
   p.out = out;
   p.meta = reinterpret_cast<uint32_t *>(at(ws, off_meta));
   p.N = kv->N; p.cap = kv->cap; p.keys_per_split = kps;
   p.B = kv->B; p.Hkv = kv->Hkv; p.G = Hq / kv->Hkv; p.Hq = Hq; p.nsplit = nsplit;
   p.scale = 1.0f / sqrtf(static_cast<float>(kv->d));
-  e = launch_dense(p, kv->d, cs);
+  const cudaError_t e = launch_dense(p, kv->d, cs);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "dense_decode");
 }
 

@@ -161,9 +161,9 @@ template <int D>
 static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
   using C = ScoreCfg<D>;
   const size_t smem = C::smem_bytes(p.G);
-  cudaError_t e = cudaFuncSetAttribute(score_gqa_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::smem_bytes(kMaxGroup)));
+  static bool done[64] = {};
+  const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D>),
+                                          static_cast<int>(C::smem_bytes(kMaxGroup)), done);
   if (e != cudaSuccess) return e;
   long long grid = num_sms();
   if (grid > p.total_tiles) grid = p.total_tiles;

@@ -121,9 +121,9 @@ __global__ void __launch_bounds__(kCollectThreads) topk_collect_kernel(const Top
       const int bin = static_cast<int>(order_key(zz[e]) >> (32 - kHistBits));
       bool ok;
       const uint32_t s1 = warp_append(valid && bin > bstar, sel_ctr, ok);
-      if (ok) irow[s1] = static_cast<int32_t>(pos);
+      if (ok && s1 < p.k_eff) irow[s1] = static_cast<int32_t>(pos);
       const uint32_t s2 = warp_append(valid && !take_all && bin == bstar, cand_ctr, ok);
-      if (ok) crow[s2] = static_cast<uint32_t>(pos);
+      if (ok && s2 < p.ldC) crow[s2] = static_cast<uint32_t>(pos);
     }
   }
 }
@@ -134,6 +134,18 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(const TopkP
   const int lane = tid & 31, warp = tid >> 5;
   int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   for (long long i = p.k_eff + tid; i < p.k; i += kFinishThreads) irow[i] = -1;
+
+  // read this row's counters, then leave the counter block zero for the next call
+  uint32_t *meta_w = p.meta + row * kMetaWords;
+  const uint32_t above = meta_w[kAbove];
+  const uint32_t n_cand = meta_w[kCandCount];
+  const uint32_t bstar = meta_w[kThreshBin];
+  __syncthreads();
+  if (tid < kError) meta_w[tid] = 0u;
+  {
+    uint32_t *h = const_cast<uint32_t *>(p.hist) + static_cast<long long>(row) * kHistBins;
+    for (int i = tid; i < kHistBins; i += kFinishThreads) h[i] = 0u;
+  }
   if (p.k_eff == 0 || p.k_eff >= p.nC) return;
 
   extern __shared__ __align__(16) uint64_t cache[];
@@ -143,13 +155,10 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(const TopkP
   __shared__ uint32_t s_cum, s_cnt, s_nb;
   __shared__ uint64_t bs[kBitonic];
 
-  const uint32_t *meta = p.meta + row * kMetaWords;
-  const uint32_t above = meta[kAbove];
-  const uint32_t n_cand = meta[kCandCount];
-  const uint32_t bstar = meta[kThreshBin];
   uint32_t rr = static_cast<uint32_t>(p.k_eff) - above;    // 1 <= rr <= n_cand
   const float *srow = p.S + static_cast<long long>(row) * p.ldS;
   const uint32_t *crow = p.cand + static_cast<long long>(row) * p.ldC;
+  if (n_cand > p.nC || above >= p.k_eff) return;   // counters not from this call
   const bool cached = n_cand <= static_cast<uint32_t>(kFinishCache);
   if (tid == 0) s_out = above;
   if (cached)
@@ -169,7 +178,10 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(const TopkP
     if (cnt == rr) {   // the whole bucket is taken
       for (uint32_t i = tid; i < n_cand; i += kFinishThreads) {
         const uint64_t x = get(i);
-        if ((x >> shift) == prefix) irow[atomicAdd(&s_out, 1u)] = static_cast<int32_t>(comp_pos(x));
+        if ((x >> shift) == prefix) {
+          const uint32_t o = atomicAdd(&s_out, 1u);
+          if (o < p.k_eff) irow[o] = static_cast<int32_t>(comp_pos(x));
+        }
       }
       return;
     }
@@ -198,7 +210,7 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(const TopkP
             __syncwarp();
           }
         }
-        for (uint32_t i = lane; i < rr; i += 32)
+        for (uint32_t i = lane; i < rr && s_out + i < p.k_eff; i += 32)
           irow[s_out + i] = static_cast<int32_t>(comp_pos(bs[i]));
       }
       return;
@@ -248,8 +260,10 @@ __global__ void __launch_bounds__(kFinishThreads) topk_finish_kernel(const TopkP
     // keys of this bucket with a larger digit are selected
     for (uint32_t i = tid; i < n_cand; i += kFinishThreads) {
       const uint64_t x = get(i);
-      if ((x >> shift) == prefix && ((x >> nshift) & dmask) > v)
-        irow[atomicAdd(&s_out, 1u)] = static_cast<int32_t>(comp_pos(x));
+      if ((x >> shift) == prefix && ((x >> nshift) & dmask) > v) {
+        const uint32_t o = atomicAdd(&s_out, 1u);
+        if (o < p.k_eff) irow[o] = static_cast<int32_t>(comp_pos(x));
+      }
     }
     rr -= cum;
     cnt = s_cnt;
@@ -270,9 +284,9 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
   }
   if (p.k > 0) {
     const size_t smem = static_cast<size_t>(kFinishCache) * sizeof(uint64_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_finish_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    static bool done[64] = {};
+    const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(topk_finish_kernel),
+                                            static_cast<int>(smem), done);
     if (e != cudaSuccess) return e;
     topk_finish_kernel<<<p.R, kFinishThreads, smem, s>>>(p);
     return cudaGetLastError();

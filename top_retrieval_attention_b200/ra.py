@@ -175,7 +175,7 @@ def decode_workspace(cache: KVCache, Hq: int, k: int, n_sink: int, n_window: int
     n = ra_decode_workspace_bytes(cache.B, Hq, cache.N, cache.d, k, n_sink, n_window)
     if n == 0:
         raise RaError(RA_ERR_SHAPE, "ra_decode_workspace_bytes")
-    return torch.empty(n, dtype=torch.uint8, device=cache.K.device)
+    return torch.zeros(n, dtype=torch.uint8, device=cache.K.device)
 
 
 def decode_step(cache: KVCache, q, k: int, n_sink: int, n_window: int, out=None, idx=None,
@@ -200,7 +200,7 @@ def dense_workspace(cache: KVCache, Hq: int):
     n = ra_dense_workspace_bytes(cache.B, Hq, cache.N, cache.d)
     if n == 0:
         raise RaError(RA_ERR_SHAPE, "ra_dense_workspace_bytes")
-    return torch.empty(n, dtype=torch.uint8, device=cache.K.device)
+    return torch.zeros(n, dtype=torch.uint8, device=cache.K.device)
 
 
 def dense_decode(cache: KVCache, q, out=None, ws=None, stream=None):
