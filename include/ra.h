@@ -139,6 +139,26 @@ ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
                          int32_t n_window, const int32_t *idx, float *out, void *ws,
                          size_t ws_bytes, ra_stream_t stream);
 
+/*
+ * ra_decode_step without a caller workspace, for callers that cannot allocate device memory
+ * (for example a plugin that its host engine hands only input and output pointers, or a serving
+ * loop that bans cudaMalloc after start-up because it can synchronise the device).  The paper
+ * has no counterpart: this is a packaging variant of ra_decode_step.
+ *   Arguments, outputs and errors are those of ra_decode_step, without ws / ws_bytes.
+ *   Scratch: a 64 MiB array inside libra (a file-scope __device__ array), held on every GPU
+ *     that loads the library until the process exits.  A shape whose
+ *     ra_decode_workspace_bytes(...) exceeds 64 MiB is rejected with RA_ERR_WORKSPACE before
+ *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 34 MB).
+ *   The first call on each device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture.
+ *   Each call clears the scratch's counter block with cudaMemsetAsync on `stream`; nothing is
+ *     allocated.  All calls on a device share the one array and it keeps the last call's
+ *     contents, so calls that overlap on the GPU (other streams, other host threads) race.
+ */
+ra_status ra_decode_step_static(const ra_kv *kv, const void *q, int32_t Hq, int32_t k,
+                                int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
+                                ra_stream_t stream);
+
 /* Workspace bytes for ra_dense_decode (split partial states).  0 for an invalid shape. */
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d);
 

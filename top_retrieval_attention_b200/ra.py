@@ -20,7 +20,8 @@ RA_OK, RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_CAPACITY, RA_ERR_WORKSPACE, RA_ERR_CUDA,
 #: every symbol include/ra.h declares
 EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
-           "ra_sparse_attn", "ra_dense_workspace_bytes", "ra_dense_decode")
+           "ra_sparse_attn", "ra_dense_workspace_bytes", "ra_dense_decode",
+           "ra_decode_step_static")
 
 
 class ra_kv(ctypes.Structure):
@@ -57,6 +58,8 @@ def lib() -> ctypes.CDLL:
             "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
             "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                                           c_void_p]),
+            "ra_decode_step_static": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32,
+                                                c_void_p, c_void_p, c_void_p]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -106,6 +109,12 @@ def ra_topk_select(kv, Hq, k, n_sink, n_window, idx, ws, ws_bytes, stream):
 def ra_sparse_attn(kv, Hq, k, n_sink, n_window, idx, out, ws, ws_bytes, stream):
     return lib().ra_sparse_attn(ctypes.byref(kv), Hq, k, n_sink, n_window, idx, out, ws,
                                 ws_bytes, stream)
+
+
+def ra_decode_step_static(kv, q, Hq, k, n_sink, n_window, out, idx, stream):
+    """ra_decode_step on libra's built-in 64 MiB scratch: for callers that cannot allocate."""
+    return lib().ra_decode_step_static(ctypes.byref(kv), q, Hq, k, n_sink, n_window, out, idx,
+                                       stream)
 
 
 def ra_dense_workspace_bytes(B, Hq, N, d) -> int:
