@@ -7,6 +7,8 @@
 namespace ra {
 
 __global__ void __launch_bounds__(256) append_kv_kernel(const AppendParams p) {
+  pdl_trigger();
+  pdl_wait();   // the previous step may still read the rows this append overwrites
   // one 16-byte unit per thread: units per row = d / 8
   const int upr = p.d / 8;
   const long long units = static_cast<long long>(p.B) * p.Hkv * p.T * upr;
@@ -30,8 +32,7 @@ cudaError_t launch_append(const AppendParams &p, cudaStream_t s) {
   long long blocks = (units + 255) / 256;
   if (blocks > 4LL * num_sms()) blocks = 4LL * num_sms();
   if (blocks < 1) blocks = 1;
-  append_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(append_kv_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
 }
 
 }  // namespace ra

@@ -16,6 +16,16 @@ constexpr int kMetaWords = 8;                 // per-row counters in the workspa
 enum MetaSlot { kSelCount = 0, kCandCount = 1, kThreshBin = 2, kAbove = 3, kDone = 4,
                 kDenseDone = 5, kError = 6 };
 
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Kernels of a decode step are launched with programmatic stream serialisation: each lets the
+// next kernel of the stream be scheduled as soon as all of its own CTAs are running, and
+// waits for its predecessor (completion and memory visibility) before touching its outputs.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 // ------------------------------------------------------------------ order-preserving keys
 
 // Maps a float to a uint32 whose unsigned order equals the float order (-0 sorts below +0;

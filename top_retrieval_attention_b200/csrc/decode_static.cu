@@ -15,6 +15,7 @@
 
 #include "../../include/ra.h"
 #include "common.cuh"
+#include "kernels.h"
 
 namespace {
 
@@ -25,8 +26,6 @@ __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 // Device address of g_scratch per device.  In host code `g_scratch` names a host-side stand-in,
 // not device memory, so the address is looked up once per device with that device current.
 void *g_scratch_addr[64] = {};
-
-size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -56,7 +55,7 @@ extern "C" ra_status ra_decode_step_static(const ra_kv *kv, const void *q, int32
   // The counter block at the front of the workspace (per query head: histogram and
   // counters) must start at zero; clear it on every call rather than trusting the last one.
   const size_t rows = static_cast<size_t>(kv->B) * static_cast<size_t>(Hq);
-  const size_t counters = align256(rows * ra::kHistBins * 4) + align256(rows * ra::kMetaWords * 4);
+  const size_t counters = ra::counter_block_bytes(rows);
   if (cudaMemsetAsync(ws, 0, counters, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return RA_ERR_CUDA;
   return ra_decode_step(kv, q, Hq, k, n_sink, n_window, out, idx, ws, kStaticScratchBytes, stream);

@@ -5,7 +5,28 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace ra {
+
+// Launches `kernel` on `s` with programmatic stream serialisation allowed, so it may be
+// scheduled while its predecessor in the stream is still finishing (it synchronises with
+// griddepcontrol.wait before reading the predecessor's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Scores of every (query head, position) of one layer, plus the first radix digit's
 // histogram of the candidates (z in S is already scaled by 1/sqrt(d)).
@@ -21,17 +42,17 @@ struct ScoreParams {
   int B, Hkv, G, Hq;
   float scale;
   int do_hist;
+  uint32_t *err;            // error word (bit kErrScoreWait: a load never landed)
 };
 
 struct TopkParams {
   const float *S;
-  const uint32_t *hist;
-  uint32_t *meta;           // [B*Hq, kMetaWords] (zeroed before the score launch)
-  uint32_t *cand;           // [B*Hq, ldC]
+  uint32_t *hist;           // [B*Hq, kHistBins] digit-1 histogram (left zero by the select)
+  uint32_t *meta;           // [B*Hq, kMetaWords] counters (left zero by the select)
+  uint2 *cand;              // [B*Hq, ldC] (position, order key): overflow of the last bucket
   int32_t *idx;             // [B*Hq, k]
   long long ldS, ldC, N;
   long long cand_lo, cand_hi, nC, k_eff;
-  long long chunk;          // positions per collect CTA
   int k, R;
 };
 
@@ -39,22 +60,24 @@ struct AttnParams {
   const float *S;
   const __nv_bfloat16 *V;
   const int32_t *idx;
-  float *part;              // [B*Hq, nsplit, d + 2]
+  float *part;              // [B*Hq, nsplit, d + 4] partial states (m, Z, pad, pad, N[d])
   float *out;               // [B*Hq, d]
   uint32_t *meta;
   long long ldS, cap, N;
   long long s1, w0, nW, k_eff;
   int k, Hq, G, Hkv, nsplit, R;
+  int range;                // entries of U per CTA (multiple of 64, <= kMaxRange)
 };
 
 struct DenseParams {
   const __nv_bfloat16 *K, *V, *q;
-  float *part;              // [B*Hq, nsplit, d + 2]
+  float *part;              // [B*Hq, nsplit, d + 4] partial states (m, Z, pad, pad, N[d])
   float *out;               // [B*Hq, d]
-  uint32_t *meta;           // [B*Hq, kMetaWords] (zeroed before the launch)
+  uint32_t *meta;           // [B*Hq, kMetaWords] counters (left zero by the merging CTA)
   long long N, cap, keys_per_split;
   int B, Hkv, G, Hq, nsplit;
   float scale;
+  uint32_t *err;            // error word (bit kErrDenseWait: a load never landed)
 };
 
 struct AppendParams {
@@ -66,11 +89,16 @@ struct AppendParams {
 
 // tuning constants the host layout needs
 constexpr int kScoreTile = 128;
-constexpr int kAttnChunk = 64;      // U entries per sparse-attention CTA
-constexpr int kCollectChunk = 4096; // positions per collect CTA
+constexpr int kMaxRange = 2048;     // U entries per sparse-attention CTA, at most
+constexpr int kAttnTargetCtas = 1184;   // 8 CTAs per SM of a 148-SM B200: sizes the U ranges
+constexpr int kSelCluster = 8;      // CTAs per query head in the top-k select (one cluster)
 constexpr int kDenseTile = 128;
 
 int num_sms();
+
+// Bytes of the counter block at the front of every workspace for `rows` query heads
+// (digit-1 histograms, then the per-row counters), 256-byte aligned sections.
+size_t counter_block_bytes(size_t rows);
 
 // Raises a kernel's dynamic shared-memory limit once per device (so that later launches,
 // including launches inside a stream capture, make no attribute call).

@@ -44,6 +44,12 @@ cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]) {
 }
 
 static constexpr size_t kAlign = 256;
+
+size_t counter_block_bytes(size_t rows) {
+  const size_t h = (rows * kHistBins * 4 + kAlign - 1) / kAlign * kAlign;
+  const size_t m = (rows * kMetaWords * 4 + kAlign - 1) / kAlign * kAlign;
+  return h + m;
+}
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 static long long round4(long long x) { return (x + 3) / 4 * 4; }
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -51,7 +57,7 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Derived sizes of one decode step (positions follow the slide "The GPU keeps 640 fixed
 // positions": W = [0, s1) u [w0, N), candidates C = [s1, w0)).
 struct Step {
-  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit;
+  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, range;
   long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC;
   size_t off_S, off_hist, off_meta, off_cand, off_part, total;
 };
@@ -73,15 +79,20 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.k_eff = std::min<long long>(k, st.nC);
   st.ldS = round4(std::max<long long>(N, 1));
   st.ldC = round4(std::max<long long>(st.nC, 1));
-  const long long nU = st.nW + st.k_eff;
-  st.nsplit = static_cast<int>(std::max<long long>(1, (nU + kAttnChunk - 1) / kAttnChunk));
+  // U ranges: enough CTAs for a few waves, each range a multiple of 64 entries
+  const long long nU = std::max<long long>(1, st.nW + st.k_eff);
+  const long long want = std::max<long long>(1, (kAttnTargetCtas + st.R - 1) / st.R);
+  long long range = (nU + want - 1) / want;
+  range = std::min<long long>(kMaxRange, std::max<long long>(64, (range + 63) / 64 * 64));
+  st.range = static_cast<int>(range);
+  st.nsplit = static_cast<int>((nU + range - 1) / range);
   // counter block first (its offsets depend on B*Hq only), then the per-call arrays
   size_t off = 0;
-  st.off_hist = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
-  st.off_meta = off; off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
-  st.off_S = off;    off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
-  st.off_cand = off; off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 4);
-  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit * (d + 2) * 4);
+  st.off_hist = off;  off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
+  st.off_meta = off;  off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
+  st.off_S = off;     off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
+  st.off_cand = off;  off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 8);
+  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit * (d + 4) * 4);
   st.total = off;
   return RA_OK;
 }
@@ -125,6 +136,7 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   p.B = st.B; p.Hkv = st.Hkv; p.G = st.G; p.Hq = st.Hq;
   p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
   p.do_hist = st.k_eff > 0 && st.k_eff < st.nC;
+  p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
   const cudaError_t e = launch_score(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
@@ -133,13 +145,12 @@ static ra_status run_topk(const Step &st, int32_t *idx, void *ws, cudaStream_t s
   if (st.k == 0) return RA_OK;
   TopkParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
-  p.hist = reinterpret_cast<const uint32_t *>(at(ws, st.off_hist));
+  p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
   p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
-  p.cand = reinterpret_cast<uint32_t *>(at(ws, st.off_cand));
+  p.cand = reinterpret_cast<uint2 *>(at(ws, st.off_cand));
   p.idx = idx;
   p.ldS = st.ldS; p.ldC = st.ldC; p.N = st.N;
   p.cand_lo = st.s1; p.cand_hi = st.w0; p.nC = st.nC; p.k_eff = st.k_eff;
-  p.chunk = kCollectChunk;
   p.k = st.k; p.R = st.R;
   cudaError_t e = launch_topk(p, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "topk");
@@ -157,6 +168,7 @@ static ra_status run_attn(const ra_kv *kv, const Step &st, const int32_t *idx, f
   p.ldS = st.ldS; p.cap = st.cap; p.N = st.N;
   p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.k_eff = st.k_eff;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.nsplit = st.nsplit; p.R = st.R;
+  p.range = st.range;
   cudaError_t e = launch_sparse_attn(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "sparse_attn");
 }
@@ -182,7 +194,7 @@ static size_t counter_bytes(int R, size_t *off_meta) {
 static size_t dense_bytes(int R, int nsplit_cap, int d, size_t *off_meta, size_t *off_part) {
   const size_t c = counter_bytes(R, off_meta);
   if (off_part) *off_part = c;
-  return align_up(c + static_cast<size_t>(R) * nsplit_cap * (d + 2) * 4);
+  return align_up(c + static_cast<size_t>(R) * nsplit_cap * (d + 4) * 4);
 }
 
 }  // namespace ra
@@ -334,6 +346,7 @@ ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out
   p.N = kv->N; p.cap = kv->cap; p.keys_per_split = kps;
   p.B = kv->B; p.Hkv = kv->Hkv; p.G = Hq / kv->Hkv; p.Hq = Hq; p.nsplit = nsplit;
   p.scale = 1.0f / sqrtf(static_cast<float>(kv->d));
+  p.err = reinterpret_cast<uint32_t *>(at(ws, off_meta)) + kError;
   const cudaError_t e = launch_dense(p, kv->d, cs);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "dense_decode");
 }

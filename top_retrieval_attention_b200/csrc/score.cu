@@ -4,16 +4,19 @@
 // keeps 640 fixed positions": GQA heads share KV storage).
 //
 // Design (HBM bound: 2d bytes of K per position against 2Gd flops):
-//   * persistent grid, one CTA per SM, each CTA streams a contiguous range of 128-key tiles;
-//   * tiles are staged global -> shared by 16-byte cp.async into an XOR-swizzled ring of
-//     kStages tiles, so several tiles are in flight per SM while one is computed;
-//   * the G query vectors are the n = 8 operand of a bf16 m16n8k16 tensor-core product with
+//   * persistent grid, one CTA per SM; each CTA streams a contiguous range of 128-key tiles
+//     (the tile cursor advances incrementally, no per-tile division);
+//   * one thread issues TMA bulk tensor loads (128-byte swizzled boxes of 128 keys x 64
+//     channels, L2 evict-first) into a ring of kStages tiles, completion counted on one
+//     mbarrier per stage; every thread waits on the stage barrier with a bounded poll;
+//   * the G query vectors are the n = 8 operand of bf16 m16n8k16 tensor-core products with
 //     fp32 accumulation; each warp scores 16 keys of the tile from ldmatrix fragments;
-//   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram
-//     (top 11 bits of the order-preserving key) of the candidate positions in shared
-//     memory, flushed to global once per KV head.
+//   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram (top
+//     11 bits of the order-preserving key) of the candidate positions in shared memory,
+//     flushed to global once per KV head.
 #include "common.cuh"
 #include "kernels.h"
+#include "tma.cuh"
 
 namespace ra {
 
@@ -21,23 +24,26 @@ template <int D>
 struct ScoreCfg {
   static constexpr int kThreads = 256;
   static constexpr int kWarps = 8;
-  static constexpr int kTile = kScoreTile;               // keys per tile (16 per warp)
-  static constexpr int kRowBytes = D * 2;
-  static constexpr int kTileBytes = kTile * kRowBytes;   // 32 KB (d=128) / 16 KB (d=64)
-  static constexpr int kStages = D == 128 ? 4 : 6;
-  static constexpr int kChunksPerRow = kRowBytes / 16;
-  static constexpr int kCopiesPerThread = kTile * kChunksPerRow / kThreads;
+  static constexpr int kTile = kScoreTile;                 // keys per tile (16 per warp)
+  static constexpr int kBoxes = D / 64;                    // 64-channel boxes per tile
+  static constexpr int kBoxBytes = kTile * 128;            // 16 KB
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;    // 32 KB (d=128) / 16 KB (d=64)
+  static constexpr int kStages = D == 128 ? 5 : 8;
   static constexpr size_t smem_bytes(int G) {
-    return static_cast<size_t>(kStages) * kTileBytes + static_cast<size_t>(G) * kHistBins * 4;
+    return 1024 + static_cast<size_t>(kStages) * kTileBytes +
+           static_cast<size_t>(G) * kHistBins * 4 + kStages * 8;
   }
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) {
+__global__ void __launch_bounds__(256, 1)
+    score_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const ScoreParams p) {
   using C = ScoreCfg<D>;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *tiles = smem;
-  uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem + C::kStages * C::kTileBytes);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t tiles = (raw + 1023u) & ~1023u;          // swizzled boxes need 1024-byte alignment
+  uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem_raw + (tiles - raw) + C::kStages * C::kTileBytes);
+  const uint32_t bars = tiles + C::kStages * C::kTileBytes + p.G * kHistBins * 4;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -47,26 +53,39 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
   const long long rem = p.total_tiles % gridDim.x;
   const long long t_begin = blockIdx.x * per + min(static_cast<long long>(blockIdx.x), rem);
   const int n_local = static_cast<int>(per + (blockIdx.x < rem ? 1 : 0));
+  pdl_trigger();
+  if (n_local <= 0) return;
 
+  if (tid == 0) {
+    prefetch_tmap(&tmK);
+    for (int s = 0; s < C::kStages; ++s) mbar_init(bars + 8 * s, 1);
+    fence_mbar_init();
+  }
   if (p.do_hist)
     for (int i = tid; i < p.G * kHistBins; i += C::kThreads) hist_s[i] = 0;
+  __syncthreads();
+  pdl_wait();   // K (appended rows) and the score / histogram buffers belong to the predecessor
 
-  auto load_tile = [&](long long t, int slot) {
-    const long long bg = t / p.tiles_per_head;
-    const long long key0 = (t - bg * p.tiles_per_head) * C::kTile;
-    const __nv_bfloat16 *src0 = p.K + (bg * p.cap + key0) * D;
-    const uint32_t dst0 = smem_u32(tiles + slot * C::kTileBytes);
+  // load cursor (thread 0 only) and compute cursor (all threads)
+  const long long bg0 = t_begin / p.tiles_per_head;
+  long long l_bg = bg0, l_key = (t_begin - bg0 * p.tiles_per_head) * C::kTile;
+  long long c_bg = bg0, c_key = l_key;
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int slot) {
+    const uint32_t bar = bars + 8 * slot;
+    mbar_arrive_expect_tx(bar, C::kTileBytes);
 #pragma unroll
-    for (int i = 0; i < C::kCopiesPerThread; ++i) {
-      const int ci = i * C::kThreads + tid;
-      const int r = ci / C::kChunksPerRow;
-      const int c = ci % C::kChunksPerRow;
-      const bool valid = key0 + r < p.N;
-      const void *src = valid ? static_cast<const void *>(src0 + static_cast<long long>(r) * D + c * 8)
-                              : static_cast<const void *>(p.K);
-      cp_async16(dst0 + swz(r, c, C::kRowBytes), src, valid ? 16u : 0u);
+    for (int bx = 0; bx < C::kBoxes; ++bx)
+      tma_load_3d(tiles + slot * C::kTileBytes + bx * C::kBoxBytes, &tmK, bx * 64,
+                  static_cast<int>(l_key), static_cast<int>(l_bg), bar, pol);
+    l_key += C::kTile;
+    if (l_key >= p.N) {
+      l_key = 0;
+      ++l_bg;
     }
   };
+  if (tid == 0)
+    for (int s = 0; s < C::kStages - 1 && s < n_local; ++s) issue(s);
 
   auto flush_hist = [&](long long bg) {
     const long long b = bg / p.Hkv;
@@ -81,12 +100,6 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
     }
   };
 
-#pragma unroll 1
-  for (int s = 0; s < C::kStages - 1; ++s) {
-    if (s < n_local) load_tile(t_begin + s, s);
-    cp_async_commit();
-  }
-
   long long cur_bg = -1;
   long long rowbase = 0;
   uint32_t bq[D / 16][2];
@@ -94,27 +107,23 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
   const int arow = warp * 16 + (lane & 7) + (mat & 1) * 8;   // ldmatrix source row
   const int g4 = lane >> 2;
   const int t4 = lane & 3;
+  int j = 0;
 
 #pragma unroll 1
-  for (int j = 0; j < n_local; ++j) {
-    cp_async_wait<C::kStages - 2>();
-    __syncthreads();
-    {
-      const int jn = j + C::kStages - 1;
-      if (jn < n_local) load_tile(t_begin + jn, jn % C::kStages);
-      cp_async_commit();
-    }
-    const long long t = t_begin + j;
-    const long long bg = t / p.tiles_per_head;
-    const long long key0 = (t - bg * p.tiles_per_head) * C::kTile;
-    if (bg != cur_bg) {
+  for (; j < n_local; ++j) {
+    const int slot = j % C::kStages;
+    const bool landed = mbar_wait(bars + 8 * slot, static_cast<uint32_t>((j / C::kStages) & 1));
+    if (!__syncthreads_and(landed)) break;     // uniform: every warp also finished tile j-1
+    if (tid == 0 && j + C::kStages - 1 < n_local) issue((j + C::kStages - 1) % C::kStages);
+
+    if (c_bg != cur_bg) {
       if (cur_bg >= 0 && p.do_hist) {
         flush_hist(cur_bg);
         __syncthreads();
       }
-      cur_bg = bg;
-      const long long b = bg / p.Hkv;
-      const long long g = bg - b * p.Hkv;
+      cur_bg = c_bg;
+      const long long b = c_bg / p.Hkv;
+      const long long g = c_bg - b * p.Hkv;
       rowbase = b * p.Hq + g * p.G;
       // B operand (col-major k x n): element (k = channel, n = query head g4)
       const uint32_t *qrow =
@@ -126,15 +135,19 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
       }
     }
 
-    const uint32_t tbase = smem_u32(tiles + (j % C::kStages) * C::kTileBytes);
+    const uint32_t tbase = tiles + slot * C::kTileBytes;
     float acc0[4] = {0.f, 0.f, 0.f, 0.f};
     float acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk += 2) {
+      // logical 16-byte chunk c of row r lives in box c / 8 at swizzled chunk (c % 8) ^ (r % 8)
+      const int c0 = 2 * kk + (mat >> 1);
+      const int c1 = c0 + 2;
       uint32_t a[4], a2[4];
-      ldmatrix_x4(tbase + swz(arow, 2 * kk + (mat >> 1), C::kRowBytes), a[0], a[1], a[2], a[3]);
-      ldmatrix_x4(tbase + swz(arow, 2 * kk + 2 + (mat >> 1), C::kRowBytes), a2[0], a2[1], a2[2],
-                  a2[3]);
+      ldmatrix_x4(tbase + (c0 >> 3) * C::kBoxBytes + arow * 128 + (((c0 & 7) ^ (arow & 7)) << 4),
+                  a[0], a[1], a[2], a[3]);
+      ldmatrix_x4(tbase + (c1 >> 3) * C::kBoxBytes + arow * 128 + (((c1 & 7) ^ (arow & 7)) << 4),
+                  a2[0], a2[1], a2[2], a2[3]);
       mma_bf16_16816(acc0, a, bq[kk][0], bq[kk][1]);
       mma_bf16_16816(acc1, a2, bq[kk + 1][0], bq[kk + 1][1]);
     }
@@ -143,7 +156,7 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int h = 2 * t4 + (e & 1);
-      const long long key = key0 + warp * 16 + g4 + (e >> 1) * 8;
+      const long long key = c_key + warp * 16 + g4 + (e >> 1) * 8;
       if (h < p.G && key < p.N) {
         const float z = canon_zero((acc0[e] + acc1[e]) * p.scale);
         p.S[(rowbase + h) * p.ldS + key] = z;
@@ -151,8 +164,22 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
           atomicAdd(&hist_s[h * kHistBins + (order_key(z) >> (32 - kHistBits))], 1u);
       }
     }
+    c_key += C::kTile;
+    if (c_key >= p.N) {
+      c_key = 0;
+      ++c_bg;
+    }
   }
-  cp_async_wait<0>();
+
+  if (j < n_local) {
+    // a stage never completed: record it, wait (bounded) for the copies still in flight
+    if (tid == 0) {
+      atomicOr(p.err, kErrScoreWait);
+      for (int jj = j; jj < n_local && jj < j + C::kStages - 1; ++jj)
+        mbar_wait(bars + 8 * (jj % C::kStages), static_cast<uint32_t>((jj / C::kStages) & 1));
+    }
+    return;
+  }
   __syncthreads();
   if (cur_bg >= 0 && p.do_hist) flush_hist(cur_bg);
 }
@@ -160,16 +187,19 @@ __global__ void __launch_bounds__(256, 1) score_gqa_kernel(const ScoreParams p) 
 template <int D>
 static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
   using C = ScoreCfg<D>;
-  const size_t smem = C::smem_bytes(p.G);
   static bool done[64] = {};
-  const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D>),
-                                          static_cast<int>(C::smem_bytes(kMaxGroup)), done);
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D>),
+                                    static_cast<int>(C::smem_bytes(kMaxGroup)), done);
   if (e != cudaSuccess) return e;
+  CUtensorMap tm;
+  if (!encode_rows_tmap(&tm, p.K, D, static_cast<uint64_t>(p.N),
+                        static_cast<uint64_t>(p.B) * p.Hkv, C::kTile, static_cast<uint64_t>(p.cap)))
+    return cudaErrorInvalidValue;
   long long grid = num_sms();
   if (grid > p.total_tiles) grid = p.total_tiles;
   if (grid < 1) grid = 1;
-  score_gqa_kernel<D><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(score_gqa_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads),
+                    C::smem_bytes(p.G), s, tm, p);
 }
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s) {
