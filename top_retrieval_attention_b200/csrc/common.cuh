@@ -13,8 +13,8 @@ constexpr int kMaxGroup = 8;                  // query heads per KV head (one n8
 constexpr int kMetaWords = 8;                 // per-row counters in the workspace
 
 // per-row counters (uint32) in the workspace's meta block
-enum MetaSlot { kSelCount = 0, kCandCount = 1, kThreshBin = 2, kAbove = 3, kDone = 4,
-                kDenseDone = 5, kError = 6 };
+enum MetaSlot { kSelCount = 0, kCandCount = 1, kError = 6, kDone = 7 };
+// kDone is shared by the sparse and the dense merge (each leaves it zero).
 
 // ------------------------------------------------------------------ programmatic dependent launch
 

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    const uint32_t prev = atomicAdd(p.meta + rowbase * kMetaWords + kDenseDone, 1u);
+    const uint32_t prev = atomicAdd(p.meta + rowbase * kMetaWords + kDone, 1u);
     s_last = prev == static_cast<uint32_t>(p.nsplit - 1);
     if (s_last) __threadfence();
   }
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(256, 1)
   for (int h = 0; h < p.G; ++h)
     merge_states<D, C::kThreads>(p.part + (rowbase + h) * p.nsplit * (D + kPartPad), p.nsplit,
                                  p.out + (rowbase + h) * D, red, buf);
-  if (tid == 0) p.meta[rowbase * kMetaWords + kDenseDone] = 0u;
+  if (tid == 0) p.meta[rowbase * kMetaWords + kDone] = 0u;
 }
 
 template <int D>

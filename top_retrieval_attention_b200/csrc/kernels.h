@@ -48,8 +48,9 @@ struct ScoreParams {
 struct TopkParams {
   const float *S;
   uint32_t *hist;           // [B*Hq, kHistBins] digit-1 histogram (left zero by the select)
+  uint32_t *hist2;          // [B*Hq, kHistBins] digit-2 histogram of the listed keys (same)
   uint32_t *meta;           // [B*Hq, kMetaWords] counters (left zero by the select)
-  uint2 *cand;              // [B*Hq, ldC] (position, order key): overflow of the last bucket
+  uint2 *cand;              // [B*Hq, ldC] (position, order key) of the keys in bin b1
   int32_t *idx;             // [B*Hq, k]
   long long ldS, ldC, N;
   long long cand_lo, cand_hi, nC, k_eff;
@@ -65,8 +66,9 @@ struct AttnParams {
   uint32_t *meta;
   long long ldS, cap, N;
   long long s1, w0, nW, k_eff;
-  int k, Hq, G, Hkv, nsplit, R;
-  int range;                // entries of U per CTA (multiple of 64, <= kMaxRange)
+  int k, Hq, G, Hkv, nsplit, R, B;
+  int nWsplit;              // static-set CTAs per KV head (64 rows of W each)
+  int nOsplit;              // retrieved-set CTAs per query head (64 rows of Omega each)
 };
 
 struct DenseParams {
@@ -89,15 +91,14 @@ struct AppendParams {
 
 // tuning constants the host layout needs
 constexpr int kScoreTile = 128;
-constexpr int kMaxRange = 2048;     // U entries per sparse-attention CTA, at most
-constexpr int kAttnTargetCtas = 1184;   // 8 CTAs per SM of a 148-SM B200: sizes the U ranges
-constexpr int kSelCluster = 8;      // CTAs per query head in the top-k select (one cluster)
+constexpr int kAttnRange = 64;      // entries of U per sparse-attention CTA
+constexpr int kTopkChunk = 8192;    // positions per top-k CTA
 constexpr int kDenseTile = 128;
 
 int num_sms();
 
 // Bytes of the counter block at the front of every workspace for `rows` query heads
-// (digit-1 histograms, then the per-row counters), 256-byte aligned sections.
+// (digit-1 and digit-2 histograms, then the per-row counters), 256-byte aligned sections.
 size_t counter_block_bytes(size_t rows);
 
 // Raises a kernel's dynamic shared-memory limit once per device (so that later launches,

@@ -40,8 +40,8 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
 }
 
 // Merges the nsplit states at prow (stride D + kPartPad) into out[0..D) with the whole block.
-// Loads are spread over (channel quad, split group) so that each thread issues few dependent
-// L2 round trips.  red: kThreads / 32 floats; buf: 4 * kThreads floats (16-byte aligned).
+// Two dependent L2 round trips: (m_S, Z_S) in one pass with a running max, then N_S with the
+// loads spread over (channel quad, split group).  red: kThreads / 32 floats; buf: 4 * kThreads floats (16-byte aligned).
 template <int D, int kThreads>
 __device__ __forceinline__ void merge_states(const float *prow, int nsplit, float *out, float *red,
                                              float *buf) {
@@ -49,13 +49,20 @@ __device__ __forceinline__ void merge_states(const float *prow, int nsplit, floa
   constexpr int kQuads = D / 4;
   constexpr int kGroups = kThreads / kQuads;
   const int tid = threadIdx.x;
-  float mm = -INFINITY;
-  for (int j = tid; j < nsplit; j += kThreads) mm = fmaxf(mm, __ldcg(prow + j * PS));
-  const float M = block_max<kThreads>(mm, red);
-  float dd = 0.f;
-  for (int j = tid; j < nsplit; j += kThreads)
-    dd += expf(__ldcg(prow + j * PS) - M) * __ldcg(prow + j * PS + 1);
-  const float den = block_sum<kThreads>(dd, red);
+  // one pass over (m_S, Z_S): each thread keeps a running (max, normaliser) of its states
+  float mt = -INFINITY, zt = 0.f;
+  for (int j = tid; j < nsplit; j += kThreads) {
+    const float m = __ldcg(prow + j * PS), z = __ldcg(prow + j * PS + 1);
+    if (m == -INFINITY) continue;   // an empty state contributes nothing
+    if (m > mt) {
+      zt = zt * expf(mt - m) + z;
+      mt = m;
+    } else {
+      zt += z * expf(m - mt);
+    }
+  }
+  const float M = block_max<kThreads>(mt, red);
+  const float den = block_sum<kThreads>(mt == -INFINITY ? 0.f : zt * expf(mt - M), red);
   const int cq = tid % kQuads, sg = tid / kQuads;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4

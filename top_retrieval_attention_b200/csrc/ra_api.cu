@@ -48,7 +48,7 @@ static constexpr size_t kAlign = 256;
 size_t counter_block_bytes(size_t rows) {
   const size_t h = (rows * kHistBins * 4 + kAlign - 1) / kAlign * kAlign;
   const size_t m = (rows * kMetaWords * 4 + kAlign - 1) / kAlign * kAlign;
-  return h + m;
+  return 2 * h + m;
 }
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 static long long round4(long long x) { return (x + 3) / 4 * 4; }
@@ -57,9 +57,9 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Derived sizes of one decode step (positions follow the slide "The GPU keeps 640 fixed
 // positions": W = [0, s1) u [w0, N), candidates C = [s1, w0)).
 struct Step {
-  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, range;
+  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, nWsplit, nOsplit;
   long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC;
-  size_t off_S, off_hist, off_meta, off_cand, off_part, total;
+  size_t off_S, off_hist, off_hist2, off_meta, off_cand, off_part, total;
 };
 
 static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
@@ -79,16 +79,13 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.k_eff = std::min<long long>(k, st.nC);
   st.ldS = round4(std::max<long long>(N, 1));
   st.ldC = round4(std::max<long long>(st.nC, 1));
-  // U ranges: enough CTAs for a few waves, each range a multiple of 64 entries
-  const long long nU = std::max<long long>(1, st.nW + st.k_eff);
-  const long long want = std::max<long long>(1, (kAttnTargetCtas + st.R - 1) / st.R);
-  long long range = (nU + want - 1) / want;
-  range = std::min<long long>(kMaxRange, std::max<long long>(64, (range + 63) / 64 * 64));
-  st.range = static_cast<int>(range);
-  st.nsplit = static_cast<int>((nU + range - 1) / range);
-  // counter block first (its offsets depend on B*Hq only), then the per-call arrays
+  // sparse attention splits: W in 64-row pieces per KV head, Omega in 64-row pieces per head
+  st.nWsplit = static_cast<int>((st.nW + kAttnRange - 1) / kAttnRange);
+  st.nOsplit = static_cast<int>((st.k_eff + kAttnRange - 1) / kAttnRange);
+  st.nsplit = std::max(1, st.nWsplit + st.nOsplit);
   size_t off = 0;
   st.off_hist = off;  off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
+  st.off_hist2 = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_meta = off;  off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
   st.off_S = off;     off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
   st.off_cand = off;  off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 8);
@@ -146,6 +143,7 @@ static ra_status run_topk(const Step &st, int32_t *idx, void *ws, cudaStream_t s
   TopkParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
   p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
+  p.hist2 = reinterpret_cast<uint32_t *>(at(ws, st.off_hist2));
   p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
   p.cand = reinterpret_cast<uint2 *>(at(ws, st.off_cand));
   p.idx = idx;
@@ -168,7 +166,7 @@ static ra_status run_attn(const ra_kv *kv, const Step &st, const int32_t *idx, f
   p.ldS = st.ldS; p.cap = st.cap; p.N = st.N;
   p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.k_eff = st.k_eff;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.nsplit = st.nsplit; p.R = st.R;
-  p.range = st.range;
+  p.B = st.B; p.nWsplit = st.nWsplit; p.nOsplit = st.nOsplit;
   cudaError_t e = launch_sparse_attn(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "sparse_attn");
 }
@@ -186,7 +184,7 @@ static int dense_nsplit_cap(long long N) {
 // Kernels leave it zero when they finish, so a workspace zero-filled once stays usable by
 // later calls with the same B * Hq (whatever N), sparse and dense alike.
 static size_t counter_bytes(int R, size_t *off_meta) {
-  const size_t m = align_up(static_cast<size_t>(R) * kHistBins * 4);
+  const size_t m = 2 * align_up(static_cast<size_t>(R) * kHistBins * 4);
   if (off_meta) *off_meta = m;
   return align_up(m + static_cast<size_t>(R) * kMetaWords * 4);
 }

@@ -2,12 +2,16 @@
 // renormalizes selected tokens", Eq. (2) with the selected set; "Two local softmax outputs
 // need global weights", Eqs. (3)-(5), and its backup slide, Appendix B).
 //
-// U is the virtual list [sinks, window, Omega].  It is cut into ranges of at most kMaxRange
-// entries, one CTA per (range, query head).  A CTA reads the already computed scores z of its
-// range (never K again), takes their max m_S, and gathers the V rows in sub-chunks of 64
-// entries, accumulating N_S = sum e^{z - m_S} v and Z_S = sum e^{z - m_S} in fp32.  The last
-// CTA of a head merges the partial states with the weights e^{m_S - m}, m = max_S m_S: the
-// exact softmax over U.
+// Two kinds of CTA, each covering at most 64 entries of the selected set:
+//   * static CTAs (one set per KV head): rows of W = sinks + window, shared by the G query
+//     heads of the KV head (slide "The GPU keeps 640 fixed positions"): each V row is
+//     gathered once and weighted for all G heads;
+//   * retrieved CTAs (one set per query head): rows of Omega, that head's top-k.
+// A warp takes 16 entries: their positions, scores z (already computed; K is never read
+// again) and V rows are loaded together, the warp reduces its own max m, sum Z and
+// N = sum e^{z - m} v with shuffles, and the CTA combines its four warps into one partial
+// state (m_S, Z_S, N_S).  The last CTA to finish a query head merges that head's partial states
+// with the weights e^{m_S - m}, m = max_S m_S: the exact softmax over U.
 #include <math.h>
 
 #include "common.cuh"
@@ -18,133 +22,188 @@ namespace ra {
 
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = kAttnThreads / 32;
-constexpr int kSub = 64;                // entries per gather sub-chunk (16 rows per warp)
+constexpr int kRowsPerWarp = kAttnRange / kAttnWarps;   // 16
 
-template <int D>
-__global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(const AttnParams p) {
-  constexpr int CPL = D / 32;                 // channels per lane in the gather
-  constexpr int RPW = kSub / kAttnWarps;      // rows per warp per sub-chunk
-  constexpr int PS = D + kPartPad;            // partial-state stride (floats)
-  const int split = blockIdx.x;
-  const int row = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = row / p.Hq;
-  const int h = row - b * p.Hq;
-  const int g = h / p.G;
-  const __nv_bfloat16 *Vh = p.V + (static_cast<long long>(b) * p.Hkv + g) * p.cap * D;
-  const float *srow = p.S + static_cast<long long>(row) * p.ldS;
-  const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
-
-  __shared__ int s_pos[kMaxRange];
-  __shared__ float s_p[kMaxRange];
-  __shared__ float s_red[kAttnWarps];
-  __shared__ __align__(16) float s_acc[4 * kAttnThreads];   // per-warp sums, then merge buffer
-  __shared__ bool s_last;
-
-  pdl_trigger();
-  pdl_wait();
-  const long long nU = p.nW + p.k_eff;
-  const long long e0 = static_cast<long long>(split) * p.range;
-  const int n = static_cast<int>(min(static_cast<long long>(p.range), nU - e0));
-
-  // positions and scores of this range; the range max
-  float mloc = -INFINITY;
-  for (int t = tid; t < n; t += kAttnThreads) {
-    const long long e = e0 + t;
-    int pos;
-    if (e < p.s1)
-      pos = static_cast<int>(e);
-    else if (e < p.nW)
-      pos = static_cast<int>(p.w0 + (e - p.s1));
-    else
-      pos = __ldg(irow + (e - p.nW));
-    if (pos < 0 || pos >= p.N) pos = -1;   // never for a completed selection
-    const float z = pos >= 0 ? __ldcg(srow + pos) : -INFINITY;
-    s_pos[t] = pos;
-    s_p[t] = z;
-    mloc = fmaxf(mloc, z);
-  }
-  const float m = block_max<kAttnThreads>(mloc, s_red);   // barrier: s_pos / s_p complete
-  float zsum = 0.f;
-  for (int t = tid; t < n; t += kAttnThreads) {
-    const float pe = s_pos[t] >= 0 ? expf(s_p[t] - m) : 0.f;
-    s_p[t] = pe;
-    zsum += pe;
-  }
-  const float Z = block_sum<kAttnThreads>(zsum, s_red);   // barrier: s_p holds the weights
-
-  float acc[CPL];
+// One warp: 16 entries (rows) at positions pos (lane j < 16 holds entry j, -1 when absent),
+// the scores of nh heads (z[h], lane j), V rows gathered 4 (d=128) or 2 (d=64) channels per
+// lane.  Produces per head the warp's max m, sum Z (lane-uniform) and acc (this lane's
+// channels).
+template <int D, int NH>
+__device__ __forceinline__ void warp_rows(const __nv_bfloat16 *Vh, int pos, const float (&z)[NH],
+                                          int nh, float (&m)[NH], float (&Zs)[NH],
+                                          float (&acc)[NH][D / 32]) {
+  constexpr int CPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  // V rows first: their loads overlap the reductions below
+  uint32_t w[kRowsPerWarp][CPL / 2];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-#pragma unroll 1
-  for (int sc = 0; sc < n; sc += kSub) {
-    if constexpr (CPL == 4) {
-      uint2 w[RPW];
-#pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int t = sc + warp + kAttnWarps * j;
-        const int ps = t < n ? s_pos[t] : -1;
-        w[j] = ps >= 0 ? __ldg(reinterpret_cast<const uint2 *>(Vh + static_cast<long long>(ps) * D) + lane)
-                       : make_uint2(0u, 0u);
-      }
-#pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int t = sc + warp + kAttnWarps * j;
-        const float pw = t < n ? s_p[t] : 0.f;
-        acc[0] += pw * bf16_lo(w[j].x);
-        acc[1] += pw * bf16_hi(w[j].x);
-        acc[2] += pw * bf16_lo(w[j].y);
-        acc[3] += pw * bf16_hi(w[j].y);
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    const int pj = __shfl_sync(0xffffffffu, pos, j);
+    if (pj >= 0) {
+      const __nv_bfloat16 *row = Vh + static_cast<long long>(pj) * D;
+      if constexpr (CPL == 4) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(row) + lane);
+        w[j][0] = v.x;
+        w[j][1] = v.y;
+      } else {
+        w[j][0] = __ldg(reinterpret_cast<const uint32_t *>(row) + lane);
       }
     } else {
-      uint32_t w[RPW];
 #pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int t = sc + warp + kAttnWarps * j;
-        const int ps = t < n ? s_pos[t] : -1;
-        w[j] = ps >= 0 ? __ldg(reinterpret_cast<const uint32_t *>(Vh + static_cast<long long>(ps) * D) + lane)
-                       : 0u;
-      }
-#pragma unroll
-      for (int j = 0; j < RPW; ++j) {
-        const int t = sc + warp + kAttnWarps * j;
-        const float pw = t < n ? s_p[t] : 0.f;
-        acc[0] += pw * bf16_lo(w[j]);
-        acc[1] += pw * bf16_hi(w[j]);
-      }
+      for (int c = 0; c < CPL / 2; ++c) w[j][c] = 0u;
     }
   }
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) s_acc[warp * D + lane * CPL + c] = acc[c];
-  __syncthreads();
-
-  float *part = p.part + (static_cast<long long>(row) * p.nsplit + split) * PS;
-  for (int c = tid; c < D; c += kAttnThreads)
-    part[kPartPad + c] = (s_acc[c] + s_acc[D + c]) + (s_acc[2 * D + c] + s_acc[3 * D + c]);
-  if (tid == 0) {
-    part[0] = m;
-    part[1] = Z;
+  for (int h = 0; h < NH; ++h) {
+    if (h >= nh) continue;
+    const float zz = (lane < kRowsPerWarp && pos >= 0) ? z[h] : -INFINITY;
+    float mh = zz;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, o));
+    mh = __shfl_sync(0xffffffffu, mh, 0);
+    const float pe = (lane < kRowsPerWarp && pos >= 0) ? expf(zz - mh) : 0.f;
+    float zs = pe;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+    m[h] = mh;
+    Zs[h] = __shfl_sync(0xffffffffu, zs, 0);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kRowsPerWarp; ++j) {
+      const float pj = __shfl_sync(0xffffffffu, pe, j);
+#pragma unroll
+      for (int c = 0; c < CPL / 2; ++c) {
+        acc[h][2 * c] += pj * bf16_lo(w[j][c]);
+        acc[h][2 * c + 1] += pj * bf16_hi(w[j][c]);
+      }
+    }
   }
-  // last-CTA hand-off: the barrier orders this CTA's partial-state stores before thread 0's
-  // release fence and counter update; the CTA that sees the final count acquires and merges
+}
+
+// Combines the four warps' states of one head (smem: m[4], Z[4], acc[4][D]) into a partial
+// state in global memory.
+template <int D>
+__device__ __forceinline__ void cta_combine(const float *wm, const float *wz, const float *wacc,
+                                            float *part) {
+  const float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+  float e[kAttnWarps];
+#pragma unroll
+  for (int i = 0; i < kAttnWarps; ++i) e[i] = wm[i] == -INFINITY ? 0.f : expf(wm[i] - M);
+  for (int c = threadIdx.x; c < D; c += kAttnThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kAttnWarps; ++i) s += e[i] * wacc[i * D + c];
+    part[kPartPad + c] = s;
+  }
+  if (threadIdx.x == 0) {
+    float zt = 0.f;
+#pragma unroll
+    for (int i = 0; i < kAttnWarps; ++i) zt += e[i] * wz[i];
+    part[0] = M;
+    part[1] = zt;
+  }
+}
+
+// Shared memory of one CTA: per-warp states of up to kMaxGroup heads, then the merge buffer.
+template <int D>
+struct AttnSmem {
+  float m[kMaxGroup][kAttnWarps];
+  float z[kMaxGroup][kAttnWarps];
+  __align__(16) float acc[kMaxGroup * kAttnWarps * D];
+  float red[kAttnWarps];
+  int last[kMaxGroup];
+};
+
+// The body for CTAs covering NH heads (NH = kMaxGroup for static CTAs, of which the first
+// nrows are real; NH = 1 for retrieved CTAs), all array indices compile-time.
+template <int D, int NH>
+__device__ __forceinline__ void attn_cta(const AttnParams &p, AttnSmem<D> &sm, int row0, int nrows,
+                                         int split, const __nv_bfloat16 *Vh, int pos,
+                                         const float (&z)[NH]) {
+  constexpr int CPL = D / 32;
+  constexpr int PS = D + kPartPad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float m[NH], Zs[NH], acc[NH][CPL];
+  warp_rows<D, NH>(Vh, pos, z, nrows, m, Zs, acc);
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    if (h < nrows) {
+      if (lane == 0) {
+        sm.m[h][warp] = m[h];
+        sm.z[h][warp] = Zs[h];
+      }
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) sm.acc[(h * kAttnWarps + warp) * D + lane * CPL + c] = acc[h][c];
+    }
+  }
   __syncthreads();
-  if (tid == 0) {
+  for (int h = 0; h < nrows; ++h)
+    cta_combine<D>(sm.m[h], sm.z[h], sm.acc + h * kAttnWarps * D,
+                   p.part + (static_cast<long long>(row0 + h) * p.nsplit + split) * PS);
+
+  // last-CTA hand-off per query head: the barrier orders this CTA's partial-state stores
+  // before the release fence and counter update; a CTA that completes a head merges it
+  __syncthreads();
+  if (tid < nrows) {
     __threadfence();
-    const uint32_t prev = atomicAdd(p.meta + row * kMetaWords + kDone, 1u);
-    s_last = prev == static_cast<uint32_t>(p.nsplit - 1);
-    if (s_last) __threadfence();
+    const uint32_t prev = atomicAdd(p.meta + (row0 + tid) * kMetaWords + kDone, 1u);
+    sm.last[tid] = prev == static_cast<uint32_t>(p.nsplit - 1);
+    if (sm.last[tid]) __threadfence();
   }
   __syncthreads();
-  if (!s_last) return;
+  for (int h = 0; h < nrows; ++h) {
+    if (!sm.last[h]) continue;   // uniform: shared flag
+    const int row = row0 + h;
+    merge_states<D, kAttnThreads>(p.part + static_cast<long long>(row) * p.nsplit * PS, p.nsplit,
+                                  p.out + static_cast<long long>(row) * D, sm.red, sm.acc);
+    if (tid == 0) p.meta[row * kMetaWords + kDone] = 0u;
+  }
+}
 
-  // merge the partial states of all ranges of this query head (Eqs. (3)-(5))
-  merge_states<D, kAttnThreads>(p.part + static_cast<long long>(row) * p.nsplit * PS, p.nsplit,
-                                p.out + static_cast<long long>(row) * D, s_red, s_acc);
-  if (tid == 0) p.meta[row * kMetaWords + kDone] = 0u;
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 6) sparse_attn_kernel(const AttnParams p) {
+  __shared__ AttnSmem<D> sm;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_trigger();
+  pdl_wait();
+  const long long n_static_ctas = static_cast<long long>(p.B) * p.Hkv * p.nWsplit;
+  if (blockIdx.x < n_static_ctas) {
+    const int grp = static_cast<int>(blockIdx.x / p.nWsplit);        // b * Hkv + g
+    const int s = static_cast<int>(blockIdx.x - static_cast<long long>(grp) * p.nWsplit);
+    const int b = grp / p.Hkv, g = grp - b * p.Hkv;
+    const int row0 = b * p.Hq + g * p.G;
+    const long long e = static_cast<long long>(s) * kAttnRange + warp * kRowsPerWarp + lane;
+    int pos = -1;
+    if (lane < kRowsPerWarp && e < p.nW) pos = static_cast<int>(e < p.s1 ? e : p.w0 + (e - p.s1));
+    float z[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h)
+      z[h] = (h < p.G && pos >= 0) ? __ldcg(p.S + (row0 + h) * p.ldS + pos) : -INFINITY;
+    attn_cta<D, kMaxGroup>(p, sm, row0, p.G, s, p.V + static_cast<long long>(grp) * p.cap * D,
+                           pos, z);
+  } else {
+    const long long id = blockIdx.x - n_static_ctas;
+    const int row = static_cast<int>(id / p.nOsplit);
+    const int s = static_cast<int>(id - static_cast<long long>(row) * p.nOsplit);
+    const int b = row / p.Hq, h = row - b * p.Hq;
+    const long long e = static_cast<long long>(s) * kAttnRange + warp * kRowsPerWarp + lane;
+    int pos = -1;
+    if (lane < kRowsPerWarp && e < p.k_eff) {
+      pos = __ldg(p.idx + static_cast<long long>(row) * p.k + e);
+      if (pos < 0 || pos >= p.N) pos = -1;   // never for a completed selection
+    }
+    float z[1];
+    z[0] = pos >= 0 ? __ldcg(p.S + row * p.ldS + pos) : -INFINITY;
+    attn_cta<D, 1>(p, sm, row, 1, p.nWsplit + s,
+                   p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D, pos, z);
+  }
 }
 
 cudaError_t launch_sparse_attn(const AttnParams &p, int d, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.R));
+  const long long ctas = static_cast<long long>(p.B) * p.Hkv * p.nWsplit +
+                         static_cast<long long>(p.R) * p.nOsplit;
+  const dim3 grid(static_cast<unsigned>(ctas));
   return d == 128 ? launch_pdl(sparse_attn_kernel<128>, grid, dim3(kAttnThreads), 0, s, p)
                   : launch_pdl(sparse_attn_kernel<64>, grid, dim3(kAttnThreads), 0, s, p);
 }

@@ -4,41 +4,32 @@
 //
 // Keys are compared as 64-bit composites (order_key(z) << 32 | ~position), so every key is
 // distinct, larger z wins and equal z goes to the lower position.  The selection is a radix
-// select over digits of the composite, done for each query head by one thread-block cluster
-// of kSelCluster CTAs, each owning a contiguous slice of the positions:
-//   1. digit 1 = the top 11 bits of order_key(z): its histogram comes from the score kernel;
-//      every CTA finds the threshold bin b1 (the bin holding the k-th largest key);
-//   2. every CTA reads its slice of z (keeping the keys in shared memory when they fit) and
-//      histograms digit 2 (the next 11 bits) of its keys in bin b1; the CTAs add up the
-//      cluster's histograms through distributed shared memory and find the bin b2;
-//   3. keys above (b1, b2) are selected and written out in rounds, each round reserving its
-//      output range with one atomic; keys in (b1, b2) go to a bucket in the shared memory of
-//      the cluster's first CTA (or, if it overflows, to a global list);
-//   4. the first CTA narrows the bucket with further 8-bit digits until it is taken whole or
-//      holds at most 64 keys, which one warp sorts with a bitonic network.
-#include <cooperative_groups.h>
+// select over digits of the composite, in one kernel over (head, chunk) CTAs:
+//   * digit 1 = the top 11 bits of order_key(z), histogrammed by the score kernel; every CTA
+//     finds the threshold bin b1 (the bin holding the k-th largest key);
+//   * keys above b1 are written out and keys in b1 listed (position and key): each thread
+//     counts its keys, one block scan places them, and each CTA reserves its output ranges
+//     with one atomic per list;
+//   * the listed keys are also histogrammed by digit 2 (the next 11 bits); the last CTA of a
+//     head finds the digit-2 threshold bin b2, emits the listed keys above (b1, b2) in one
+//     pass and narrows the (b1, b2) bucket with further 8-bit digits until it is taken whole
+//     or holds at most 64 keys, which one warp sorts with a bitonic network.
+// A digit-1 bin is a range of z (order_key is monotone), so the per-key test is a pair of
+// float comparisons.  The histogram and counters are left zero for the next call.
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
 
-namespace cg = cooperative_groups;
-
 namespace ra {
 
-constexpr int kSelThreads = 512;
-constexpr int kKeyCache = 16384;     // keys of a slice kept in shared memory (64 KB)
-constexpr int kRound = 2048;         // positions per emission round
-constexpr int kBucketCap = 4096;     // (b1, b2) bucket held in shared memory (32 KB)
+constexpr int kTkThreads = 256;
+constexpr int kBucketCap = 4096;     // bucket held in shared memory by the tail (32 KB)
 constexpr int kBitonic = 64;
 constexpr int kDigit2Shift = 10;     // digit 2 = bits [10, 21) of the order key
+constexpr int kPerThread = kTopkChunk / kTkThreads;   // 32 keys per thread
+constexpr int kVec = kPerThread / 4;                  // float4 loads per thread
 
-struct SelectSmem {
-  uint32_t keys[kKeyCache];
-  uint64_t bucket[kBucketCap];
-  uint32_t h2[kHistBins];
-  uint32_t list[kRound];
-};
 
 __device__ __forceinline__ uint64_t make_composite(uint32_t key, uint32_t pos) {
   return (static_cast<uint64_t>(key) << 32) | (0xFFFFFFFFu - pos);
@@ -73,16 +64,24 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t *warp_t
   return r;
 }
 
-// Finds, in a histogram owned kPer bins per thread from the top (loc[0] = highest bin of this
-// thread, thread 0 owns the highest bins), the bin holding the `want`-th largest element.
-// Exactly one thread writes *bin_out, *above_out (elements in higher bins) and *cnt_out.
-template <int kThreads, int kPer>
-__device__ __forceinline__ void find_threshold(const uint32_t (&loc)[kPer], uint32_t want,
-                                               uint32_t *warp_tot, int *bin_out,
-                                               uint32_t *above_out, uint32_t *cnt_out) {
+// Threshold bin of a 2048-bin histogram h (global, read through L2): the bin holding the
+// `want`-th largest element, the count above it and its own count.  Whole block, one result
+// in shared memory (valid after the call).
+struct Thresh {
+  int bin;
+  uint32_t above, cnt;
+};
+template <int kThreads>
+__device__ __forceinline__ Thresh find_threshold(const uint32_t *h, uint32_t want,
+                                                 uint32_t *warp_tot, Thresh *out) {
+  constexpr int kPer = kHistBins / kThreads;
+  uint32_t loc[kPer];   // loc[0] = highest bin of this thread; thread 0 owns the highest bins
   uint32_t s = 0;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) s += loc[i];
+  for (int i = 0; i < kPer; ++i) {
+    loc[i] = __ldcg(h + kHistBins - kPer * (threadIdx.x + 1) + (kPer - 1 - i));
+    s += loc[i];
+  }
   const uint32_t incl = block_incl_scan<kThreads>(s, warp_tot);
   const uint32_t excl = incl - s;
   if (excl < want && want <= incl) {
@@ -90,210 +89,231 @@ __device__ __forceinline__ void find_threshold(const uint32_t (&loc)[kPer], uint
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       if (cum + loc[i] >= want) {
-        *bin_out = kHistBins - kPer * (static_cast<int>(threadIdx.x) + 1) + (kPer - 1 - i);
-        *above_out = cum;
-        *cnt_out = loc[i];
+        out->bin = kHistBins - kPer * (static_cast<int>(threadIdx.x) + 1) + (kPer - 1 - i);
+        out->above = cum;
+        out->cnt = loc[i];
         break;
       }
       cum += loc[i];
     }
   }
+  __syncthreads();
+  return *out;
 }
 
-__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
-    topk_select_kernel(const TopkParams p) {
-  constexpr int kPer = kHistBins / kSelThreads;   // 4 histogram bins per thread
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  SelectSmem &sm = *reinterpret_cast<SelectSmem *>(smem_raw);
-  __shared__ uint32_t warp_tot[kSelThreads / 32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above, s_cnt;
-  __shared__ uint32_t s_nlist, s_base, s_bucket_n, s_out;
-  __shared__ uint32_t h256[256];
-  __shared__ uint64_t bs[kBitonic];
+// The float whose order key is `key` (order_key is a bijection on bit patterns and monotone,
+// so key(z) >= key  <=>  z >= key_float(key) for the finite keys used as thresholds here).
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const unsigned rank = cluster.block_rank();
-  const int row = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// This CTA's chunk of z (kPerThread values per thread, all loads in flight).  Element j of a
+// thread is chunk offset off(j) = 4 * ((j / 4) * kTkThreads + tid) + j % 4.
+__device__ __forceinline__ void load_chunk(const float *src, int l0, int l1, float (&z)[kPerThread]) {
+#pragma unroll
+  for (int u = 0; u < kVec; ++u) {
+    const int i = 4 * (u * kTkThreads + static_cast<int>(threadIdx.x));
+    const float4 v = (i + 3 >= l0 && i < l1) ? __ldcg(reinterpret_cast<const float4 *>(src + i))
+                                             : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    z[4 * u] = v.x;
+    z[4 * u + 1] = v.y;
+    z[4 * u + 2] = v.z;
+    z[4 * u + 3] = v.w;
+  }
+}
+__device__ __forceinline__ int chunk_off(int j) {
+  return 4 * ((j / 4) * kTkThreads + static_cast<int>(threadIdx.x)) + (j & 3);
+}
+
+// Last-CTA hand-off per head: after this CTA's global writes, count it in; true for the CTA
+// that completes the head (it then sees every other CTA's writes).
+__device__ __forceinline__ bool last_of_row(uint32_t *counter, uint32_t total, bool *s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t prev = atomicAdd(counter, 1u);
+    *s_flag = prev == total - 1;
+    if (*s_flag) {
+      __threadfence();
+      *counter = 0u;   // left zero for the next kernel that counts with it
+    }
+  }
+  __syncthreads();
+  return *s_flag;
+}
+
+// ---- one pass per (head, chunk): keys above the digit-1 threshold bin b1 are emitted, keys
+//      in b1 are listed with their order keys; the head's last CTA selects the rest from
+//      that list and leaves the histogram and counters zero
+__global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkParams p) {
+  __shared__ __align__(16) uint64_t bucket[kBucketCap];   // the last CTA's (b1, b2) bucket
+  __shared__ uint32_t warp_tot[kTkThreads / 32];
+  __shared__ Thresh s_t;
+  __shared__ uint32_t h2[kHistBins];      // digit-2 histogram of this CTA's listed keys
+  __shared__ uint64_t bs[kBitonic];
+  __shared__ uint32_t s_ns, s_nc, s_bs, s_bc, s_out, s_cnt, s_cum, s_nb;
+  __shared__ int s_digit;
+  __shared__ bool s_last;
+  uint32_t *h256 = h2;                    // the last CTA's 8-bit digit histogram
   pdl_trigger();
   pdl_wait();
-
+  const int row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
-  uint32_t *meta = p.meta + row * kMetaWords;
-  if (rank == 0)
-    for (long long i = p.k_eff + tid; i < p.k; i += kSelThreads) irow[i] = -1;
-  if (p.k_eff == 0) return;   // uniform over the cluster: no cluster barrier is reached
-
-  // this CTA's slice of the candidates
-  const long long part = ((p.N + kSelCluster - 1) / kSelCluster + 3) & ~3LL;
-  long long lo = static_cast<long long>(rank) * part, hi = lo + part;
-  if (lo < p.cand_lo) lo = p.cand_lo;
-  if (hi > p.cand_hi) hi = p.cand_hi;
-  const int n_my = hi > lo ? static_cast<int>(hi - lo) : 0;
-  const bool cached = n_my <= kKeyCache;
-  const float *srow = p.S + static_cast<long long>(row) * p.ldS + lo;
+  if (blockIdx.x == 0)
+    for (long long i = p.k_eff + tid; i < p.k; i += kTkThreads) irow[i] = -1;
+  if (p.k_eff == 0) return;
+  const long long c0 = static_cast<long long>(blockIdx.x) * kTopkChunk;
+  const int l0 = static_cast<int>(max(c0, p.cand_lo) - c0);
+  const int l1 = static_cast<int>(min(c0 + kTopkChunk, p.cand_hi) - c0);
+  if (l0 >= l1) return;
   const bool take_all = p.k_eff >= p.nC;
-
-  // ---- 1. digit-1 threshold (every CTA, from the score kernel's histogram)
+  // the chunk's loads go out first and are in flight while the threshold is found
+  float z[kPerThread];
+  load_chunk(p.S + static_cast<long long>(row) * p.ldS + c0, l0, l1, z);
+  uint32_t *meta = p.meta + row * kMetaWords;
+  uint32_t *h1g = p.hist + static_cast<long long>(row) * kHistBins;
   int b1 = -1;
-  uint32_t above1 = 0;
+  float zlo = -INFINITY, zhi = -INFINITY;   // emit z >= zhi; list zlo <= z < zhi
   if (!take_all) {
-    const uint32_t *h = p.hist + static_cast<long long>(row) * kHistBins;
-    uint32_t loc[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) loc[i] = __ldcg(h + kHistBins - kPer * (tid + 1) + (kPer - 1 - i));
-    find_threshold<kSelThreads, kPer>(loc, static_cast<uint32_t>(p.k_eff), warp_tot, &s_bin,
-                                      &s_above, &s_cnt);
+    const Thresh t1 = find_threshold<kTkThreads>(h1g, static_cast<uint32_t>(p.k_eff), warp_tot, &s_t);
+    b1 = t1.bin;
+    zlo = key_float(static_cast<uint32_t>(b1) << (32 - kHistBits));
+    zhi = b1 + 1 < kHistBins ? key_float(static_cast<uint32_t>(b1 + 1) << (32 - kHistBits)) : INFINITY;
   }
-  for (int i = tid; i < kHistBins; i += kSelThreads) sm.h2[i] = 0;
-  if (tid == 0) {
-    s_nlist = 0;
-    s_bucket_n = 0;
+  for (int i = tid; i < kHistBins; i += kTkThreads) h2[i] = 0;
+  const bool edge = l0 > 0 || l1 < kTopkChunk;
+  uint2 *crow = p.cand + static_cast<long long>(row) * p.ldC;
+  // count this thread's selected (z >= zhi) and listed (zlo <= z < zhi) keys ...
+  uint32_t ns = 0, nc = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThread; ++j) {
+    bool in = true;
+    if (edge) in = chunk_off(j) >= l0 && chunk_off(j) < l1;
+    ns += (in && z[j] >= zhi) ? 1u : 0u;
+    nc += (in && z[j] >= zlo && z[j] < zhi) ? 1u : 0u;
+  }
+  // ... place them with one block scan and one global reservation per list ...
+  const uint32_t packed = ns | (nc << 16);   // at most kPerThread each
+  const uint32_t incl = block_incl_scan<kTkThreads>(packed, warp_tot);
+  if (tid == kTkThreads - 1) {
+    s_ns = incl & 0xFFFFu;
+    s_nc = incl >> 16;
+    s_bs = s_ns ? atomicAdd(meta + kSelCount, s_ns) : 0u;
+    s_bc = s_nc ? atomicAdd(meta + kCandCount, s_nc) : 0u;
   }
   __syncthreads();
-  if (!take_all) {
-    b1 = s_bin;
-    above1 = s_above;
-  }
-
-  // ---- 2. keys of the slice (cached when they fit) and their digit-2 histogram in bin b1
-  constexpr int kLd = 8;
-  for (int i0 = 0; i0 < n_my; i0 += kLd * kSelThreads) {
-    float zb[kLd];
+  uint32_t os = s_bs + ((incl - packed) & 0xFFFFu);
+  uint32_t oc = s_bc + ((incl - packed) >> 16);
+  // ... and write them
+  bool any_cand = false;
+  if (ns | nc) {
 #pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int i = i0 + u * kSelThreads + tid;
-      zb[u] = i < n_my ? __ldcg(srow + i) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int i = i0 + u * kSelThreads + tid;
-      if (i < n_my) {
-        const uint32_t key = order_key(zb[u]);
-        if (cached) sm.keys[i] = key;
-        if (!take_all && static_cast<int>(key >> (32 - kHistBits)) == b1)
-          atomicAdd(&sm.h2[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+    for (int j = 0; j < kPerThread; ++j) {
+      bool in = true;
+      if (edge) in = chunk_off(j) >= l0 && chunk_off(j) < l1;
+      const uint32_t pos = static_cast<uint32_t>(c0 + chunk_off(j));
+      if (in && z[j] >= zhi) {
+        if (os < p.k_eff) irow[os] = static_cast<int32_t>(pos);
+        ++os;
+      } else if (in && z[j] >= zlo) {
+        const uint32_t key = order_key(z[j]);
+        if (oc < p.ldC) crow[oc] = make_uint2(pos, key);
+        ++oc;
+        atomicAdd(&h2[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+        any_cand = true;
       }
     }
   }
-  cluster.sync();   // every slice's digit-2 histogram is complete; digit-1 histogram read
+  uint32_t *h2g = p.hist2 + static_cast<long long>(row) * kHistBins;
+  if (__syncthreads_or(any_cand))
+    for (int i = tid; i < kHistBins; i += kTkThreads)
+      if (h2[i]) atomicAdd(h2g + i, h2[i]);
 
-  // ---- digit-2 threshold over the cluster's summed histograms
-  uint32_t b2 = 0, above2 = 0, cnt2 = 0, rr = 0;
-  if (!take_all) {
-    if (rank == 0)   // leave the digit-1 histogram zero for the next call
-      for (int i = tid; i < kHistBins; i += kSelThreads)
-        p.hist[static_cast<long long>(row) * kHistBins + i] = 0u;
-    uint32_t loc2[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) loc2[i] = 0;
-    for (int r = 0; r < kSelCluster; ++r) {
-      const uint32_t *rh = cluster.map_shared_rank(sm.h2, r);
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) loc2[i] += rh[kHistBins - kPer * (tid + 1) + (kPer - 1 - i)];
-    }
-    rr = static_cast<uint32_t>(p.k_eff) - above1;
-    find_threshold<kSelThreads, kPer>(loc2, rr, warp_tot, &s_bin, &s_above, &s_cnt);
-    __syncthreads();
-    b2 = static_cast<uint32_t>(s_bin);
-    above2 = s_above;
-    cnt2 = s_cnt;
-  }
-  const bool bucket_in_smem = cnt2 <= static_cast<uint32_t>(kBucketCap);
-  uint64_t *bucket0 = cluster.map_shared_rank(sm.bucket, 0);
-  uint32_t *bucket0_n = cluster.map_shared_rank(&s_bucket_n, 0);
-
-  // ---- 3. emit the keys above (b1, b2); route (b1, b2) keys to the bucket
-  constexpr int kPerRound = kRound / kSelThreads;   // 4 positions per thread per round
-  for (int r0 = 0; r0 < n_my; r0 += kRound) {
-    uint32_t kb[kPerRound];
-#pragma unroll
-    for (int u = 0; u < kPerRound; ++u) {   // all loads of the round in flight together
-      const int i = r0 + u * kSelThreads + tid;
-      kb[u] = i < n_my ? (cached ? sm.keys[i] : order_key(__ldcg(srow + i))) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < kPerRound; ++u) {
-      const int i = r0 + u * kSelThreads + tid;   // warp-uniform trip count: lanes differ by 1
-      const bool in = i < n_my;
-      const uint32_t key = kb[u];
-      const int bin = static_cast<int>(key >> (32 - kHistBits));
-      const uint32_t d2 = (key >> kDigit2Shift) & (kHistBins - 1);
-      const bool sel = in && (take_all || bin > b1 || (bin == b1 && d2 > b2));
-      const bool buck = in && !take_all && bin == b1 && d2 == b2;
-      bool ok;
-      const uint32_t o = warp_append(sel, &s_nlist, ok);
-      if (ok) sm.list[o] = static_cast<uint32_t>(lo + i);
-      if (buck) {
-        const uint32_t pos = static_cast<uint32_t>(lo + i);
-        if (bucket_in_smem) {
-          const uint32_t b = atomicAdd(bucket0_n, 1u);
-          if (b < static_cast<uint32_t>(kBucketCap)) bucket0[b] = make_composite(key, pos);
-        } else {
-          const uint32_t b = atomicAdd(meta + kCandCount, 1u);
-          if (b < p.ldC) p.cand[static_cast<long long>(row) * p.ldC + b] = make_uint2(pos, key);
-        }
-      }
-    }
-    __syncthreads();
-    const uint32_t n = s_nlist;
-    if (tid == 0 && n) s_base = atomicAdd(meta + kSelCount, n);
-    __syncthreads();
-    for (uint32_t i = tid; i < n; i += kSelThreads) {
-      const uint32_t o = s_base + i;
-      if (o < p.k_eff) irow[o] = static_cast<int32_t>(sm.list[i]);
-    }
-    __syncthreads();
-    if (tid == 0) s_nlist = 0;
-    __syncthreads();
-  }
-  cluster.sync();   // all emissions and bucket entries are in place
-  if (rank != 0) return;
-  if (tid == 0) meta[kSelCount] = 0u;
-  if (take_all) return;
-
-  // ---- 4. the first CTA selects the remaining rr2 keys from the (b1, b2) bucket
-  uint32_t rr2 = rr - above2;                       // 1 <= rr2 <= cnt2
-  const uint32_t out0 = static_cast<uint32_t>(p.k_eff) - rr2;
-  const uint32_t n_list = bucket_in_smem ? cnt2 : min(cnt2, static_cast<uint32_t>(p.ldC));
-  const uint2 *crow = p.cand + static_cast<long long>(row) * p.ldC;
-  auto get = [&](uint32_t i) -> uint64_t {
-    if (bucket_in_smem) return sm.bucket[i];
-    const uint2 c = __ldcg(&crow[i]);
-    return make_composite(c.y, c.x);
-  };
-  if (tid == 0) s_out = out0;
+  const uint32_t parts = static_cast<uint32_t>((p.cand_hi - 1) / kTopkChunk - p.cand_lo / kTopkChunk + 1);
+  if (!last_of_row(meta + kDone, parts, &s_last)) return;
+  // ---- the head's last CTA: the remaining rr keys come from the bin-b1 list
+  const uint32_t above = __ldcg(meta + kSelCount);
+  const uint32_t n_list = min(__ldcg(meta + kCandCount), static_cast<uint32_t>(p.ldC));
   __syncthreads();
-  if (tid == 0) meta[kCandCount] = 0u;
+  if (tid < kError) meta[tid] = 0u;
+  if (take_all) return;   // nothing was histogrammed or listed
+  if (above >= p.k_eff || n_list == 0) {   // counters not from this call
+    for (int i = tid; i < kHistBins; i += kTkThreads) {
+      h1g[i] = 0u;
+      h2g[i] = 0u;
+    }
+    return;
+  }
+  uint32_t rr = static_cast<uint32_t>(p.k_eff) - above;   // 1 <= rr <= n_list
+  if (tid == 0) s_out = above;
   auto emit = [&](bool pred, uint32_t pos) {
     bool ok;
     const uint32_t o = warp_append(pred, &s_out, ok);
     if (ok && o < p.k_eff) irow[o] = static_cast<int32_t>(pos);
   };
   const uint32_t wbase = static_cast<uint32_t>(tid - lane);
+  // digit 2 over the complete list: threshold bin b2; one batched pass emits the keys above
+  // (b1, b2) and gathers the (b1, b2) bucket into shared memory
+  const Thresh t2 = find_threshold<kTkThreads>(h2g, rr, warp_tot, &s_t);
+  for (int i = tid; i < kHistBins; i += kTkThreads) {
+    h1g[i] = 0u;
+    h2g[i] = 0u;
+  }
+  const uint32_t b2 = static_cast<uint32_t>(t2.bin);
+  rr -= t2.above;
+  const uint32_t cnt2 = t2.cnt;                           // 1 <= rr <= cnt2
+  const bool in_smem = cnt2 <= static_cast<uint32_t>(kBucketCap);
+  if (tid == 0) s_nb = 0;
+  __syncthreads();
+  constexpr int kBatch = 16;
+  for (uint32_t i0 = wbase; i0 < n_list; i0 += kBatch * kTkThreads) {
+    uint2 cb[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const uint32_t i = i0 + u * kTkThreads + lane;
+      cb[u] = i < n_list ? __ldcg(&crow[i]) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const uint32_t i = i0 + u * kTkThreads + lane;
+      const uint32_t d2 = (cb[u].y >> kDigit2Shift) & (kHistBins - 1);
+      emit(i < n_list && d2 > b2, cb[u].x);
+      bool ok;
+      const uint32_t o = warp_append(i < n_list && d2 == b2 && in_smem, &s_nb, ok);
+      if (ok && o < static_cast<uint32_t>(kBucketCap)) bucket[o] = make_composite(cb[u].y, cb[u].x);
+    }
+  }
+  __syncthreads();
+  // the (b1, b2) bucket: in shared memory, or (all keys alike) over the stored list
+  const uint32_t n_buck = in_smem ? cnt2 : n_list;
+  auto get = [&](uint32_t i) -> uint64_t {
+    if (in_smem) return bucket[i];
+    const uint2 c = __ldcg(&crow[i]);
+    return make_composite(c.y, c.x);
+  };
   uint64_t prefix = (static_cast<uint64_t>(b1) << kHistBits) | b2;
   int shift = 64 - 2 * kHistBits;
   uint32_t cnt = cnt2;
   // every round fixes 8 more bits of a unique 64-bit key: at most ceil(42 / 8) + 1 rounds
 #pragma unroll 1
   for (int round = 0; round < 8; ++round) {
-    if (cnt == rr2) {   // the whole bucket is taken
-      for (uint32_t i0 = wbase; i0 < n_list; i0 += kSelThreads) {
+    if (cnt == rr) {   // the whole bucket is taken
+      for (uint32_t i0 = wbase; i0 < n_buck; i0 += kTkThreads) {
         const uint32_t i = i0 + lane;
-        const uint64_t x = i < n_list ? get(i) : 0ull;
-        emit(i < n_list && (x >> shift) == prefix, comp_pos(x));
+        const uint64_t x = i < n_buck ? get(i) : 0ull;
+        emit(i < n_buck && (x >> shift) == prefix, comp_pos(x));
       }
       return;
     }
     if (cnt <= kBitonic) {   // bitonic finish of the threshold bucket
       if (tid < kBitonic) bs[tid] = 0;
-      if (tid == 0) s_bucket_n = 0;
+      if (tid == 0) s_nb = 0;
       __syncthreads();
-      for (uint32_t i = tid; i < n_list; i += kSelThreads) {
+      for (uint32_t i = tid; i < n_buck; i += kTkThreads) {
         const uint64_t x = get(i);
         if ((x >> shift) == prefix) {
-          const uint32_t o = atomicAdd(&s_bucket_n, 1u);
+          const uint32_t o = atomicAdd(&s_nb, 1u);
           if (o < kBitonic) bs[o] = x;
         }
       }
@@ -315,7 +335,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
           }
         }
         const uint32_t o0 = s_out;
-        for (uint32_t i = lane; i < rr2 && o0 + i < p.k_eff; i += 32)
+        for (uint32_t i = lane; i < rr && o0 + i < p.k_eff; i += 32)
           irow[o0 + i] = static_cast<int32_t>(comp_pos(bs[i]));
       }
       return;
@@ -324,34 +344,34 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
     const int nshift = shift > 8 ? shift - 8 : 0;
     const int nb = shift - nshift;
     const uint64_t dmask = (1ull << nb) - 1;
-    if (tid < 256) h256[tid] = 0;
+    h256[tid] = 0;
     __syncthreads();
-    for (uint32_t i = tid; i < n_list; i += kSelThreads) {
+    for (uint32_t i = tid; i < n_buck; i += kTkThreads) {
       const uint64_t x = get(i);
       if ((x >> shift) == prefix) atomicAdd(&h256[(x >> nshift) & dmask], 1u);
     }
     __syncthreads();
     if (warp == 0) {
       // lane l owns digits [256 - 8(l+1), 256 - 8l), highest first
-      uint32_t lc[8], s = 0;
+      uint32_t lc[8], sum = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         lc[i] = h256[255 - 8 * lane - i];
-        s += lc[i];
+        sum += lc[i];
       }
-      uint32_t incl = s;
+      uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+        const uint32_t nn = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += nn;
       }
-      const uint32_t excl = incl - s;
-      if (excl < rr2 && rr2 <= incl) {
+      const uint32_t excl = incl - sum;
+      if (excl < rr && rr <= incl) {
         uint32_t cum = excl;
         for (int i = 0; i < 8; ++i) {
-          if (cum + lc[i] >= rr2) {
-            s_bin = 255 - 8 * lane - i;
-            s_above = cum;
+          if (cum + lc[i] >= rr) {
+            s_digit = 255 - 8 * lane - i;
+            s_cum = cum;
             s_cnt = lc[i];
             break;
           }
@@ -360,14 +380,14 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
       }
     }
     __syncthreads();
-    const uint64_t v = static_cast<uint64_t>(s_bin);
-    const uint32_t cum = s_above;
-    for (uint32_t i0 = wbase; i0 < n_list; i0 += kSelThreads) {
+    const uint64_t v = static_cast<uint64_t>(s_digit);
+    const uint32_t cum = s_cum;
+    for (uint32_t i0 = wbase; i0 < n_buck; i0 += kTkThreads) {
       const uint32_t i = i0 + lane;
-      const uint64_t x = i < n_list ? get(i) : 0ull;
-      emit(i < n_list && (x >> shift) == prefix && ((x >> nshift) & dmask) > v, comp_pos(x));
+      const uint64_t x = i < n_buck ? get(i) : 0ull;
+      emit(i < n_buck && (x >> shift) == prefix && ((x >> nshift) & dmask) > v, comp_pos(x));
     }
-    rr2 -= cum;
+    rr -= cum;
     cnt = s_cnt;
     prefix = (prefix << nb) | v;
     shift = nshift;
@@ -378,13 +398,9 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
 
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
   if (p.k <= 0) return cudaSuccess;
-  static bool done[64] = {};
-  const size_t smem = sizeof(SelectSmem);
-  const cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(topk_select_kernel),
-                                          static_cast<int>(smem), done);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(topk_select_kernel, dim3(kSelCluster, static_cast<unsigned>(p.R)),
-                    dim3(kSelThreads), smem, s, p);
+  const long long chunks = (p.N + kTopkChunk - 1) / kTopkChunk;
+  const dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(p.R));
+  return launch_pdl(topk_collect_kernel, grid, dim3(kTkThreads), 0, s, p);
 }
 
 }  // namespace ra
