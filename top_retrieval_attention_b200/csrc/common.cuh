@@ -13,7 +13,8 @@ constexpr int kMaxGroup = 8;                  // query heads per KV head (one n8
 constexpr int kMetaWords = 8;                 // per-row counters in the workspace
 
 // per-row counters (uint32) in the workspace's meta block
-enum MetaSlot { kSelCount = 0, kCandCount = 1, kError = 6, kDone = 7 };
+enum MetaSlot { kSelCount = 0, kCandCount = 1, kBuckCount = 2, kThresh1 = 3, kAbove1 = 4,
+                kError = 6, kDone = 7 };
 // kDone is shared by the sparse and the dense merge (each leaves it zero).
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -51,6 +51,7 @@ struct TopkParams {
   uint32_t *hist2;          // [B*Hq, kHistBins] digit-2 histogram of the listed keys (same)
   uint32_t *meta;           // [B*Hq, kMetaWords] counters (left zero by the select)
   uint2 *cand;              // [B*Hq, ldC] (position, order key) of the keys in bin b1
+  uint2 *bucket;            // [B*Hq, kTopkBucket] the keys in (b1, b2)
   int32_t *idx;             // [B*Hq, k]
   long long ldS, ldC, N;
   long long cand_lo, cand_hi, nC, k_eff;
@@ -67,8 +68,9 @@ struct AttnParams {
   long long ldS, cap, N;
   long long s1, w0, nW, k_eff;
   int k, Hq, G, Hkv, nsplit, R, B;
-  int nWsplit;              // static-set CTAs per KV head (64 rows of W each)
-  int nOsplit;              // retrieved-set CTAs per query head (64 rows of Omega each)
+  int nWsplit;              // static-set CTAs per KV head, wrange rows of W each
+  int nOsplit;              // retrieved-set CTAs per query head, orange rows of Omega each
+  long long wrange, orange; // multiples of kAttnRange
 };
 
 struct DenseParams {
@@ -91,8 +93,10 @@ struct AppendParams {
 
 // tuning constants the host layout needs
 constexpr int kScoreTile = 128;
-constexpr int kAttnRange = 64;      // entries of U per sparse-attention CTA
+constexpr int kAttnRange = 64;      // entries of U a sparse-attention CTA takes at a time
+constexpr int kAttnWave = 768;      // about one wave of sparse-attention CTAs on 148 SMs
 constexpr int kTopkChunk = 8192;    // positions per top-k CTA
+constexpr int kTopkBucket = 4096;   // (b1, b2) bucket entries kept per query head
 constexpr int kDenseTile = 128;
 
 int num_sms();

@@ -57,9 +57,9 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Derived sizes of one decode step (positions follow the slide "The GPU keeps 640 fixed
 // positions": W = [0, s1) u [w0, N), candidates C = [s1, w0)).
 struct Step {
-  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, nWsplit, nOsplit;
-  long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC;
-  size_t off_S, off_hist, off_hist2, off_meta, off_cand, off_part, total;
+  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, nsplit_cap, nWsplit, nOsplit;
+  long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC, wrange, orange;
+  size_t off_S, off_hist, off_hist2, off_meta, off_cand, off_buck, off_part, total;
 };
 
 static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
@@ -79,17 +79,33 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.k_eff = std::min<long long>(k, st.nC);
   st.ldS = round4(std::max<long long>(N, 1));
   st.ldC = round4(std::max<long long>(st.nC, 1));
-  // sparse attention splits: W in 64-row pieces per KV head, Omega in 64-row pieces per head
-  st.nWsplit = static_cast<int>((st.nW + kAttnRange - 1) / kAttnRange);
-  st.nOsplit = static_cast<int>((st.k_eff + kAttnRange - 1) / kAttnRange);
-  st.nsplit = std::max(1, st.nWsplit + st.nOsplit);
+  // sparse attention splits: W per KV head and Omega per query head, in ranges of whole
+  // 64-entry groups sized so that the retrieved CTAs make about one wave
+  {
+    const long long per_head = std::max<long long>(1, kAttnWave / st.R);
+    const long long quads = static_cast<long long>(B) * Hkv * ((Hq / Hkv + 3) / 4);
+    const long long per_group = std::max<long long>(1, kAttnWave / 3 / quads);
+    auto rng = [](long long n, long long parts) {
+      const long long groups = (n + kAttnRange - 1) / kAttnRange;
+      return std::max<long long>(1, (groups + parts - 1) / parts) * kAttnRange;
+    };
+    st.orange = rng(st.k_eff, per_head);
+    st.wrange = rng(st.nW, per_group);
+    st.nOsplit = static_cast<int>((st.k_eff + st.orange - 1) / st.orange);
+    st.nWsplit = static_cast<int>((st.nW + st.wrange - 1) / st.wrange);
+    st.nsplit = std::max(1, st.nWsplit + st.nOsplit);
+    // the layout must not depend on Hkv (the workspace size is asked without it): reserve
+    // partial states for the largest static split count, one per 64 rows of W
+    st.nsplit_cap = std::max(1, static_cast<int>((st.nW + kAttnRange - 1) / kAttnRange) + st.nOsplit);
+  }
   size_t off = 0;
   st.off_hist = off;  off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_hist2 = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_meta = off;  off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
   st.off_S = off;     off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
   st.off_cand = off;  off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 8);
-  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit * (d + 4) * 4);
+  st.off_buck = off;  off = align_up(off + static_cast<size_t>(st.R) * kTopkBucket * 8);
+  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit_cap * (d + 4) * 4);
   st.total = off;
   return RA_OK;
 }
@@ -146,6 +162,7 @@ static ra_status run_topk(const Step &st, int32_t *idx, void *ws, cudaStream_t s
   p.hist2 = reinterpret_cast<uint32_t *>(at(ws, st.off_hist2));
   p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
   p.cand = reinterpret_cast<uint2 *>(at(ws, st.off_cand));
+  p.bucket = reinterpret_cast<uint2 *>(at(ws, st.off_buck));
   p.idx = idx;
   p.ldS = st.ldS; p.ldC = st.ldC; p.N = st.N;
   p.cand_lo = st.s1; p.cand_hi = st.w0; p.nC = st.nC; p.k_eff = st.k_eff;
@@ -167,6 +184,7 @@ static ra_status run_attn(const ra_kv *kv, const Step &st, const int32_t *idx, f
   p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.k_eff = st.k_eff;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.nsplit = st.nsplit; p.R = st.R;
   p.B = st.B; p.nWsplit = st.nWsplit; p.nOsplit = st.nOsplit;
+  p.wrange = st.wrange; p.orange = st.orange;
   cudaError_t e = launch_sparse_attn(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "sparse_attn");
 }

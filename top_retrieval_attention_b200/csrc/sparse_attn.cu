@@ -2,10 +2,10 @@
 // renormalizes selected tokens", Eq. (2) with the selected set; "Two local softmax outputs
 // need global weights", Eqs. (3)-(5), and its backup slide, Appendix B).
 //
-// Two kinds of CTA, each covering at most 64 entries of the selected set:
-//   * static CTAs (one set per KV head): rows of W = sinks + window, shared by the G query
-//     heads of the KV head (slide "The GPU keeps 640 fixed positions"): each V row is
-//     gathered once and weighted for all G heads;
+// Two kinds of CTA, each covering a range of the selected set, 64 entries at a time:
+//   * static CTAs (one set per KV head and quad of its query heads): rows of W = sinks +
+//     window, shared by the G query heads of the KV head (slide "The GPU keeps 640 fixed
+//     positions"): each V row is gathered once and weighted for up to four heads;
 //   * retrieved CTAs (one set per query head): rows of Omega, that head's top-k.
 // A warp takes 16 entries: their positions, scores z (already computed; K is never read
 // again) and V rows are loaded together, the warp reduces its own max m, sum Z and
@@ -23,6 +23,7 @@ namespace ra {
 constexpr int kAttnThreads = 128;
 constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int kRowsPerWarp = kAttnRange / kAttnWarps;   // 16
+constexpr int kStaticHeads = 4;   // query heads served by one static CTA (a KV head's quad)
 
 // One warp: 16 entries (rows) at positions pos (lane j < 16 holds entry j, -1 when absent),
 // the scores of nh heads (z[h], lane j), V rows gathered 4 (d=128) or 2 (d=64) channels per
@@ -105,27 +106,62 @@ __device__ __forceinline__ void cta_combine(const float *wm, const float *wz, co
   }
 }
 
-// Shared memory of one CTA: per-warp states of up to kMaxGroup heads, then the merge buffer.
+// Shared memory of one CTA: per-warp states of up to kStaticHeads heads, then the merge buffer.
 template <int D>
 struct AttnSmem {
-  float m[kMaxGroup][kAttnWarps];
-  float z[kMaxGroup][kAttnWarps];
-  __align__(16) float acc[kMaxGroup * kAttnWarps * D];
+  float m[kStaticHeads][kAttnWarps];
+  float z[kStaticHeads][kAttnWarps];
+  __align__(16) float acc[kStaticHeads * kAttnWarps * D + (D == 64 ? 256 : 0)];
   float red[kAttnWarps];
-  int last[kMaxGroup];
+  int last[kStaticHeads];
 };
 
-// The body for CTAs covering NH heads (NH = kMaxGroup for static CTAs, of which the first
-// nrows are real; NH = 1 for retrieved CTAs), all array indices compile-time.
+// Running per-warp state of NH heads, merged group by group (online softmax):
+//   m' = max(m, m_g), Z' = Z e^{m - m'} + Z_g e^{m_g - m'}, acc' likewise.
 template <int D, int NH>
+__device__ __forceinline__ void fold(float (&m)[NH], float (&Zs)[NH], float (&acc)[NH][D / 32],
+                                     const float (&mg)[NH], const float (&Zg)[NH],
+                                     const float (&ag)[NH][D / 32], int nh) {
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    if (h >= nh || mg[h] == -INFINITY) continue;
+    const float mn = fmaxf(m[h], mg[h]);
+    const float a = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
+    const float bsc = expf(mg[h] - mn);
+    Zs[h] = Zs[h] * a + Zg[h] * bsc;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) acc[h][c] = acc[h][c] * a + ag[h][c] * bsc;
+    m[h] = mn;
+  }
+}
+
+// The body for CTAs covering NH heads (NH = kMaxGroup for static CTAs, of which the first
+// nrows are real; NH = 1 for retrieved CTAs), all array indices compile-time.  The CTA's
+// entries [e_lo, e_hi) are taken 64 at a time; entry(e) gives the position and the scores.
+template <int D, int NH, typename Entry>
 __device__ __forceinline__ void attn_cta(const AttnParams &p, AttnSmem<D> &sm, int row0, int nrows,
-                                         int split, const __nv_bfloat16 *Vh, int pos,
-                                         const float (&z)[NH]) {
+                                         int split, const __nv_bfloat16 *Vh, long long e_lo,
+                                         long long e_hi, Entry entry) {
   constexpr int CPL = D / 32;
   constexpr int PS = D + kPartPad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float m[NH], Zs[NH], acc[NH][CPL];
-  warp_rows<D, NH>(Vh, pos, z, nrows, m, Zs, acc);
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    m[h] = -INFINITY;
+    Zs[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+  }
+  for (long long g0 = e_lo; g0 < e_hi; g0 += kAttnRange) {
+    const long long e = g0 + warp * kRowsPerWarp + lane;
+    int pos = -1;
+    float z[NH];
+    entry(lane < kRowsPerWarp && e < e_hi ? e : -1, pos, z);
+    float mg[NH], Zg[NH], ag[NH][CPL];
+    warp_rows<D, NH>(Vh, pos, z, nrows, mg, Zg, ag);
+    fold<D, NH>(m, Zs, acc, mg, Zg, ag, nrows);
+  }
 #pragma unroll
   for (int h = 0; h < NH; ++h) {
     if (h < nrows) {
@@ -164,44 +200,51 @@ __device__ __forceinline__ void attn_cta(const AttnParams &p, AttnSmem<D> &sm, i
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 6) sparse_attn_kernel(const AttnParams p) {
   __shared__ AttnSmem<D> sm;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_trigger();
   pdl_wait();
-  const long long n_static_ctas = static_cast<long long>(p.B) * p.Hkv * p.nWsplit;
+  const int n_quads = (p.G + kStaticHeads - 1) / kStaticHeads;   // head quads per KV head
+  const long long n_static_ctas = static_cast<long long>(p.B) * p.Hkv * n_quads * p.nWsplit;
   if (blockIdx.x < n_static_ctas) {
-    const int grp = static_cast<int>(blockIdx.x / p.nWsplit);        // b * Hkv + g
-    const int s = static_cast<int>(blockIdx.x - static_cast<long long>(grp) * p.nWsplit);
+    // (KV head, quad of its query heads, range of W)
+    const long long gq = blockIdx.x / p.nWsplit;
+    const int s = static_cast<int>(blockIdx.x - gq * p.nWsplit);
+    const int grp = static_cast<int>(gq / n_quads);                  // b * Hkv + g
+    const int quad = static_cast<int>(gq - static_cast<long long>(grp) * n_quads);
     const int b = grp / p.Hkv, g = grp - b * p.Hkv;
-    const int row0 = b * p.Hq + g * p.G;
-    const long long e = static_cast<long long>(s) * kAttnRange + warp * kRowsPerWarp + lane;
-    int pos = -1;
-    if (lane < kRowsPerWarp && e < p.nW) pos = static_cast<int>(e < p.s1 ? e : p.w0 + (e - p.s1));
-    float z[kMaxGroup];
+    const int row0 = b * p.Hq + g * p.G + quad * kStaticHeads;
+    const int nrows = min(kStaticHeads, p.G - quad * kStaticHeads);
+    const long long e_lo = static_cast<long long>(s) * p.wrange;
+    const long long e_hi = min(e_lo + p.wrange, p.nW);
+    auto entry = [&](long long e, int &pos, float (&z)[kStaticHeads]) {
+      pos = e < 0 ? -1 : static_cast<int>(e < p.s1 ? e : p.w0 + (e - p.s1));
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h)
-      z[h] = (h < p.G && pos >= 0) ? __ldcg(p.S + (row0 + h) * p.ldS + pos) : -INFINITY;
-    attn_cta<D, kMaxGroup>(p, sm, row0, p.G, s, p.V + static_cast<long long>(grp) * p.cap * D,
-                           pos, z);
+      for (int h = 0; h < kStaticHeads; ++h)
+        z[h] = (h < nrows && pos >= 0) ? __ldcg(p.S + (row0 + h) * p.ldS + pos) : -INFINITY;
+    };
+    attn_cta<D, kStaticHeads>(p, sm, row0, nrows, s,
+                              p.V + static_cast<long long>(grp) * p.cap * D, e_lo, e_hi, entry);
   } else {
     const long long id = blockIdx.x - n_static_ctas;
     const int row = static_cast<int>(id / p.nOsplit);
     const int s = static_cast<int>(id - static_cast<long long>(row) * p.nOsplit);
     const int b = row / p.Hq, h = row - b * p.Hq;
-    const long long e = static_cast<long long>(s) * kAttnRange + warp * kRowsPerWarp + lane;
-    int pos = -1;
-    if (lane < kRowsPerWarp && e < p.k_eff) {
-      pos = __ldg(p.idx + static_cast<long long>(row) * p.k + e);
-      if (pos < 0 || pos >= p.N) pos = -1;   // never for a completed selection
-    }
-    float z[1];
-    z[0] = pos >= 0 ? __ldcg(p.S + row * p.ldS + pos) : -INFINITY;
+    const long long e_lo = static_cast<long long>(s) * p.orange;
+    const long long e_hi = min(e_lo + p.orange, p.k_eff);
+    const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
+    const float *srow = p.S + row * p.ldS;
+    auto entry = [&](long long e, int &pos, float (&z)[1]) {
+      pos = e < 0 ? -1 : __ldg(irow + e);
+      if (pos >= p.N) pos = -1;   // never for a completed selection
+      z[0] = pos >= 0 ? __ldcg(srow + pos) : -INFINITY;
+    };
     attn_cta<D, 1>(p, sm, row, 1, p.nWsplit + s,
-                   p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D, pos, z);
+                   p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D, e_lo, e_hi,
+                   entry);
   }
 }
 
 cudaError_t launch_sparse_attn(const AttnParams &p, int d, cudaStream_t s) {
-  const long long ctas = static_cast<long long>(p.B) * p.Hkv * p.nWsplit +
+  const long long ctas = static_cast<long long>(p.B) * p.Hkv * ((p.G + 3) / 4) * p.nWsplit +
                          static_cast<long long>(p.R) * p.nOsplit;
   const dim3 grid(static_cast<unsigned>(ctas));
   return d == 128 ? launch_pdl(sparse_attn_kernel<128>, grid, dim3(kAttnThreads), 0, s, p)

@@ -4,18 +4,18 @@
 //
 // Keys are compared as 64-bit composites (order_key(z) << 32 | ~position), so every key is
 // distinct, larger z wins and equal z goes to the lower position.  The selection is a radix
-// select over digits of the composite, in one kernel over (head, chunk) CTAs:
-//   * digit 1 = the top 11 bits of order_key(z), histogrammed by the score kernel; every CTA
-//     finds the threshold bin b1 (the bin holding the k-th largest key);
-//   * keys above b1 are written out and keys in b1 listed (position and key): each thread
-//     counts its keys, one block scan places them, and each CTA reserves its output ranges
-//     with one atomic per list;
-//   * the listed keys are also histogrammed by digit 2 (the next 11 bits); the last CTA of a
-//     head finds the digit-2 threshold bin b2, emits the listed keys above (b1, b2) in one
-//     pass and narrows the (b1, b2) bucket with further 8-bit digits until it is taken whole
-//     or holds at most 64 keys, which one warp sorts with a bitonic network.
+// select over digits of the composite, in two kernels:
+//   * collect, (head, chunk) CTAs: digit 1 = the top 11 bits of order_key(z), histogrammed
+//     by the score kernel; every CTA finds the threshold bin b1 (the bin holding the k-th
+//     largest key), writes out the keys above b1 and lists the keys in b1 (position and
+//     key), placing them with one block scan and one reservation atomic per list, and
+//     histograms digit 2 (the next 11 bits) of the listed keys;
+//   * refine, (head, part) CTAs over the list: the digit-2 threshold bin b2; listed keys
+//     above (b1, b2) are written out and those in (b1, b2) moved to a bucket; the last CTA
+//     of a head narrows the bucket with further 8-bit digits until it is taken whole or
+//     holds at most 64 keys, which one warp sorts with a bitonic network.
 // A digit-1 bin is a range of z (order_key is monotone), so the per-key test is a pair of
-// float comparisons.  The histogram and counters are left zero for the next call.
+// float comparisons.  Histograms and counters are left zero for the next call.
 #include <math.h>
 
 #include "common.cuh"
@@ -24,9 +24,10 @@
 namespace ra {
 
 constexpr int kTkThreads = 256;
-constexpr int kBucketCap = 4096;     // bucket held in shared memory by the tail (32 KB)
+constexpr int kBucketCap = kTopkBucket;   // bucket entries kept per head (32 KB in the tail)
 constexpr int kBitonic = 64;
 constexpr int kDigit2Shift = 10;     // digit 2 = bits [10, 21) of the order key
+constexpr int kRefineParts = 16;     // refine CTAs per query head
 constexpr int kPerThread = kTopkChunk / kTkThreads;   // 32 keys per thread
 constexpr int kVec = kPerThread / 4;                  // float4 loads per thread
 
@@ -146,19 +147,14 @@ __device__ __forceinline__ bool last_of_row(uint32_t *counter, uint32_t total, b
 //      in b1 are listed with their order keys; the head's last CTA selects the rest from
 //      that list and leaves the histogram and counters zero
 __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkParams p) {
-  __shared__ __align__(16) uint64_t bucket[kBucketCap];   // the last CTA's (b1, b2) bucket
   __shared__ uint32_t warp_tot[kTkThreads / 32];
   __shared__ Thresh s_t;
   __shared__ uint32_t h2[kHistBins];      // digit-2 histogram of this CTA's listed keys
-  __shared__ uint64_t bs[kBitonic];
-  __shared__ uint32_t s_ns, s_nc, s_bs, s_bc, s_out, s_cnt, s_cum, s_nb;
-  __shared__ int s_digit;
-  __shared__ bool s_last;
-  uint32_t *h256 = h2;                    // the last CTA's 8-bit digit histogram
+  __shared__ uint32_t s_ns, s_nc, s_bs, s_bc;
   pdl_trigger();
   pdl_wait();
   const int row = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   if (blockIdx.x == 0)
     for (long long i = p.k_eff + tid; i < p.k; i += kTkThreads) irow[i] = -1;
@@ -174,10 +170,12 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
   uint32_t *meta = p.meta + row * kMetaWords;
   uint32_t *h1g = p.hist + static_cast<long long>(row) * kHistBins;
   int b1 = -1;
+  uint32_t above1 = 0;
   float zlo = -INFINITY, zhi = -INFINITY;   // emit z >= zhi; list zlo <= z < zhi
   if (!take_all) {
     const Thresh t1 = find_threshold<kTkThreads>(h1g, static_cast<uint32_t>(p.k_eff), warp_tot, &s_t);
     b1 = t1.bin;
+    above1 = t1.above;
     zlo = key_float(static_cast<uint32_t>(b1) << (32 - kHistBits));
     zhi = b1 + 1 < kHistBins ? key_float(static_cast<uint32_t>(b1 + 1) << (32 - kHistBits)) : INFINITY;
   }
@@ -230,75 +228,128 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
     for (int i = tid; i < kHistBins; i += kTkThreads)
       if (h2[i]) atomicAdd(h2g + i, h2[i]);
 
-  const uint32_t parts = static_cast<uint32_t>((p.cand_hi - 1) / kTopkChunk - p.cand_lo / kTopkChunk + 1);
-  if (!last_of_row(meta + kDone, parts, &s_last)) return;
-  // ---- the head's last CTA: the remaining rr keys come from the bin-b1 list
-  const uint32_t above = __ldcg(meta + kSelCount);
+  if (!take_all && blockIdx.x == p.cand_lo / kTopkChunk && tid == 0) {
+    meta[kThresh1] = static_cast<uint32_t>(b1);
+    meta[kAbove1] = above1;   // the keys above b1, all written out by this kernel
+  }
+}
+
+// ---- refine, (head, part) CTAs over the head's list of bin-b1 keys: the digit-2 threshold
+//      bin b2, the listed keys above (b1, b2) written out, those in (b1, b2) moved to the
+//      head's bucket; the head's last CTA selects the rest from the bucket and leaves the
+//      histograms and counters zero
+__global__ void __launch_bounds__(kTkThreads) topk_refine_kernel(const TopkParams p) {
+  __shared__ __align__(16) uint64_t bucket[kBucketCap];
+  __shared__ uint32_t warp_tot[kTkThreads / 32];
+  __shared__ Thresh s_t;
+  __shared__ uint32_t h256[256];
+  __shared__ uint64_t bs[kBitonic];
+  __shared__ uint32_t s_bs, s_out, s_cnt, s_cum, s_nb;
+  __shared__ int s_digit;
+  __shared__ bool s_last;
+  pdl_trigger();
+  pdl_wait();
+  const int row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (p.k_eff == 0) return;
+  const bool take_all = p.k_eff >= p.nC;
+  uint32_t *meta = p.meta + row * kMetaWords;
+  uint32_t *h1g = p.hist + static_cast<long long>(row) * kHistBins;
+  uint32_t *h2g = p.hist2 + static_cast<long long>(row) * kHistBins;
+  int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
+  const uint2 *crow = p.cand + static_cast<long long>(row) * p.ldC;        // bin-b1 list
+  uint2 *brow = p.bucket + static_cast<long long>(row) * kBucketCap;       // (b1, b2) bucket
+  const uint32_t above1 = __ldcg(meta + kAbove1);    // keys above b1, written by collect
   const uint32_t n_list = min(__ldcg(meta + kCandCount), static_cast<uint32_t>(p.ldC));
+  const uint32_t b1 = __ldcg(meta + kThresh1);
+  const uint32_t wbase = static_cast<uint32_t>(tid - lane);
+  uint32_t rr = static_cast<uint32_t>(p.k_eff) - min(above1, static_cast<uint32_t>(p.k_eff));
+  const bool active = !take_all && rr > 0 && n_list > 0;
+  uint32_t b2 = 0, above2 = 0;
+  if (active) {
+    const Thresh t2 = find_threshold<kTkThreads>(h2g, rr, warp_tot, &s_t);
+    b2 = static_cast<uint32_t>(t2.bin);
+    above2 = t2.above;
+    // this CTA's part of the list: keys above (b1, b2) counted, placed and written; keys in
+    // (b1, b2) appended to the bucket
+    const uint32_t per = (n_list + gridDim.x - 1) / gridDim.x;
+    const uint32_t i_lo = blockIdx.x * per, i_hi = min(n_list, i_lo + per);
+    constexpr int kBatch = 8;
+    for (uint32_t i0 = i_lo; i0 < i_hi; i0 += kBatch * kTkThreads) {
+      uint2 cb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const uint32_t i = i0 + u * kTkThreads + tid;
+        cb[u] = i < i_hi ? __ldcg(&crow[i]) : make_uint2(0u, 0u);
+      }
+      uint32_t n_up = 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const uint32_t i = i0 + u * kTkThreads + tid;
+        const uint32_t d2 = (cb[u].y >> kDigit2Shift) & (kHistBins - 1);
+        n_up += (i < i_hi && d2 > b2) ? 1u : 0u;
+        if (i < i_hi && d2 == b2) {   // a handful per head
+          const uint32_t o = atomicAdd(meta + kBuckCount, 1u);
+          if (o < static_cast<uint32_t>(kBucketCap)) brow[o] = cb[u];
+        }
+      }
+      const uint32_t incl = block_incl_scan<kTkThreads>(n_up, warp_tot);
+      if (tid == kTkThreads - 1) s_bs = incl ? atomicAdd(meta + kSelCount, incl) : 0u;
+      __syncthreads();
+      uint32_t o = s_bs + incl - n_up;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const uint32_t i = i0 + u * kTkThreads + tid;
+        const uint32_t d2 = (cb[u].y >> kDigit2Shift) & (kHistBins - 1);
+        if (i < i_hi && d2 > b2) {
+          if (o < p.k_eff) irow[o] = static_cast<int32_t>(cb[u].x);
+          ++o;
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  if (!last_of_row(meta + kDone, gridDim.x, &s_last)) return;
+  // ---- the head's last CTA
+  const uint32_t n_bk = __ldcg(meta + kBuckCount);
   __syncthreads();
   if (tid < kError) meta[tid] = 0u;
-  if (take_all) return;   // nothing was histogrammed or listed
-  if (above >= p.k_eff || n_list == 0) {   // counters not from this call
+  if (!take_all)
     for (int i = tid; i < kHistBins; i += kTkThreads) {
       h1g[i] = 0u;
       h2g[i] = 0u;
     }
-    return;
-  }
-  uint32_t rr = static_cast<uint32_t>(p.k_eff) - above;   // 1 <= rr <= n_list
-  if (tid == 0) s_out = above;
-  auto emit = [&](bool pred, uint32_t pos) {
-    bool ok;
-    const uint32_t o = warp_append(pred, &s_out, ok);
-    if (ok && o < p.k_eff) irow[o] = static_cast<int32_t>(pos);
-  };
-  const uint32_t wbase = static_cast<uint32_t>(tid - lane);
-  // digit 2 over the complete list: threshold bin b2; one batched pass emits the keys above
-  // (b1, b2) and gathers the (b1, b2) bucket into shared memory
-  const Thresh t2 = find_threshold<kTkThreads>(h2g, rr, warp_tot, &s_t);
-  for (int i = tid; i < kHistBins; i += kTkThreads) {
-    h1g[i] = 0u;
-    h2g[i] = 0u;
-  }
-  const uint32_t b2 = static_cast<uint32_t>(t2.bin);
-  rr -= t2.above;
-  const uint32_t cnt2 = t2.cnt;                           // 1 <= rr <= cnt2
-  const bool in_smem = cnt2 <= static_cast<uint32_t>(kBucketCap);
-  if (tid == 0) s_nb = 0;
-  __syncthreads();
-  constexpr int kBatch = 16;
-  for (uint32_t i0 = wbase; i0 < n_list; i0 += kBatch * kTkThreads) {
-    uint2 cb[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const uint32_t i = i0 + u * kTkThreads + lane;
-      cb[u] = i < n_list ? __ldcg(&crow[i]) : make_uint2(0u, 0u);
+  if (!active) return;
+  uint32_t rr2 = rr - above2;                    // 1 <= rr2 <= size of the bucket
+  // a bucket of at most kBucketCap keys is complete in brow and goes to shared memory; a larger
+  // one (only with massive ties) is read from the whole list, filtered by its digits
+  const bool in_smem = n_bk <= static_cast<uint32_t>(kBucketCap);
+  const uint32_t n_buck = in_smem ? n_bk : n_list;
+  if (in_smem)
+    for (uint32_t i = tid; i < n_buck; i += kTkThreads) {
+      const uint2 c = __ldcg(&brow[i]);
+      bucket[i] = make_composite(c.y, c.x);
     }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const uint32_t i = i0 + u * kTkThreads + lane;
-      const uint32_t d2 = (cb[u].y >> kDigit2Shift) & (kHistBins - 1);
-      emit(i < n_list && d2 > b2, cb[u].x);
-      bool ok;
-      const uint32_t o = warp_append(i < n_list && d2 == b2 && in_smem, &s_nb, ok);
-      if (ok && o < static_cast<uint32_t>(kBucketCap)) bucket[o] = make_composite(cb[u].y, cb[u].x);
-    }
-  }
+  if (tid == 0) s_out = above1 + above2;
   __syncthreads();
-  // the (b1, b2) bucket: in shared memory, or (all keys alike) over the stored list
-  const uint32_t n_buck = in_smem ? cnt2 : n_list;
   auto get = [&](uint32_t i) -> uint64_t {
     if (in_smem) return bucket[i];
     const uint2 c = __ldcg(&crow[i]);
     return make_composite(c.y, c.x);
   };
+  auto emit = [&](bool pred, uint32_t pos) {
+    bool ok;
+    const uint32_t o = warp_append(pred, &s_out, ok);
+    if (ok && o < p.k_eff) irow[o] = static_cast<int32_t>(pos);
+  };
   uint64_t prefix = (static_cast<uint64_t>(b1) << kHistBits) | b2;
   int shift = 64 - 2 * kHistBits;
-  uint32_t cnt = cnt2;
+  uint32_t cnt = n_bk;
   // every round fixes 8 more bits of a unique 64-bit key: at most ceil(42 / 8) + 1 rounds
 #pragma unroll 1
   for (int round = 0; round < 8; ++round) {
-    if (cnt == rr) {   // the whole bucket is taken
+    if (cnt == rr2) {   // the whole bucket is taken
       for (uint32_t i0 = wbase; i0 < n_buck; i0 += kTkThreads) {
         const uint32_t i = i0 + lane;
         const uint64_t x = i < n_buck ? get(i) : 0ull;
@@ -335,7 +386,7 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
           }
         }
         const uint32_t o0 = s_out;
-        for (uint32_t i = lane; i < rr && o0 + i < p.k_eff; i += 32)
+        for (uint32_t i = lane; i < rr2 && o0 + i < p.k_eff; i += 32)
           irow[o0 + i] = static_cast<int32_t>(comp_pos(bs[i]));
       }
       return;
@@ -366,10 +417,10 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
         if (lane >= o) incl += nn;
       }
       const uint32_t excl = incl - sum;
-      if (excl < rr && rr <= incl) {
+      if (excl < rr2 && rr2 <= incl) {
         uint32_t cum = excl;
         for (int i = 0; i < 8; ++i) {
-          if (cum + lc[i] >= rr) {
+          if (cum + lc[i] >= rr2) {
             s_digit = 255 - 8 * lane - i;
             s_cum = cum;
             s_cnt = lc[i];
@@ -387,7 +438,7 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
       const uint64_t x = i < n_buck ? get(i) : 0ull;
       emit(i < n_buck && (x >> shift) == prefix && ((x >> nshift) & dmask) > v, comp_pos(x));
     }
-    rr -= cum;
+    rr2 -= cum;
     cnt = s_cnt;
     prefix = (prefix << nb) | v;
     shift = nshift;
@@ -399,8 +450,12 @@ __global__ void __launch_bounds__(kTkThreads, 4) topk_collect_kernel(const TopkP
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t s) {
   if (p.k <= 0) return cudaSuccess;
   const long long chunks = (p.N + kTopkChunk - 1) / kTopkChunk;
-  const dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(p.R));
-  return launch_pdl(topk_collect_kernel, grid, dim3(kTkThreads), 0, s, p);
+  cudaError_t e = launch_pdl(topk_collect_kernel,
+                             dim3(static_cast<unsigned>(chunks), static_cast<unsigned>(p.R)),
+                             dim3(kTkThreads), 0, s, p);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_refine_kernel, dim3(kRefineParts, static_cast<unsigned>(p.R)),
+                    dim3(kTkThreads), 0, s, p);
 }
 
 }  // namespace ra
