@@ -40,33 +40,39 @@ __device__ inline uint16_t to_bf16_bits(double x) {
   return static_cast<uint16_t>((bits + 0x7FFFu + ((bits >> 16) & 1u)) >> 16);
 }
 
-// one thread per 8 consecutive channels of one row
-__global__ void fill_kv_kernel(uint16_t *K, uint16_t *V, int B, int Hkv, long long cap, int d,
-                               long long row0, long long nrows, uint64_t seed, int layer,
-                               int with_offset) {
-  const int per_row = d / 8;
-  const long long total = static_cast<long long>(B) * Hkv * nrows * per_row;
-  for (long long w = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; w < total;
-       w += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c8 = static_cast<int>(w % per_row);
-    const long long r = (w / per_row) % nrows;
-    const long long bg = w / (per_row * nrows);
-    const int b = static_cast<int>(bg / Hkv), g = static_cast<int>(bg % Hkv);
+// Block (x, bg): a thread owns 8 consecutive channels (c8) of every row r = row0 + phase
+// (mod rows in flight); the stream keys and the channel offsets are computed once per thread.
+__global__ void __launch_bounds__(256) fill_kv_kernel(uint16_t *K, uint16_t *V, int Hkv,
+                                                      long long cap, int d, long long row0,
+                                                      long long nrows, uint64_t seed, int layer,
+                                                      int with_offset) {
+  const int per_row = d / 8;                     // threads per row
+  const int phases = 256 / per_row;              // rows in flight per block
+  const int bg = blockIdx.y;
+  const int b = bg / Hkv, g = bg % Hkv;
+  const int c8 = threadIdx.x % per_row;
+  const int phase = threadIdx.x / per_row;
+  const uint64_t kk = stream_key(seed, kKindK, layer, b, g);
+  const uint64_t kv = stream_key(seed, kKindV, layer, b, g);
+  double off[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    off[j] = with_offset ? __dmul_rn(kOffStd, normal_at(stream_key(seed, kKindKoff, layer, b, g),
+                                                        static_cast<uint64_t>(c8 * 8 + j)))
+                         : 0.0;
+  const long long step = static_cast<long long>(gridDim.x) * phases;
+  for (long long r = static_cast<long long>(blockIdx.x) * phases + phase; r < nrows; r += step) {
     const long long i = row0 + r;
-    const uint64_t kk = stream_key(seed, kKindK, layer, b, g);
-    const uint64_t kv = stream_key(seed, kKindV, layer, b, g);
-    const uint64_t ko = stream_key(seed, kKindKoff, layer, b, g);
     uint16_t outk[8], outv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int c = c8 * 8 + j;
-      const uint64_t e = static_cast<uint64_t>(i) * d + c;
+      const uint64_t e = static_cast<uint64_t>(i) * d + c8 * 8 + j;
       double xk = normal_at(kk, e);
-      if (with_offset) xk = __dadd_rn(xk, __dmul_rn(kOffStd, normal_at(ko, c)));
+      if (with_offset) xk = __dadd_rn(xk, off[j]);
       outk[j] = to_bf16_bits(xk);
       outv[j] = to_bf16_bits(normal_at(kv, e));
     }
-    const long long off = (bg * cap + i) * d + c8 * 8;
+    const long long o = (static_cast<long long>(bg) * cap + i) * d + c8 * 8;
     uint4 pk, pv;
     pk.x = outk[0] | (static_cast<uint32_t>(outk[1]) << 16);
     pk.y = outk[2] | (static_cast<uint32_t>(outk[3]) << 16);
@@ -76,8 +82,8 @@ __global__ void fill_kv_kernel(uint16_t *K, uint16_t *V, int B, int Hkv, long lo
     pv.y = outv[2] | (static_cast<uint32_t>(outv[3]) << 16);
     pv.z = outv[4] | (static_cast<uint32_t>(outv[5]) << 16);
     pv.w = outv[6] | (static_cast<uint32_t>(outv[7]) << 16);
-    *reinterpret_cast<uint4 *>(K + off) = pk;
-    *reinterpret_cast<uint4 *>(V + off) = pv;
+    *reinterpret_cast<uint4 *>(K + o) = pk;
+    *reinterpret_cast<uint4 *>(V + o) = pv;
   }
 }
 
@@ -103,11 +109,14 @@ int synth_fill_kv(void *K, void *V, int32_t B, int32_t Hkv, int32_t cap, int32_t
       row0 + nrows > cap)
     return -1;
   if (nrows == 0) return 0;
-  const long long total = static_cast<long long>(B) * Hkv * nrows * (d / 8);
-  long long blocks = (total + 255) / 256;
-  if (blocks > 148LL * 32) blocks = 148LL * 32;
-  fill_kv_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint16_t *>(K), static_cast<uint16_t *>(V), B, Hkv, cap, d, row0, nrows, seed,
+  if (static_cast<long long>(B) * Hkv > 65535) return -1;
+  const int phases = 256 / (d / 8);
+  long long bx = (nrows + phases - 1) / phases;
+  const long long want = (148LL * 16 + static_cast<long long>(B) * Hkv - 1) / (static_cast<long long>(B) * Hkv);
+  if (bx > want) bx = want;
+  const dim3 grid(static_cast<unsigned>(bx < 1 ? 1 : bx), static_cast<unsigned>(B * Hkv));
+  fill_kv_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint16_t *>(K), static_cast<uint16_t *>(V), Hkv, cap, d, row0, nrows, seed,
       layer, with_offset);
   return static_cast<int>(cudaGetLastError());
 }
