@@ -305,14 +305,10 @@ def run_ours(args, w, rank, local_rank, world, dist):
         ra.check(ra.ra_score_gqa(kv, qptr, Hq, k, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
         if ev is not None:
             ev[2].record(stream)
-        ra.check(ra.ra_topk_select(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
-                                   ws.data_ptr(), ws_bytes, sp), "topk")
+        ra.check(ra.ra_select_attend(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+                                     outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "select_attend")
         if ev is not None:
             ev[3].record(stream)
-        ra.check(ra.ra_sparse_attn(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
-                                   outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "attn")
-        if ev is not None:
-            ev[4].record(stream)
         c.N = N - 1
 
     def step(s, evs=None):
@@ -329,10 +325,8 @@ def run_ours(args, w, rank, local_rank, world, dist):
             ev[layer][0].record(stream)
             ra.check(ra.ra_score_gqa(kv, qptr, Hq, k, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
             ev[layer][1].record(stream)
-            ra.check(ra.ra_topk_select(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
-                                       ws.data_ptr(), ws_bytes, sp), "topk")
-            ra.check(ra.ra_sparse_attn(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
-                                       outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "attn")
+            ra.check(ra.ra_select_attend(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+                                         outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "select_attend")
             c.N = N - 1
 
     # warm-up, then (for short timed regions) an untimed soak so clocks reach steady state
@@ -381,19 +375,18 @@ def run_ours(args, w, rank, local_rank, world, dist):
     # phase breakdown (diagnostic, not the timed region): events between every kernel phase,
     # which also removes the programmatic-launch overlap at each boundary
     psteps = min(steps, 2000)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(L)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)]
            for _ in range(psteps)]
     for s in range(psteps):
         step(s, evs[s])
     torch.cuda.synchronize()
-    ph = {"append": [], "score": [], "topk": [], "attn": []}
+    ph = {"append": [], "score": [], "select_attend": []}
     for s in range(psteps):
         for layer in range(L):
             e = evs[s][layer]
             ph["append"].append(e[0].elapsed_time(e[1]))
             ph["score"].append(e[1].elapsed_time(e[2]))
-            ph["topk"].append(e[2].elapsed_time(e[3]))
-            ph["attn"].append(e[3].elapsed_time(e[4]))
+            ph["select_attend"].append(e[2].elapsed_time(e[3]))
     ph_us = {kk: 1000.0 * statistics.mean(v) for kk, v in ph.items()}
 
     # algorithmic bytes: K once per KV head, plus the V rows of U per query head
@@ -415,7 +408,7 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 "algorithmic_bytes_per_launch": k_bytes,
                 "frac_of_nominal_8tbs": kscan_gbs / NOMINAL_HBM_GBS,
                 "score_kernel_sha": src_hash}
-    launches_per_layer = 2 + (1 if k_eff > 0 else 0) + (1 if k > 0 else 0) + 1
+    launches_per_layer = 3   # append, score, select + attention
     result = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

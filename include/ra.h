@@ -90,7 +90,7 @@ ra_status ra_append_kv(ra_kv *kv, const void *k_new, const void *v_new, int32_t 
 
 /*
  * Workspace bytes that ra_decode_step (and its three phases) need for this shape.
- * Returns 0 for an invalid shape.  The size grows with B*Hq*N (scores and candidates).
+ * Returns 0 for an invalid shape.  The size grows with B*Hq*N (the fp32 scores).
  */
 size_t ra_decode_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, int32_t k,
                                  int32_t n_sink, int32_t n_window);
@@ -122,13 +122,18 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
                          ra_stream_t stream);
 
 /*
- * The three phases of ra_decode_step, exposed so a caller can time or interleave them.
- * Run in this order with the same arguments and workspace, they are ra_decode_step; run them
- * only as that complete sequence (ra_topk_select re-zeroes what ra_score_gqa counted).
- *   ra_score_gqa   : z for every (query head, position) into ws, plus the per-head score
- *                    histogram of the candidates (one pass over K per KV head).
- *   ra_topk_select : Omega into idx from the scores in ws (radix select + bitonic finish).
- *   ra_sparse_attn : out from the scores in ws, V rows of U = W u Omega, and the merge.
+ * The phases of ra_decode_step, exposed so a caller can time or interleave them.  All take the
+ * arguments of ra_decode_step and the same workspace, and must run as one of the complete
+ * sequences  ra_score_gqa, ra_select_attend  (which is ra_decode_step)  or
+ * ra_score_gqa, ra_topk_select, ra_sparse_attn  (ra_topk_select re-zeroes what ra_score_gqa
+ * counted).
+ *   ra_score_gqa     : z for every (query head, position) into ws, plus the per-head score
+ *                      histogram of the candidates (one pass over K per KV head).
+ *   ra_topk_select   : Omega into idx from the scores in ws (radix select over the histogram,
+ *                      bitonic finish).
+ *   ra_sparse_attn   : out from the scores in ws, the V rows of U = W u Omega (Omega read from
+ *                      idx), and the merge of the split partial states (Eqs. (3)-(5)).
+ *   ra_select_attend : ra_topk_select then ra_sparse_attn in one launch.
  */
 ra_status ra_score_gqa(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
                        int32_t n_window, void *ws, size_t ws_bytes, ra_stream_t stream);
@@ -138,6 +143,9 @@ ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
 ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
                          int32_t n_window, const int32_t *idx, float *out, void *ws,
                          size_t ws_bytes, ra_stream_t stream);
+ra_status ra_select_attend(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                           int32_t n_window, int32_t *idx, float *out, void *ws, size_t ws_bytes,
+                           ra_stream_t stream);
 
 /*
  * ra_decode_step without a caller workspace, for callers that cannot allocate device memory
@@ -148,7 +156,7 @@ ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
  *   Scratch: a 64 MiB array inside libra (a file-scope __device__ array), held on every GPU
  *     that loads the library until the process exits.  A shape whose
  *     ra_decode_workspace_bytes(...) exceeds 64 MiB is rejected with RA_ERR_WORKSPACE before
- *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 50 MiB).
+ *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 17 MiB).
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream capture.
  *   Each call clears the scratch's counter block with cudaMemsetAsync on `stream`; nothing is

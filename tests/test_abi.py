@@ -60,8 +60,8 @@ def _kv(B=1, Hkv=2, d=128, cap=100, N=50, K=FAKE, V=FAKE):
 
 def test_workspace_bytes():
     n = ra.ra_decode_workspace_bytes(1, 32, 131072, 128, 1310, 128, 512)
-    # scores (32 x 131072 fp32) + histograms + counters + candidates + partial states
-    assert n >= 32 * 131072 * 4 * 2
+    # scores (32 x 131072 fp32) + digit-1 histograms (32 x 2048) + counters
+    assert n >= 32 * 131072 * 4 + 32 * 2048 * 4 + 32 * 8 * 4
     assert n % 256 == 0
     assert ra.ra_decode_workspace_bytes(1, 32, 131072, 96, 10, 0, 0) == 0     # d
     assert ra.ra_decode_workspace_bytes(0, 32, 131072, 128, 10, 0, 0) == 0    # B
@@ -111,6 +111,9 @@ def test_phases_validate_like_the_step():
     assert ra.ra_topk_select(kv, 4, 10, 4, 8, 0, FAKE, big, None) == ra.RA_ERR_ARG
     assert ra.ra_sparse_attn(kv, 4, 10, 4, 8, FAKE, 0, FAKE, big, None) == ra.RA_ERR_ARG
     assert ra.ra_sparse_attn(kv, 4, 10, 4, 8, FAKE, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
+    assert ra.ra_select_attend(kv, 4, 10, 4, 8, 0, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_select_attend(kv, 4, 10, 4, 8, FAKE, 0, FAKE, big, None) == ra.RA_ERR_ARG
+    assert ra.ra_select_attend(kv, 4, 10, 4, 8, FAKE, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
 
 
 def test_dense_rejects_bad_arguments():

@@ -70,7 +70,9 @@ SMALL = [
     (1, 4, 2, 2500, 128, 5000, 8, 8),      # k >= |C|: full attention
     (1, 16, 2, 9000, 128, 700, 128, 512),  # G = 8
     (3, 4, 4, 5000, 64, 257, 0, 64),       # G = 1, batch 3
-    (1, 4, 1, 70000, 128, 900, 128, 512),  # several collect chunks, ragged tail
+    (1, 4, 1, 70000, 128, 900, 128, 512),  # a 16-CTA cluster per head, ragged chunks
+    (1, 4, 1, 70000, 128, 40000, 128, 512),  # keys above b1 overflow a CTA's list: re-read path
+    (2, 16, 2, 150000, 64, 3000, 3, 100),  # batch 2, G = 8, unaligned sink end
 ]
 
 
@@ -136,10 +138,18 @@ def test_phases_equal_the_step():
     assert ra.ra_topk_select(cache.kv, 8, 77, 4, 64, idx2.data_ptr(), ws.data_ptr(), ws.numel(), s) == 0
     assert ra.ra_sparse_attn(cache.kv, 8, 77, 4, 64, idx2.data_ptr(), out2.data_ptr(),
                              ws.data_ptr(), ws.numel(), s) == 0
+    out3 = torch.empty_like(out1)
+    idx3 = torch.empty((1, 8, 77), dtype=torch.int32, device="cuda")
+    assert ra.ra_score_gqa(cache.kv, qd.data_ptr(), 8, 77, 4, 64, ws.data_ptr(), ws.numel(), s) == 0
+    assert ra.ra_select_attend(cache.kv, 8, 77, 4, 64, idx3.data_ptr(), out3.data_ptr(),
+                               ws.data_ptr(), ws.numel(), s) == 0
     torch.cuda.synchronize()
-    # Omega's order (atomics) decides the split partition, so sums may round differently
+    # Omega's order in idx (shared-memory list appends) decides the attention split, so sums
+    # may round differently
     np.testing.assert_allclose(out1.cpu().numpy(), out2.cpu().numpy(), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(out1.cpu().numpy(), out3.cpu().numpy(), rtol=1e-5, atol=1e-6)
     assert np.array_equal(np.sort(idx1.cpu().numpy(), -1), np.sort(idx2.cpu().numpy(), -1))
+    assert np.array_equal(np.sort(idx1.cpu().numpy(), -1), np.sort(idx3.cpu().numpy(), -1))
 
 
 def test_append_then_decode_equals_decode_of_the_full_cache():

@@ -5,5 +5,5 @@ from .ra import (  # noqa: F401
     RA_ERR_WORKSPACE, RA_OK, RaError, append_kv, check, decode_step, decode_workspace,
     dense_decode, dense_workspace, lib, ra_append_kv, ra_decode_step, ra_decode_workspace_bytes,
     ra_decode_step_static, ra_dense_decode, ra_dense_workspace_bytes, ra_kv, ra_last_error, ra_score_gqa,
-    ra_sparse_attn, ra_status_str, ra_topk_select, ra_version,
+    ra_select_attend, ra_sparse_attn, ra_status_str, ra_topk_select, ra_version,
 )

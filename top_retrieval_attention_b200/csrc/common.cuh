@@ -12,10 +12,9 @@ constexpr int kHistBins = 1 << kHistBits;     // 2048 bins per query head
 constexpr int kMaxGroup = 8;                  // query heads per KV head (one n8 MMA tile)
 constexpr int kMetaWords = 8;                 // per-row counters in the workspace
 
-// per-row counters (uint32) in the workspace's meta block
-enum MetaSlot { kSelCount = 0, kCandCount = 1, kBuckCount = 2, kThresh1 = 3, kAbove1 = 4,
-                kError = 6, kDone = 7 };
-// kDone is shared by the sparse and the dense merge (each leaves it zero).
+// per-row counters (uint32) in the workspace's meta block: the error word (row 0) and the
+// dense merge's CTA counter (left zero by the merging CTA)
+enum MetaSlot { kError = 6, kDone = 7 };
 
 // ------------------------------------------------------------------ programmatic dependent launch
 
@@ -37,6 +36,12 @@ __device__ __forceinline__ uint32_t order_key(float z) {
 }
 
 __device__ __forceinline__ float canon_zero(float z) { return z == 0.0f ? 0.0f : z; }
+
+// The float whose order key is `key` (the inverse bijection of order_key on bit patterns): for
+// finite scores z >= key_float(K) exactly when order_key(z) >= K.
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
 
 // ------------------------------------------------------------------ async copies
 

@@ -45,32 +45,27 @@ struct ScoreParams {
   uint32_t *err;            // error word (bit kErrScoreWait: a load never landed)
 };
 
-struct TopkParams {
-  const float *S;
-  uint32_t *hist;           // [B*Hq, kHistBins] digit-1 histogram (left zero by the select)
-  uint32_t *hist2;          // [B*Hq, kHistBins] digit-2 histogram of the listed keys (same)
-  uint32_t *meta;           // [B*Hq, kMetaWords] counters (left zero by the select)
-  uint2 *cand;              // [B*Hq, ldC] (position, order key) of the keys in bin b1
-  uint2 *bucket;            // [B*Hq, kTopkBucket] the keys in (b1, b2)
-  int32_t *idx;             // [B*Hq, k]
-  long long ldS, ldC, N;
-  long long cand_lo, cand_hi, nC, k_eff;
-  int k, R;
-};
+// Top-k selection and sparse attention of one decode step, one thread-block cluster per query
+// head (row = b * Hq + h).  mode: kSaSelect writes idx from the scores; kSaAttend computes out
+// from the scores, idx and V; both in one launch for the decode step.
+constexpr int kSaSelect = 1;
+constexpr int kSaAttend = 2;
+constexpr int kMaxCluster = 16;        // CTAs per query head at most
+constexpr int kDigit2Shift = 10;       // digit 2 = bits [10, 21) of the order key
+constexpr uint32_t kErrSelect = 4u;    // error bit: the selection's counts were inconsistent
 
-struct AttnParams {
-  const float *S;
-  const __nv_bfloat16 *V;
-  const int32_t *idx;
-  float *part;              // [B*Hq, nsplit, d + 4] partial states (m, Z, pad, pad, N[d])
+struct SaParams {
+  const float *S;           // [B*Hq, ldS] scores
+  uint32_t *hist;           // [B*Hq, kHistBins] digit-1 histogram (left zero by the select)
+  uint2 *list;              // [B*Hq, ldL] (position, order key) of the threshold-bin keys
+  const __nv_bfloat16 *V;   // [B, Hkv, cap, d]
+  int32_t *idx;             // [B*Hq, k]: written (select) or read (attention only)
   float *out;               // [B*Hq, d]
-  uint32_t *meta;
-  long long ldS, cap, N;
-  long long s1, w0, nW, k_eff;
-  int k, Hq, G, Hkv, nsplit, R, B;
-  int nWsplit;              // static-set CTAs per KV head, wrange rows of W each
-  int nOsplit;              // retrieved-set CTAs per query head, orange rows of Omega each
-  long long wrange, orange; // multiples of kAttnRange
+  uint32_t *err;            // error word
+  long long ldS, ldL, cap, N;
+  long long s1, w0, nW, nC, k_eff;   // W = [0, s1) u [w0, N), C = [s1, w0)
+  long long cbase, cper;    // CTA r of a cluster owns candidates [cbase + r cper, + cper)
+  int k, Hq, G, Hkv, mode;
 };
 
 struct DenseParams {
@@ -93,16 +88,12 @@ struct AppendParams {
 
 // tuning constants the host layout needs
 constexpr int kScoreTile = 128;
-constexpr int kAttnRange = 64;      // entries of U a sparse-attention CTA takes at a time
-constexpr int kAttnWave = 768;      // about one wave of sparse-attention CTAs on 148 SMs
-constexpr int kTopkChunk = 8192;    // positions per top-k CTA
-constexpr int kTopkBucket = 4096;   // (b1, b2) bucket entries kept per query head
 constexpr int kDenseTile = 128;
 
 int num_sms();
 
-// Bytes of the counter block at the front of every workspace for `rows` query heads
-// (digit-1 and digit-2 histograms, then the per-row counters), 256-byte aligned sections.
+// Bytes of the counter block at the front of every workspace for `rows` query heads (the
+// digit-1 histograms, then the per-row counters), 256-byte aligned sections.
 size_t counter_block_bytes(size_t rows);
 
 // Raises a kernel's dynamic shared-memory limit once per device (so that later launches,
@@ -110,8 +101,10 @@ size_t counter_block_bytes(size_t rows);
 cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]);
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s);
-cudaError_t launch_topk(const TopkParams &p, cudaStream_t s);
-cudaError_t launch_sparse_attn(const AttnParams &p, int d, cudaStream_t s);
+// Cluster size for one query head: a power of two <= kMaxCluster (16 only where the device
+// schedules 16-CTA clusters of this kernel), chunks of at most 64K scores, grown to fill the GPU.
+int select_cluster_size(long long nC, int R, int d);
+cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s);
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
 

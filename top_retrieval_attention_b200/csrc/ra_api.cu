@@ -48,7 +48,7 @@ static constexpr size_t kAlign = 256;
 size_t counter_block_bytes(size_t rows) {
   const size_t h = (rows * kHistBins * 4 + kAlign - 1) / kAlign * kAlign;
   const size_t m = (rows * kMetaWords * 4 + kAlign - 1) / kAlign * kAlign;
-  return 2 * h + m;
+  return h + m;
 }
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 static long long round4(long long x) { return (x + 3) / 4 * 4; }
@@ -57,9 +57,9 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Derived sizes of one decode step (positions follow the slide "The GPU keeps 640 fixed
 // positions": W = [0, s1) u [w0, N), candidates C = [s1, w0)).
 struct Step {
-  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, nsplit, nsplit_cap, nWsplit, nOsplit;
-  long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldC, wrange, orange;
-  size_t off_S, off_hist, off_hist2, off_meta, off_cand, off_buck, off_part, total;
+  int B, Hq, Hkv, G, d, k, n_sink, n_window, R, ncl;
+  long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldL, cbase, cper;
+  size_t off_S, off_hist, off_meta, off_list, total;
 };
 
 static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
@@ -78,36 +78,27 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.nC = st.w0 - st.s1;
   st.k_eff = std::min<long long>(k, st.nC);
   st.ldS = round4(std::max<long long>(N, 1));
-  st.ldC = round4(std::max<long long>(st.nC, 1));
-  // sparse attention splits: W per KV head and Omega per query head, in ranges of whole
-  // 64-entry groups sized so that the retrieved CTAs make about one wave
-  {
-    const long long per_head = std::max<long long>(1, kAttnWave / st.R);
-    const long long quads = static_cast<long long>(B) * Hkv * ((Hq / Hkv + 3) / 4);
-    const long long per_group = std::max<long long>(1, kAttnWave / 3 / quads);
-    auto rng = [](long long n, long long parts) {
-      const long long groups = (n + kAttnRange - 1) / kAttnRange;
-      return std::max<long long>(1, (groups + parts - 1) / parts) * kAttnRange;
-    };
-    st.orange = rng(st.k_eff, per_head);
-    st.wrange = rng(st.nW, per_group);
-    st.nOsplit = static_cast<int>((st.k_eff + st.orange - 1) / st.orange);
-    st.nWsplit = static_cast<int>((st.nW + st.wrange - 1) / st.wrange);
-    st.nsplit = std::max(1, st.nWsplit + st.nOsplit);
-    // the layout must not depend on Hkv (the workspace size is asked without it): reserve
-    // partial states for the largest static split count, one per 64 rows of W
-    st.nsplit_cap = std::max(1, static_cast<int>((st.nW + kAttnRange - 1) / kAttnRange) + st.nOsplit);
-  }
+  st.ldL = round4(std::max<long long>(st.nC, 1));
+  st.ncl = 1;
+  st.cbase = st.s1 & ~3LL;
+  st.cper = round4(std::max<long long>(st.w0 - st.cbase, 1));
   size_t off = 0;
   st.off_hist = off;  off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
-  st.off_hist2 = off; off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_meta = off;  off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
   st.off_S = off;     off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
-  st.off_cand = off;  off = align_up(off + static_cast<size_t>(st.R) * st.ldC * 8);
-  st.off_buck = off;  off = align_up(off + static_cast<size_t>(st.R) * kTopkBucket * 8);
-  st.off_part = off; off = align_up(off + static_cast<size_t>(st.R) * st.nsplit_cap * (d + 4) * 4);
+  // the threshold-bin lists are needed only when the selection is a proper subset of C
+  st.off_list = off;
+  if (st.k_eff > 0 && st.k_eff < st.nC) off = align_up(off + static_cast<size_t>(st.R) * st.ldL * 8);
   st.total = off;
   return RA_OK;
+}
+
+// The selection's cluster split of C (host only, so the workspace size stays a pure function of
+// the shape): chunks start at multiples of 4 so the CTAs read the score row in float4 units.
+static void plan_clusters(Step &st) {
+  st.ncl = select_cluster_size(st.nC, st.R, st.d);
+  const long long span = std::max<long long>(st.w0 - st.cbase, 1);
+  st.cper = round4((span + st.ncl - 1) / st.ncl);
 }
 
 static ra_status check_kv(const ra_kv *kv) {
@@ -130,6 +121,7 @@ static ra_status plan_step(const ra_kv *kv, int Hq, int k, int n_sink, int n_win
   if (kv->N == 0 || st.nW + st.k_eff == 0) return RA_ERR_EMPTY;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return RA_ERR_WORKSPACE;
   if (ws_bytes < st.total) return RA_ERR_WORKSPACE;
+  plan_clusters(st);
   return RA_OK;
 }
 
@@ -154,39 +146,24 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
 
-static ra_status run_topk(const Step &st, int32_t *idx, void *ws, cudaStream_t stream) {
-  if (st.k == 0) return RA_OK;
-  TopkParams p{};
+// Selection (kSaSelect), attention (kSaAttend) or both in one launch.
+static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, int32_t *idx,
+                                   float *out, void *ws, cudaStream_t stream) {
+  if (mode == kSaSelect && st.k == 0) return RA_OK;
+  SaParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
   p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
-  p.hist2 = reinterpret_cast<uint32_t *>(at(ws, st.off_hist2));
-  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
-  p.cand = reinterpret_cast<uint2 *>(at(ws, st.off_cand));
-  p.bucket = reinterpret_cast<uint2 *>(at(ws, st.off_buck));
-  p.idx = idx;
-  p.ldS = st.ldS; p.ldC = st.ldC; p.N = st.N;
-  p.cand_lo = st.s1; p.cand_hi = st.w0; p.nC = st.nC; p.k_eff = st.k_eff;
-  p.k = st.k; p.R = st.R;
-  cudaError_t e = launch_topk(p, stream);
-  return e == cudaSuccess ? RA_OK : cuda_fail(e, "topk");
-}
-
-static ra_status run_attn(const ra_kv *kv, const Step &st, const int32_t *idx, float *out,
-                          void *ws, cudaStream_t stream) {
-  AttnParams p{};
-  p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
+  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.idx = idx;
-  p.part = reinterpret_cast<float *>(at(ws, st.off_part));
   p.out = out;
-  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
-  p.ldS = st.ldS; p.cap = st.cap; p.N = st.N;
-  p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.k_eff = st.k_eff;
-  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.nsplit = st.nsplit; p.R = st.R;
-  p.B = st.B; p.nWsplit = st.nWsplit; p.nOsplit = st.nOsplit;
-  p.wrange = st.wrange; p.orange = st.orange;
-  cudaError_t e = launch_sparse_attn(p, st.d, stream);
-  return e == cudaSuccess ? RA_OK : cuda_fail(e, "sparse_attn");
+  p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+  p.ldS = st.ldS; p.ldL = st.ldL; p.cap = st.cap; p.N = st.N;
+  p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.nC = st.nC; p.k_eff = st.k_eff;
+  p.cbase = st.cbase; p.cper = st.cper;
+  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.mode = mode;
+  const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "select_attend");
 }
 
 // Dense flash-decode split plan: as many splits per KV head as keep the grid close to a
@@ -202,7 +179,7 @@ static int dense_nsplit_cap(long long N) {
 // Kernels leave it zero when they finish, so a workspace zero-filled once stays usable by
 // later calls with the same B * Hq (whatever N), sparse and dense alike.
 static size_t counter_bytes(int R, size_t *off_meta) {
-  const size_t m = 2 * align_up(static_cast<size_t>(R) * kHistBins * 4);
+  const size_t m = align_up(static_cast<size_t>(R) * kHistBins * 4);
   if (off_meta) *off_meta = m;
   return align_up(m + static_cast<size_t>(R) * kMetaWords * 4);
 }
@@ -280,7 +257,7 @@ ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
   ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
   if (s != RA_OK) return s;
   if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
-  return run_topk(st, idx, ws, reinterpret_cast<cudaStream_t>(stream));
+  return run_select_attend(kv, st, kSaSelect, idx, nullptr, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
@@ -290,7 +267,19 @@ ra_status ra_sparse_attn(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
   ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
   if (s != RA_OK) return s;
   if ((k > 0 && (!idx || !aligned16(idx))) || !out || !aligned16(out)) return RA_ERR_ARG;
-  return run_attn(kv, st, idx, out, ws, reinterpret_cast<cudaStream_t>(stream));
+  return run_select_attend(kv, st, kSaAttend, const_cast<int32_t *>(idx), out, ws,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_select_attend(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
+                           int32_t n_window, int32_t *idx, float *out, void *ws, size_t ws_bytes,
+                           ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if ((k > 0 && (!idx || !aligned16(idx))) || !out || !aligned16(out)) return RA_ERR_ARG;
+  return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, int32_t n_sink,
@@ -304,9 +293,7 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   s = run_score(kv, q, st, ws, cs);
   if (s != RA_OK) return s;
-  s = run_topk(st, idx, ws, cs);
-  if (s != RA_OK) return s;
-  return run_attn(kv, st, idx, out, ws, cs);
+  return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws, cs);
 }
 
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d) {

@@ -1,0 +1,727 @@
+// Exact per-query-head top-k selection fused with the sparse attention over the selected set
+// (RetrievalAttention slides: "The GPU keeps 640 fixed positions" -- W and Omega disjoint, one
+// index set per query head; "Sparse attention renormalizes selected tokens" -- Eq. (2) over
+// U = W u Omega; "Two local softmax outputs need global weights" -- Eqs. (3)-(5)).
+//
+// One thread-block cluster per query head (b, h); the cluster's CTAs split the head's
+// candidate positions C = [s1, w0) into contiguous chunks.
+//
+// Selection, a radix select over the 64-bit composite x = order_key(z) << 32 | ~position (all
+// keys distinct: larger z first, equal z to the lower position):
+//   * digit 1 (the top 11 bits of order_key) was histogrammed by the score kernel; every CTA
+//     finds the threshold bin b1 (the bin of the k-th largest key) from it;
+//   * one streaming pass over the CTA's chunk of scores keeps the positions of the keys above
+//     b1 ("sure") in shared memory, keeps the keys in b1 (the "list") in shared memory, past
+//     its capacity in the CTA's slice of a per-head list in the workspace, and histograms
+//     digit 2 of the list;
+//   * each later digit is settled across the cluster: every CTA sums one slice of the CTAs'
+//     digit histograms through distributed shared memory, the threshold digit is found from
+//     the slice totals, keys above it are written out at offsets from a cluster-wide prefix
+//     of per-CTA counts, and the keys at it either are all taken, or (at most 64 of them) are
+//     sent to the first CTA for a bitonic finish, or become the next round's domain;
+//   * a CTA with more sure keys than its shared array holds (very large k) writes them out from
+//     its chunk of the score row, re-read.
+// Attention: the CTAs split U (W first, then Omega from idx) into ranges; a warp takes 8
+// entries at a time (scores from the score row, V rows gathered 8 bytes per lane), keeps an
+// online-softmax state, the CTA combines its warps, and the first CTA merges the cluster's
+// partial states (m_S, Z_S, N_S) with weights e^{m_S - m} into the output.
+#include <cooperative_groups.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace ra {
+
+constexpr int kSaThreads = 256;
+constexpr int kSaWarps = kSaThreads / 32;
+constexpr int kSureCap = 4096;    // keys above b1 kept per CTA: positions
+constexpr int kListSmem = 1536;   // keys in b1 kept in shared memory per CTA (the rest in the
+                                  // CTA's slice of the workspace list)
+constexpr int kFinish = 64;       // bitonic finish size (one warp)
+constexpr int kStreamVec = 8;     // float4 score loads per thread in flight
+
+template <int D>
+struct SaSmem {
+  uint32_t sure[kSureCap];
+  uint2 list[kListSmem];          // (position, order key) of the first keys in b1
+  float wacc[kSaWarps * D];       // attention: per-warp numerators
+  uint32_t h[kHistBins];          // digit histogram of the current round (slice reduced in place)
+  unsigned long long fin[kFinish];  // first CTA: keys of the final bucket
+  float pacc[D];                  // this CTA's partial state (read by the first CTA)
+  float pm, pz;
+  float wm[kSaWarps], wz[kSaWarps];
+  uint32_t x_a[kMaxCluster];      // per-rank exchange slots (written remotely before a barrier)
+  uint32_t x_b[kMaxCluster];
+  uint32_t x_tot[kMaxCluster];
+  uint32_t warp_tot[2 * kSaWarps];
+  uint32_t n_sure, n_list;
+  int t_bin;
+  uint32_t t_above, t_cnt;
+};
+
+__device__ __forceinline__ unsigned long long composite(uint32_t key, uint32_t pos) {
+  return (static_cast<unsigned long long>(key) << 32) | (0xFFFFFFFFu - pos);
+}
+__device__ __forceinline__ uint32_t composite_pos(unsigned long long x) {
+  return 0xFFFFFFFFu - static_cast<uint32_t>(x);
+}
+
+// Block-wide inclusive prefix sums of two counters at once; warp_tot holds 2 * kSaWarps words.
+// Returns the inclusive sums; the block totals are left in tot_a / tot_b.
+__device__ __forceinline__ uint2 block_scan2(uint32_t a, uint32_t b, uint32_t *warp_tot,
+                                             uint32_t &tot_a, uint32_t &tot_b) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t na = __shfl_up_sync(0xffffffffu, a, o);
+    const uint32_t nb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += na;
+      b += nb;
+    }
+  }
+  if (lane == 31) {
+    warp_tot[warp] = a;
+    warp_tot[kSaWarps + warp] = b;
+  }
+  __syncthreads();
+  uint32_t pa = 0, pb = 0;
+  tot_a = 0;
+  tot_b = 0;
+#pragma unroll
+  for (int w = 0; w < kSaWarps; ++w) {
+    const uint32_t ta = warp_tot[w], tb = warp_tot[kSaWarps + w];
+    if (w < warp) {
+      pa += ta;
+      pb += tb;
+    }
+    tot_a += ta;
+    tot_b += tb;
+  }
+  __syncthreads();   // warp_tot may be reused
+  return make_uint2(a + pa, b + pb);
+}
+
+// Threshold in a histogram of nb bins (digit value ascending with the bin index): the bin that
+// holds the want-th largest key, counting base_above keys as already above every bin here.
+// Sets sm.t_bin (-1 if the bins hold fewer than want - base_above keys), sm.t_above (keys above
+// the bin, base_above included) and sm.t_cnt.  src is global memory written by an earlier kernel
+// (kGlobal, read through L2) or shared memory, possibly another CTA's.  Whole block; the result
+// is valid after the call.
+template <int D, bool kGlobal>
+__device__ __forceinline__ void find_thresh(SaSmem<D> &sm, const uint32_t *src, int nb,
+                                            uint32_t want, uint32_t base_above) {
+  const int tid = threadIdx.x;
+  const int per = (nb + kSaThreads - 1) / kSaThreads;   // <= 8 bins per thread
+  uint32_t loc[8];
+  uint32_t s = 0;
+  // thread t owns bins [nb - per (t + 1), nb - per t): thread 0 the highest
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int bin = nb - per * (tid + 1) + (per - 1 - i);
+    loc[i] = (i < per && bin >= 0 && bin < nb) ? (kGlobal ? __ldcg(src + bin) : src[bin]) : 0u;
+    s += loc[i];
+  }
+  if (tid == 0) sm.t_bin = -1;
+  uint32_t ta, tb;
+  const uint2 incl = block_scan2(s, 0u, sm.warp_tot, ta, tb);
+  const uint32_t excl = base_above + incl.x - s;
+  if (excl < want && want <= excl + s) {
+    uint32_t cum = excl;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < per && cum + loc[i] >= want) {
+        sm.t_bin = nb - per * (tid + 1) + (per - 1 - i);
+        sm.t_above = cum;
+        sm.t_cnt = loc[i];
+        break;
+      }
+      cum += loc[i];
+    }
+  }
+  __syncthreads();
+}
+
+// The CTA's threshold-bin keys (position, order key): the first kListSmem in shared memory,
+// the rest in the CTA's slice of the head's list in the workspace (read back through L2).
+template <int D>
+struct ListSrc {
+  const SaSmem<D> *sm;
+  const uint2 *spill;
+  uint32_t n;
+  template <class F>
+  __device__ __forceinline__ void for_each(F f) const {
+    for (uint32_t i = threadIdx.x; i < n; i += kSaThreads) {
+      const uint2 e = i < static_cast<uint32_t>(kListSmem) ? sm->list[i] : __ldcg(spill + i);
+      f(composite(e.y, e.x));
+    }
+  }
+};
+
+// The CTA's candidates [lo, hi), re-read from the score row (float4 units from the aligned
+// chunk start a0).  Iteration order per thread is fixed, so a counting pass and a writing pass
+// agree on every thread's running offsets.
+struct ChunkSrc {
+  const float *srow;
+  long long a0, lo, hi;
+  template <class F>
+  __device__ __forceinline__ void for_each(F f) const {
+    for (long long b = a0 + 4LL * threadIdx.x; b < hi; b += 4LL * kSaThreads) {
+      if (b + 4 <= lo) continue;
+      const float4 v = __ldcg(reinterpret_cast<const float4 *>(srow + b));
+      const float zz[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long pos = b + e;
+        if (pos >= lo && pos < hi) f(composite(order_key(zz[e]), static_cast<uint32_t>(pos)));
+      }
+    }
+  }
+};
+
+// Bitonic finish in the first CTA: the n <= kFinish keys in sm.fin, the `want` largest written
+// to irow[o0 ..].  One warp.
+template <int D>
+__device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32_t want,
+                                               int32_t *irow, uint32_t o0) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (uint32_t i = n + tid; i < kFinish; i += kSaThreads) sm.fin[i] = 0ull;   // below every key
+  __syncthreads();
+  if (tid < 32) {
+#pragma unroll 1
+    for (int size = 2; size <= kFinish; size <<= 1) {
+#pragma unroll 1
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const int i = 2 * stride * (lane / stride) + (lane % stride);
+        const int j = i + stride;
+        const unsigned long long a = sm.fin[i], b = sm.fin[j];
+        const bool desc = (i & size) == 0;
+        if (desc ? (a < b) : (a > b)) {
+          sm.fin[i] = b;
+          sm.fin[j] = a;
+        }
+        __syncwarp();
+      }
+    }
+    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = static_cast<int32_t>(composite_pos(sm.fin[i]));
+  }
+}
+
+// Rounds below digit 1 over the keys of bin b1 (src): digit 2 first, whose histogram is already
+// complete in every CTA's sm.h with the cluster synchronised since, then further 11-bit digits
+// of the composite.  `want` keys are still to be chosen; they go to irow[base ..).  Every CTA of
+// the cluster runs the same rounds (all decisions come from cluster-wide totals).
+template <int D, class Src>
+__device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
+                              int ncl, const Src &src, uint32_t b1, uint32_t want, uint32_t base,
+                              int32_t *irow) {
+  const int tid = threadIdx.x;
+  const uint32_t k_eff = static_cast<uint32_t>(p.k_eff);
+  unsigned long long prefix = b1;
+  int sh = 64 - kHistBits;   // composite bits below digit 1
+  bool have_hist = true;
+#pragma unroll 1
+  for (int round = 0; round < 6 && sh > 0; ++round) {
+    const int w = sh < kHistBits ? sh : kHistBits;
+    const int nsh = sh - w;
+    const uint32_t mask = (1u << w) - 1u;
+    const int nb = 1 << w;
+    if (!have_hist) {
+      src.for_each([&](unsigned long long x) {
+        if ((x >> sh) == prefix) atomicAdd(&sm.h[static_cast<uint32_t>(x >> nsh) & mask], 1u);
+      });
+      __syncthreads();
+      cl.sync();   // every CTA's digit histogram is complete
+    }
+    have_hist = false;
+    // this CTA's slice of the cluster-summed histogram, in place; its total to every CTA
+    const int sz = nb / ncl;
+    const int s0 = rank * sz;
+    uint32_t part = 0;
+    for (int bin = s0 + tid; bin < s0 + sz; bin += kSaThreads) {
+      uint32_t s = 0;
+      for (int c = 0; c < ncl; ++c) s += cl.map_shared_rank(sm.h, c)[bin];
+      sm.h[bin] = s;
+      part += s;
+    }
+    uint32_t tot, unused;
+    block_scan2(part, 0u, sm.warp_tot, tot, unused);
+    if (tid < ncl) cl.map_shared_rank(sm.x_tot, tid)[rank] = tot;
+    cl.sync();   // slices summed, slice totals exchanged
+    // the slice holding the want-th largest key (highest slices first), then its digit
+    uint32_t above = 0;
+    int rs = ncl - 1;
+    for (; rs > 0; --rs) {
+      if (above + sm.x_tot[rs] >= want) break;
+      above += sm.x_tot[rs];
+    }
+    find_thresh<D, false>(sm, cl.map_shared_rank(sm.h, rs) + rs * sz, sz, want, above);
+    if (sm.t_bin < 0) {   // inconsistent counts (never for a score row and its own histogram)
+      if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);
+      return;
+    }
+    const uint32_t t = static_cast<uint32_t>(rs * sz + sm.t_bin);
+    const uint32_t up = sm.t_above;   // keys of the prefix above digit t, cluster-wide
+    const uint32_t eq = sm.t_cnt;     // keys of the prefix at digit t
+    const uint32_t want2 = want - up; // 1 <= want2 <= eq
+    const bool take_eq = want2 == eq;
+    const bool fin = !take_eq && eq <= static_cast<uint32_t>(kFinish);
+    uint32_t cu = 0, ce = 0;
+    src.for_each([&](unsigned long long x) {
+      if ((x >> sh) == prefix) {
+        const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
+        cu += dg > t ? 1u : 0u;
+        ce += dg == t ? 1u : 0u;
+      }
+    });
+    uint32_t tu, te;
+    const uint2 inc = block_scan2(cu, ce, sm.warp_tot, tu, te);
+    if (tid < ncl) {
+      cl.map_shared_rank(sm.x_a, tid)[rank] = tu;
+      cl.map_shared_rank(sm.x_b, tid)[rank] = te;
+    }
+    cl.sync();   // per-CTA counts exchanged
+    uint32_t off_u = 0, off_e = 0;
+    for (int c = 0; c < rank; ++c) {
+      off_u += sm.x_a[c];
+      off_e += sm.x_b[c];
+    }
+    uint32_t ou = base + off_u + inc.x - cu;
+    uint32_t oe = off_e + inc.y - ce;
+    unsigned long long *fin0 = cl.map_shared_rank(sm.fin, 0);
+    src.for_each([&](unsigned long long x) {
+      if ((x >> sh) != prefix) return;
+      const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
+      if (dg > t) {
+        if (ou < k_eff) irow[ou] = static_cast<int32_t>(composite_pos(x));
+        ++ou;
+      } else if (dg == t) {
+        if (take_eq) {
+          if (base + up + oe < k_eff) irow[base + up + oe] = static_cast<int32_t>(composite_pos(x));
+        } else if (fin && oe < static_cast<uint32_t>(kFinish)) {
+          fin0[oe] = x;
+        }
+        ++oe;
+      }
+    });
+    if (take_eq) return;
+    if (fin) {
+      cl.sync();   // the final bucket is complete in the first CTA
+      if (rank == 0) bitonic_finish(sm, eq, min(want2, k_eff - min(k_eff, base + up)), irow, base + up);
+      return;
+    }
+    // next digit: every remote read of sm.h came before the last barrier
+    for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
+    __syncthreads();
+    prefix = (prefix << w) | t;
+    sh = nsh;
+    want = want2;
+    base += up;
+  }
+  if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);   // unreachable for distinct keys
+}
+
+// Appends this lane's hit (if any) to sm.sure / sm.list with one shared atomic per list and
+// warp: all 32 lanes call it together.
+template <int D>
+__device__ __forceinline__ void place_hit(SaSmem<D> &sm, uint2 *spill, bool has, uint32_t pos,
+                                          float z, uint32_t b1, uint32_t lt) {
+  const uint32_t key = order_key(z);
+  const uint32_t d1 = key >> (32 - kHistBits);
+  const bool up = has && d1 > b1, eq = has && d1 == b1;
+  const uint32_t mu = __ballot_sync(0xffffffffu, up), me = __ballot_sync(0xffffffffu, eq);
+  uint32_t bu = 0, be = 0;
+  if ((threadIdx.x & 31) == 0) {
+    if (mu) bu = atomicAdd(&sm.n_sure, static_cast<uint32_t>(__popc(mu)));
+    if (me) be = atomicAdd(&sm.n_list, static_cast<uint32_t>(__popc(me)));
+  }
+  bu = __shfl_sync(0xffffffffu, bu, 0);
+  be = __shfl_sync(0xffffffffu, be, 0);
+  if (up) {
+    const uint32_t o = bu + __popc(mu & lt);
+    if (o < static_cast<uint32_t>(kSureCap)) sm.sure[o] = pos;
+  }
+  if (eq) {
+    const uint32_t o = be + __popc(me & lt);
+    const uint2 ent = make_uint2(pos, key);
+    if (o < static_cast<uint32_t>(kListSmem)) sm.list[o] = ent;
+    else spill[o] = ent;
+    atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+  }
+}
+
+// One pass over the CTA's candidates [lo, hi) of the score row: positions of keys above the
+// digit-1 threshold bin b1 go to sm.sure, keys in b1 to sm.list and, past its capacity, to
+// `spill` (room for hi - lo entries), with their digit-2 histogram in sm.h.  Hits (z >= zlo,
+// the bottom of bin b1) are a few percent of the keys: each thread makes a bit mask of its
+// hits with one compare per score, re-reads its first four hits (L1 or L2) with the loads in
+// flight together, and the warp places them in lock-step rounds; a lane with more hits places
+// the rest alone.  The counters keep counting past the capacities.
+template <int D>
+__device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, uint2 *spill,
+                                             long long a0, long long lo, long long hi,
+                                             uint32_t b1) {
+  constexpr long long kStep = 4LL * kSaThreads * kStreamVec;
+  static_assert(4 * kStreamVec <= 32, "one mask bit per score");
+  constexpr int kPre = 4;
+  const float zlo = key_float(b1 << (32 - kHistBits));
+  const uint32_t lt = lanemask_lt();
+  for (long long it = a0; it < hi; it += kStep) {
+    const long long b0 = it + 4LL * threadIdx.x;
+    float4 v[kStreamVec];
+#pragma unroll
+    for (int u = 0; u < kStreamVec; ++u) {
+      const long long b = b0 + 4LL * kSaThreads * u;
+      v[u] = (b < hi && b + 4 > lo) ? __ldg(reinterpret_cast<const float4 *>(srow + b))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const bool interior = it >= lo && it + kStep <= hi;
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < kStreamVec; ++u) {
+      uint32_t bits = (v[u].x >= zlo ? 1u : 0u) | (v[u].y >= zlo ? 2u : 0u) |
+                      (v[u].z >= zlo ? 4u : 0u) | (v[u].w >= zlo ? 8u : 0u);
+      if (!interior) {
+        const long long b = b0 + 4LL * kSaThreads * u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (b + e < lo || b + e >= hi) bits &= ~(1u << e);
+      }
+      m |= bits << (4 * u);
+    }
+    if (!__any_sync(0xffffffffu, m != 0u)) continue;
+    uint32_t pp[kPre];
+    float zz[kPre];
+    int np = 0;
+#pragma unroll
+    for (int r = 0; r < kPre; ++r) {
+      const int j = m ? __ffs(m) - 1 : 0;
+      pp[r] = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
+      np += m ? 1 : 0;
+      m &= m ? m - 1 : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < kPre; ++r) zz[r] = r < np ? __ldg(srow + pp[r]) : 0.f;
+    const int rounds = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(np));
+#pragma unroll
+    for (int r = 0; r < kPre; ++r)
+      if (r < rounds) place_hit(sm, spill, r < np, pp[r], zz[r], b1, lt);
+    // lanes with more than kPre hits (rare): one by one, all lanes in lock-step
+    while (__any_sync(0xffffffffu, m != 0u)) {
+      const bool has = m != 0u;
+      const int j = has ? __ffs(m) - 1 : 0;
+      m &= has ? m - 1 : 0u;
+      const uint32_t pos = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
+      place_hit(sm, spill, has, pos, has ? __ldg(srow + pos) : 0.f, b1, lt);
+    }
+  }
+}
+
+// Omega of one query head into irow (cluster-wide; every CTA takes the same branches).
+template <int D>
+__device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
+                             int ncl, int row) {
+  const int tid = threadIdx.x;
+  int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
+  if (rank == 0)
+    for (long long i = p.k_eff + tid; i < p.k; i += kSaThreads) irow[i] = -1;
+  if (p.k_eff == 0) return;
+  const long long a0 = p.cbase + static_cast<long long>(rank) * p.cper;
+  const long long lo = max(a0, p.s1), hi = min(a0 + p.cper, p.w0);
+  if (p.k_eff >= p.nC) {   // every candidate is selected
+    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - p.s1] = static_cast<int32_t>(i);
+    return;
+  }
+  const uint32_t k_eff = static_cast<uint32_t>(p.k_eff);
+  const float *srow = p.S + static_cast<long long>(row) * p.ldS;
+  uint32_t *h1 = p.hist + static_cast<long long>(row) * kHistBins;
+  for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
+  if (tid == 0) {
+    sm.n_sure = 0u;
+    sm.n_list = 0u;
+  }
+  // digit 1: the threshold bin of the score kernel's candidate histogram
+  find_thresh<D, true>(sm, h1, kHistBins, k_eff, 0u);
+  const int b1i = sm.t_bin;
+  const uint32_t above1 = sm.t_above;
+  const uint32_t b1 = b1i < 0 ? 0u : static_cast<uint32_t>(b1i);
+  uint2 *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - p.s1);
+  if (b1i >= 0) stream_chunk(sm, srow, spill, a0, lo, hi, b1);
+  __syncthreads();
+  if (tid < ncl) cl.map_shared_rank(sm.x_a, tid)[rank] = sm.n_sure;
+  cl.sync();   // lists, counts and digit-2 histograms complete; every CTA has read h1
+  if (b1i < 0) {   // the histogram does not count k_eff candidates: not this row's scores
+    if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);
+    return;
+  }
+  if (rank == 0)
+    for (int i = tid; i < kHistBins; i += kSaThreads) h1[i] = 0u;   // left zero for the next call
+  uint32_t off = 0;
+  for (int c = 0; c < rank; ++c) off += sm.x_a[c];
+  const ChunkSrc chunk{srow, a0, lo, hi};
+  // the keys above b1 take idx slots [0, above1), CTA by CTA
+  if (sm.n_sure <= static_cast<uint32_t>(kSureCap)) {
+    for (uint32_t i = tid; i < sm.n_sure; i += kSaThreads)
+      if (off + i < k_eff) irow[off + i] = static_cast<int32_t>(sm.sure[i]);
+  } else {   // more sure keys than sm.sure holds: from the chunk again
+    uint32_t cu = 0;
+    chunk.for_each([&](unsigned long long x) { cu += (x >> (64 - kHistBits)) > b1 ? 1u : 0u; });
+    uint32_t tu, unused;
+    const uint2 inc = block_scan2(cu, 0u, sm.warp_tot, tu, unused);
+    uint32_t o = off + inc.x - cu;
+    chunk.for_each([&](unsigned long long x) {
+      if ((x >> (64 - kHistBits)) > b1) {
+        if (o < k_eff) irow[o] = static_cast<int32_t>(composite_pos(x));
+        ++o;
+      }
+    });
+  }
+  // the keys of b1, from the CTAs' lists
+  select_rounds(p, sm, cl, rank, ncl, ListSrc<D>{&sm, spill, sm.n_list}, b1, k_eff - above1,
+                above1, irow);
+}
+
+// Softmax attention of one query head over U = W u Omega (Omega read from idx), split across
+// the cluster; the first CTA merges the partial states into out.  Each CTA stages its entries'
+// positions and scores in shared memory (in blocks of kStage), then its warps gather 16 V rows
+// at a time and keep online-softmax states.
+constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
+constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
+
+template <int D>
+__device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
+                             int ncl, int row) {
+  constexpr int CPL = D / 32;   // channels per lane
+  constexpr int kPer = kStage / kSaThreads;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long nU = p.nW + p.k_eff;
+  const long long per = (nU + ncl - 1) / ncl;
+  const long long e_lo = static_cast<long long>(rank) * per;
+  const long long e_hi = min(nU, e_lo + per);
+  const int b = row / p.Hq, h = row - b * p.Hq;
+  const __nv_bfloat16 *Vh = p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D;
+  const float *srow = p.S + static_cast<long long>(row) * p.ldS;
+  const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
+  int *spos = reinterpret_cast<int *>(sm.sure);
+  float *sz = reinterpret_cast<float *>(sm.sure + kStage);
+  float m = -INFINITY, zs = 0.f, acc[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  for (long long blk = e_lo; blk < e_hi; blk += kStage) {
+    const int nb = static_cast<int>(min(static_cast<long long>(kStage), e_hi - blk));
+    // positions (W computed, Omega from idx), then their scores: two rounds of loads in flight
+    int pp[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * kSaThreads;
+      const long long e = blk + i;
+      long long pos = -1;
+      if (i < nb) pos = e < p.nW ? (e < p.s1 ? e : p.w0 + (e - p.s1)) : __ldcg(irow + (e - p.nW));
+      pp[j] = (pos >= 0 && pos < p.N) ? static_cast<int>(pos) : -1;   // always, for a complete idx
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * kSaThreads;
+      const float z = pp[j] >= 0 ? __ldcg(srow + pp[j]) : -INFINITY;
+      if (i < nb) {
+        spos[i] = pp[j];
+        sz[i] = z;
+      }
+    }
+    __syncthreads();
+    for (int g = warp * kAttnRows; g < nb; g += kAttnRows * kSaWarps) {
+      const bool mine = lane < kAttnRows && g + lane < nb;
+      const int pos = mine ? spos[g + lane] : -1;
+      const float z = mine && pos >= 0 ? sz[g + lane] : -INFINITY;
+      uint32_t wv[kAttnRows][CPL / 2];
+#pragma unroll
+      for (int j = 0; j < kAttnRows; ++j) {
+        const int pj = __shfl_sync(0xffffffffu, pos, j);
+        if (pj >= 0) {
+          const __nv_bfloat16 *vr = Vh + static_cast<long long>(pj) * D;
+          if constexpr (CPL == 4) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(vr) + lane);
+            wv[j][0] = v.x;
+            wv[j][1] = v.y;
+          } else {
+            wv[j][0] = __ldg(reinterpret_cast<const uint32_t *>(vr) + lane);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < CPL / 2; ++c) wv[j][c] = 0u;
+        }
+      }
+      float mg = z;   // lanes >= 16 hold -inf; the xor partners stay within groups of 16
+#pragma unroll
+      for (int o = kAttnRows / 2; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
+      mg = __shfl_sync(0xffffffffu, mg, 0);
+      if (mg == -INFINITY) continue;   // warp-uniform: no entry in this group
+      const float mn = fmaxf(m, mg);
+      const float sc = expf(m - mn);   // 0 while m is -inf
+      const float pe = z == -INFINITY ? 0.f : expf(z - mn);
+      float ps = pe;
+#pragma unroll
+      for (int o = kAttnRows / 2; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+      ps = __shfl_sync(0xffffffffu, ps, 0);
+      zs = zs * sc + ps;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[c] *= sc;
+#pragma unroll
+      for (int j = 0; j < kAttnRows; ++j) {
+        const float pj = __shfl_sync(0xffffffffu, pe, j);
+#pragma unroll
+        for (int c = 0; c < CPL / 2; ++c) {
+          acc[2 * c] += pj * bf16_lo(wv[j][c]);
+          acc[2 * c + 1] += pj * bf16_hi(wv[j][c]);
+        }
+      }
+      m = mn;
+    }
+    __syncthreads();   // the staging area is reused by the next block
+  }
+  // the CTA's warps -> one partial state (m_S, Z_S, N_S) in this CTA's shared memory
+  if (lane == 0) {
+    sm.wm[warp] = m;
+    sm.wz[warp] = zs;
+  }
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) sm.wacc[warp * D + lane * CPL + c] = acc[c];
+  __syncthreads();
+  float M = sm.wm[0];
+#pragma unroll
+  for (int i = 1; i < kSaWarps; ++i) M = fmaxf(M, sm.wm[i]);
+  float ew[kSaWarps];
+#pragma unroll
+  for (int i = 0; i < kSaWarps; ++i) ew[i] = sm.wm[i] == -INFINITY ? 0.f : expf(sm.wm[i] - M);
+  for (int c = tid; c < D; c += kSaThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSaWarps; ++i) s += ew[i] * sm.wacc[i * D + c];
+    sm.pacc[c] = s;
+  }
+  if (tid == 0) {
+    float zt = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSaWarps; ++i) zt += ew[i] * sm.wz[i];
+    sm.pm = M;
+    sm.pz = zt;
+  }
+  cl.sync();   // every CTA's partial state is ready
+  if (rank == 0) {
+    float Mx = -INFINITY;
+    for (int c = 0; c < ncl; ++c) Mx = fmaxf(Mx, cl.map_shared_rank(&sm.pm, c)[0]);
+    float den = 0.f;
+    for (int c = 0; c < ncl; ++c) {
+      const float mc = cl.map_shared_rank(&sm.pm, c)[0];
+      if (mc != -INFINITY) den += expf(mc - Mx) * cl.map_shared_rank(&sm.pz, c)[0];
+    }
+    for (int ch = tid; ch < D; ch += kSaThreads) {
+      float num = 0.f;
+      for (int c = 0; c < ncl; ++c) {
+        const float mc = cl.map_shared_rank(&sm.pm, c)[0];
+        if (mc != -INFINITY) num += expf(mc - Mx) * cl.map_shared_rank(sm.pacc, c)[ch];
+      }
+      p.out[static_cast<long long>(row) * D + ch] = num / den;
+    }
+  }
+  cl.sync();   // the first CTA has read every partial state
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaParams p) {
+  __shared__ SaSmem<D> sm;
+  cg::cluster_group cl = cg::this_cluster();
+  const int ncl = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int row = blockIdx.y;
+  pdl_trigger();
+  pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
+  if (p.mode & kSaSelect) select_phase<D>(p, sm, cl, rank, ncl, row);
+  if (p.mode & kSaAttend) {
+    if (p.mode & kSaSelect) {
+      __threadfence();
+      cl.sync();   // Omega complete in idx and visible to the cluster
+    }
+    attend_phase<D>(p, sm, cl, rank, ncl, row);
+  } else {
+    cl.sync();   // no CTA leaves while the cluster may still use its shared memory
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+// Clusters of `ncl` CTAs of this kernel that the device runs at once (0 if it cannot run
+// them), queried once per device and size.
+template <int D>
+static int active_clusters_t(int ncl) {
+  static int cache[64][5];
+  static bool done[64][5] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ncl <= 8 ? 1 : 0;
+  int li = 0;
+  while ((1 << li) < ncl) ++li;
+  if (!done[dev][li]) {
+    if (ncl > 8)
+      (void)cudaFuncSetAttribute(select_attend_kernel<D>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ncl), 1);
+    cfg.blockDim = dim3(kSaThreads);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(ncl);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, select_attend_kernel<D>, &cfg) != cudaSuccess) n = 0;
+    (void)cudaGetLastError();   // a refused query leaves no error behind
+    cache[dev][li] = n;
+    done[dev][li] = true;
+  }
+  return cache[dev][li];
+}
+
+// The cluster size of a query head (a power of two <= kMaxCluster): chunks of at most 64K
+// candidates (a head whose threshold bin is crowded then spreads over several CTAs), grown while
+// the clusters of all R heads still run in one wave and chunks keep at least 4096 candidates;
+// a size whose last wave would be nearly empty is halved.
+int select_cluster_size(long long nC, int R, int d) {
+  auto active = [d](int n) { return d == 128 ? active_clusters_t<128>(n) : active_clusters_t<64>(n); };
+  int n = 1;
+  while (n < kMaxCluster && 65536LL * n < nC && active(2 * n) > 0) n *= 2;
+  while (n < kMaxCluster && nC >= 8192LL * n && active(2 * n) >= R) n *= 2;
+  const int a = active(n);
+  if (n > 1 && a > 0 && R > a && (R % a) * 4 < a && active(n / 2) > 0) n /= 2;
+  return n;
+}
+
+template <int D>
+static cudaError_t launch_sa_t(const SaParams &p, int R, int ncl, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ncl), static_cast<unsigned>(R));
+  cfg.blockDim = dim3(kSaThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ncl);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D>, p);
+}
+
+cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s) {
+  if (ncl < 1 || ncl > kMaxCluster || (ncl & (ncl - 1)) != 0) return cudaErrorInvalidValue;
+  return d == 128 ? launch_sa_t<128>(p, R, ncl, s) : launch_sa_t<64>(p, R, ncl, s);
+}
+
+}  // namespace ra

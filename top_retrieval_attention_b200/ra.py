@@ -20,7 +20,7 @@ RA_OK, RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_CAPACITY, RA_ERR_WORKSPACE, RA_ERR_CUDA,
 #: every symbol include/ra.h declares
 EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
-           "ra_sparse_attn", "ra_dense_workspace_bytes", "ra_dense_decode",
+           "ra_sparse_attn", "ra_select_attend", "ra_dense_workspace_bytes", "ra_dense_decode",
            "ra_decode_step_static")
 
 
@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
                                          c_size_t, c_void_p]),
             "ra_sparse_attn": (c_int32, [P, c_int32, c_int32, c_int32, c_int32, c_void_p, c_void_p,
                                          c_void_p, c_size_t, c_void_p]),
+            "ra_select_attend": (c_int32, [P, c_int32, c_int32, c_int32, c_int32, c_void_p,
+                                           c_void_p, c_void_p, c_size_t, c_void_p]),
             "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
             "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                                           c_void_p]),
@@ -109,6 +111,11 @@ def ra_topk_select(kv, Hq, k, n_sink, n_window, idx, ws, ws_bytes, stream):
 def ra_sparse_attn(kv, Hq, k, n_sink, n_window, idx, out, ws, ws_bytes, stream):
     return lib().ra_sparse_attn(ctypes.byref(kv), Hq, k, n_sink, n_window, idx, out, ws,
                                 ws_bytes, stream)
+
+
+def ra_select_attend(kv, Hq, k, n_sink, n_window, idx, out, ws, ws_bytes, stream):
+    return lib().ra_select_attend(ctypes.byref(kv), Hq, k, n_sink, n_window, idx, out, ws,
+                                  ws_bytes, stream)
 
 
 def ra_decode_step_static(kv, q, Hq, k, n_sink, n_window, out, idx, stream):
