@@ -51,6 +51,7 @@ struct ScoreParams {
 constexpr int kSaSelect = 1;
 constexpr int kSaAttend = 2;
 constexpr int kMaxCluster = 16;        // CTAs per query head at most
+constexpr int kMaxAttnSplit = 4;       // clusters per query head in the attention-only launch
 constexpr int kDigit2Shift = 10;       // digit 2 = bits [10, 21) of the order key
 constexpr uint32_t kErrSelect = 4u;    // error bit: the selection's counts were inconsistent
 
@@ -61,11 +62,14 @@ struct SaParams {
   const __nv_bfloat16 *V;   // [B, Hkv, cap, d]
   int32_t *idx;             // [B*Hq, k]: written (select) or read (attention only)
   float *out;               // [B*Hq, d]
+  float *part;              // [B*Hq, kMaxAttnSplit, d + 4] partial states of the clusters
+  uint32_t *meta;           // [B*Hq, kMetaWords] counters (kDone left zero)
   uint32_t *err;            // error word
   long long ldS, ldL, cap, N;
   long long s1, w0, nW, nC, k_eff;   // W = [0, s1) u [w0, N), C = [s1, w0)
   long long cbase, cper;    // CTA r of a cluster owns candidates [cbase + r cper, + cper)
   int k, Hq, G, Hkv, mode;
+  int nsplit;               // clusters per query head (grid z); > 1 only for attention alone
 };
 
 struct DenseParams {
@@ -104,6 +108,9 @@ cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s);
 // Cluster size for one query head: a power of two <= kMaxCluster (16 only where the device
 // schedules 16-CTA clusters of this kernel), chunks of at most 64K scores, grown to fill the GPU.
 int select_cluster_size(long long nC, int R, int d);
+// Clusters per query head for the attention over nU entries on its own: 1 while a CTA of one
+// cluster takes at most 1024 entries, else up to kMaxAttnSplit while all clusters run in one wave.
+int attn_split(long long nU, int R, int ncl, int d);
 cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s);
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);

@@ -59,7 +59,7 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 struct Step {
   int B, Hq, Hkv, G, d, k, n_sink, n_window, R, ncl;
   long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldL, cbase, cper;
-  size_t off_S, off_hist, off_meta, off_list, total;
+  size_t off_S, off_hist, off_meta, off_list, off_part, total;
 };
 
 static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
@@ -89,6 +89,7 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   // the threshold-bin lists are needed only when the selection is a proper subset of C
   st.off_list = off;
   if (st.k_eff > 0 && st.k_eff < st.nC) off = align_up(off + static_cast<size_t>(st.R) * st.ldL * 8);
+  st.off_part = off;  off = align_up(off + static_cast<size_t>(st.R) * kMaxAttnSplit * (d + 4) * 4);
   st.total = off;
   return RA_OK;
 }
@@ -146,7 +147,9 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
 
-// Selection (kSaSelect), attention (kSaAttend) or both in one launch.
+// Selection (kSaSelect), attention (kSaAttend) or both.  Both run in one launch unless the
+// attention is large enough to want more clusters per head than the selection uses (then it is
+// a second launch with nsplit clusters per head).
 static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, int32_t *idx,
                                    float *out, void *ws, cudaStream_t stream) {
   if (mode == kSaSelect && st.k == 0) return RA_OK;
@@ -157,13 +160,25 @@ static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, in
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.idx = idx;
   p.out = out;
+  p.part = reinterpret_cast<float *>(at(ws, st.off_part));
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
   p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
   p.ldS = st.ldS; p.ldL = st.ldL; p.cap = st.cap; p.N = st.N;
   p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.nC = st.nC; p.k_eff = st.k_eff;
   p.cbase = st.cbase; p.cper = st.cper;
-  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv; p.mode = mode;
+  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
+  const int split = (mode & kSaAttend) ? attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d) : 1;
+  if (mode & kSaSelect) {
+    p.mode = split == 1 ? mode : kSaSelect;   // the attention joins the launch when it can
+    p.nsplit = 1;
+    const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "select_attend");
+    if (p.mode == mode) return RA_OK;
+  }
+  p.mode = kSaAttend;
+  p.nsplit = split;
   const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
-  return e == cudaSuccess ? RA_OK : cuda_fail(e, "select_attend");
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "attend");
 }
 
 // Dense flash-decode split plan: as many splits per KV head as keep the grid close to a

@@ -30,6 +30,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "merge.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -44,7 +45,7 @@ constexpr int kFinish = 64;       // bitonic finish size (one warp)
 constexpr int kStreamVec = 8;     // float4 score loads per thread in flight
 
 template <int D>
-struct SaSmem {
+struct __align__(16) SaSmem {
   uint32_t sure[kSureCap];
   uint2 list[kListSmem];          // (position, order key) of the first keys in b1
   float wacc[kSaWarps * D];       // attention: per-warp numerators
@@ -485,9 +486,10 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
 }
 
 // Softmax attention of one query head over U = W u Omega (Omega read from idx), split across
-// the cluster; the first CTA merges the partial states into out.  Each CTA stages its entries'
-// positions and scores in shared memory (in blocks of kStage), then its warps gather 16 V rows
-// at a time and keep online-softmax states.
+// the nsplit clusters of the head (grid z) and the CTAs of each; the first CTA of a cluster
+// merges the cluster's partial states, and with several clusters the last one to finish merges
+// theirs (Eqs. (3)-(5)).  Each CTA stages its entries' positions and scores in shared memory (in
+// blocks of kStage), then its warps gather 16 V rows at a time and keep online-softmax states.
 constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
 constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
 
@@ -498,8 +500,9 @@ __device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   constexpr int kPer = kStage / kSaThreads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long nU = p.nW + p.k_eff;
-  const long long per = (nU + ncl - 1) / ncl;
-  const long long e_lo = static_cast<long long>(rank) * per;
+  const long long parts = static_cast<long long>(ncl) * p.nsplit;
+  const long long per = (nU + parts - 1) / parts;
+  const long long e_lo = (static_cast<long long>(blockIdx.z) * ncl + rank) * per;
   const long long e_hi = min(nU, e_lo + per);
   const int b = row / p.Hq, h = row - b * p.Hq;
   const __nv_bfloat16 *Vh = p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D;
@@ -618,13 +621,38 @@ __device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
       const float mc = cl.map_shared_rank(&sm.pm, c)[0];
       if (mc != -INFINITY) den += expf(mc - Mx) * cl.map_shared_rank(&sm.pz, c)[0];
     }
+    // one cluster: the output; several: this cluster's state for the last one to merge
+    constexpr int PS = D + kPartPad;
+    float *prow = p.part + static_cast<long long>(row) * kMaxAttnSplit * PS;
+    float *mine = prow + static_cast<long long>(blockIdx.z) * PS;
     for (int ch = tid; ch < D; ch += kSaThreads) {
       float num = 0.f;
       for (int c = 0; c < ncl; ++c) {
         const float mc = cl.map_shared_rank(&sm.pm, c)[0];
         if (mc != -INFINITY) num += expf(mc - Mx) * cl.map_shared_rank(sm.pacc, c)[ch];
       }
-      p.out[static_cast<long long>(row) * D + ch] = num / den;
+      if (p.nsplit == 1) p.out[static_cast<long long>(row) * D + ch] = num / den;
+      else mine[kPartPad + ch] = num;
+    }
+    if (p.nsplit > 1) {
+      if (tid == 0) {
+        mine[0] = Mx;
+        mine[1] = den;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        const uint32_t prev = atomicAdd(p.meta + static_cast<long long>(row) * kMetaWords + kDone, 1u);
+        sm.t_bin = prev == static_cast<uint32_t>(p.nsplit - 1) ? 1 : 0;
+        if (sm.t_bin) __threadfence();
+      }
+      __syncthreads();
+      if (sm.t_bin) {   // the head's last cluster: merge the nsplit states
+        merge_states<D, kSaThreads>(prow, p.nsplit, p.out + static_cast<long long>(row) * D,
+                                    reinterpret_cast<float *>(sm.warp_tot),
+                                    reinterpret_cast<float *>(sm.sure));
+        if (tid == 0) p.meta[static_cast<long long>(row) * kMetaWords + kDone] = 0u;
+      }
     }
   }
   cl.sync();   // the first CTA has read every partial state
@@ -703,7 +731,8 @@ int select_cluster_size(long long nC, int R, int d) {
 template <int D>
 static cudaError_t launch_sa_t(const SaParams &p, int R, int ncl, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(ncl), static_cast<unsigned>(R));
+  cfg.gridDim = dim3(static_cast<unsigned>(ncl), static_cast<unsigned>(R),
+                     static_cast<unsigned>(p.nsplit < 1 ? 1 : p.nsplit));
   cfg.blockDim = dim3(kSaThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -719,8 +748,18 @@ static cudaError_t launch_sa_t(const SaParams &p, int R, int ncl, cudaStream_t s
   return cudaLaunchKernelEx(&cfg, select_attend_kernel<D>, p);
 }
 
+int attn_split(long long nU, int R, int ncl, int d) {
+  if (nU <= 1024LL * ncl) return 1;
+  const int a = d == 128 ? active_clusters_t<128>(ncl) : active_clusters_t<64>(ncl);
+  int n = 1;
+  while (2 * n <= kMaxAttnSplit && static_cast<long long>(R) * 2 * n <= a && nU > 512LL * ncl * n) n *= 2;
+  return n;
+}
+
 cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s) {
   if (ncl < 1 || ncl > kMaxCluster || (ncl & (ncl - 1)) != 0) return cudaErrorInvalidValue;
+  if (p.nsplit < 1 || p.nsplit > kMaxAttnSplit || (p.nsplit > 1 && (p.mode & kSaSelect)))
+    return cudaErrorInvalidValue;
   return d == 128 ? launch_sa_t<128>(p, R, ncl, s) : launch_sa_t<64>(p, R, ncl, s);
 }
 
