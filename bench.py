@@ -40,14 +40,15 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one score-kernel launch, from an ncu capture,
-# keyed by the sha256 of the score kernel's sources it was taken on (so a changed kernel
-# reports null until it is captured again).  Values are per launch of the named workload.
-TRAFFIC = {}
+# keyed by the sha256 of the score kernel's own sources (score.cu and its TMA helpers) it was
+# taken on, so a changed kernel reports null until it is captured again.  Values are per launch
+# of the named workload (profiles/score_gqa_l8b_128k.md).
+TRAFFIC = {("063948ee6f144422", "l8b_128k_k1pct"): 275.65e6}
 
 
 def score_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("score.cu", "common.cuh", "kernels.h"):
+    for f in ("score.cu", "tma.cuh", "tmap.cu"):
         with open(os.path.join(ROOT, "top_retrieval_attention_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

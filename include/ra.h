@@ -156,7 +156,7 @@ ra_status ra_select_attend(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sin
  *   Scratch: a 64 MiB array inside libra (a file-scope __device__ array), held on every GPU
  *     that loads the library until the process exits.  A shape whose
  *     ra_decode_workspace_bytes(...) exceeds 64 MiB is rejected with RA_ERR_WORKSPACE before
- *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 17 MiB).
+ *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 48 MiB).
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream capture.
  *   Each call clears the scratch's counter block with cudaMemsetAsync on `stream`; nothing is

@@ -36,7 +36,7 @@ def test_static_variant_matches_the_workspace_entry_point_twice_in_a_row():
     from parity import check_out
     from synth import gen
 
-    w = gen.workload("l8b_128k_k1pct")          # needs about 50 MiB of scratch
+    w = gen.workload("l8b_128k_k1pct")          # needs about 48 MiB of scratch
     need = ra.ra_decode_workspace_bytes(w.B, w.Hq, w.N, w.d, w.k, w.n_sink, w.n_window)
     assert 0 < need <= 64 << 20
     cache, q0, _ = cache_from_workload(w)
