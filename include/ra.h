@@ -167,6 +167,35 @@ ra_status ra_decode_step_static(const ra_kv *kv, const void *q, int32_t Hq, int3
                                 int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
                                 ra_stream_t stream);
 
+/*
+ * Exact top-k of a batch of prefill queries: for every query row (b, h, m) of q, Omega = the
+ * min(k, |C|) largest z_i = q[b,h,m] . K[b,h/G,i] / sqrt(d) over the candidates C = [0,N) \ W,
+ * ties to the lower position (the decode step's selection, one query at a time; no causal mask).
+ * These are the nearest-key lists the slides build the query-aware index from (slide
+ * "Query-aware index construction": prefill queries and their top-k keys).  With G * M query
+ * rows per KV head the scores are a dense contraction, computed on the tcgen05 tensor cores
+ * (bf16 x bf16 -> fp32 in tensor memory).
+ *   q   : bf16 [B, Hq, M, d], device.   M >= 1, B * M <= 65535.
+ *   idx : int32 [B, Hq, M, k], device (may be NULL only when k == 0); entries past
+ *         min(k, |C|) are -1; order within a row unspecified.
+ *   ws  : at least ra_prefill_workspace_bytes(...) bytes, 256-byte aligned (no zero-fill
+ *         needed).  It holds the fp32 scores of every query row (B * Hq * M * N * 4 bytes).
+ * The two phases ra_prefill_score (scores into ws) and ra_prefill_select (idx from ws), run in
+ * that order with the same arguments, are ra_prefill_topk.
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_EMPTY (N == 0), RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ */
+size_t ra_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t M, int64_t N, int32_t d,
+                                  int32_t k, int32_t n_sink, int32_t n_window);
+ra_status ra_prefill_topk(const ra_kv *kv, const void *q, int32_t Hq, int32_t M, int32_t k,
+                          int32_t n_sink, int32_t n_window, int32_t *idx, void *ws,
+                          size_t ws_bytes, ra_stream_t stream);
+ra_status ra_prefill_score(const ra_kv *kv, const void *q, int32_t Hq, int32_t M, int32_t k,
+                           int32_t n_sink, int32_t n_window, void *ws, size_t ws_bytes,
+                           ra_stream_t stream);
+ra_status ra_prefill_select(const ra_kv *kv, int32_t Hq, int32_t M, int32_t k, int32_t n_sink,
+                            int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
+                            ra_stream_t stream);
+
 /* Workspace bytes for ra_dense_decode (split partial states).  0 for an invalid shape. */
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d);
 

@@ -197,3 +197,35 @@ def dense_decode(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray) -> 
         for h in range(Hq):
             out[b, h] = dense_head(q_bits[b, h], K_bits[b, h // G], V_bits[b, h // G])
     return out
+
+
+# ------------------------------------------------------------------------------------
+# exact top-k of the prefill queries (slide "Prefill queries teach the key graph what
+# matters": the prefill queries' exact top-k keys are the links the index is built from)
+
+
+def prefill_score_matrix(Q_bits: np.ndarray, K_bits: np.ndarray) -> np.ndarray:
+    """Z[m, i] = q_m k_i^T / sqrt(d) for the M queries of one head against its N keys
+    (Eq. (1) for every query at once: one matrix product, exact on bf16 inputs in fp64)."""
+    Q = bf16_to_f64(Q_bits)
+    K = bf16_to_f64(K_bits)
+    return (Q @ K.T) / math.sqrt(K.shape[1])
+
+
+def prefill_topk(Q_bits: np.ndarray, K_bits: np.ndarray, k: int, n_sink: int,
+                 n_window: int):
+    """Omega for every prefill query: Q [B, Hq, M, d], K [B, Hkv, N, d] (bf16 bits).
+    Query row (b, h, m) scores the keys of KV head h // G and keeps the min(k, |C|) largest
+    over the same candidates C as the decode step (ties to the lower position).
+    Returns a [B][Hq][M] nested list of position arrays."""
+    B, Hq, M, _ = Q_bits.shape
+    Hkv, N = K_bits.shape[1], K_bits.shape[2]
+    G = Hq // Hkv
+    C = candidate_set(N, n_sink, n_window)
+    out = [[[None] * M for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            Z = prefill_score_matrix(Q_bits[b, h], K_bits[b, h // G])
+            for m in range(M):
+                out[b][h][m] = select_topk(Z[m], C, k)
+    return out

@@ -375,3 +375,64 @@ def test_kv_capacity_table1():
     for label, gb in rows:
         cap = thousands[label] * 1000 * per_token / 2**30
         assert abs(cap - float(gb)) <= 0.06, (label, cap, gb)
+
+
+# ---------------------------------------------------------------- prefill queries' top-k
+
+
+def test_prefill_score_matrix_matches_exact_rationals():
+    """Z = Q K^T / sqrt(d) for a batch of queries: every entry against Fraction arithmetic
+    (d = 64, so the scale 1/8 is exact), catching a transposed operand or wrong scale."""
+    d = 64
+    Q = rand_bf16((5, d))
+    K = rand_bf16((7, d))
+    Z = oracle.prefill_score_matrix(Q, K)
+    Qf = oracle.bf16_to_f64(Q)
+    Kf = oracle.bf16_to_f64(K)
+    for m in range(5):
+        for i in range(7):
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(Qf[m], Kf[i])) / 8
+            assert abs(Z[m, i] - float(exact)) <= 4e-16 * d * max(1.0, abs(float(exact)))
+
+
+@pytest.mark.parametrize("trial", range(12))
+def test_prefill_topk_brute_force(trial):
+    """Every query row of a tiny batch: the returned set is the unique k-subset of C that
+    dominates the rest pairwise under exactly computed scores (ties to the lower position),
+    with query head h reading KV head h // G."""
+    rng = np.random.default_rng(100 + trial)
+    B, Hkv, G, M, N, d = 1, 2, 2, 3, int(rng.integers(2, 11)), 64
+    n_sink, n_window = int(rng.integers(0, 2)), int(rng.integers(0, 2))
+    # few distinct values so that exact score ties occur
+    Q = gen.f64_to_bf16_bits(rng.integers(-2, 3, size=(B, Hkv * G, M, d)).astype(np.float64))
+    K = gen.f64_to_bf16_bits(rng.integers(-1, 2, size=(B, Hkv, N, d)).astype(np.float64))
+    C = oracle.candidate_set(N, n_sink, n_window).tolist()
+    for k in (0, 1, 2, 5):
+        om = oracle.prefill_topk(Q, K, k, n_sink, n_window)
+        k_eff = min(k, len(C))
+        for h in range(Hkv * G):
+            Kf = oracle.bf16_to_f64(K[0, h // G])
+            for m in range(M):
+                qf = oracle.bf16_to_f64(Q[0, h, m])
+                z = {i: sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(qf, Kf[i]))
+                     for i in C}
+                winners = [set(S) for S in itertools.combinations(C, k_eff)
+                           if all(_dominates(z[a], a, z[b], b)
+                                  for a in S for b in C if b not in S)]
+                assert len(winners) == 1
+                assert set(om[0][h][m].tolist()) == winners[0]
+
+
+def test_prefill_topk_rows_are_decode_selections():
+    """A prefill query's selection is the decode step's selection for that query alone (the
+    decode oracle scores by a matrix-vector product, the prefill oracle by a matrix product)."""
+    B, Hq, Hkv, M, N, d = 2, 4, 2, 6, 300, 128
+    Q = rand_bf16((B, Hq, M, d))
+    K = rand_bf16((B, Hkv, N, d))
+    V = rand_bf16((B, Hkv, N, d))
+    om = oracle.prefill_topk(Q, K, 20, 4, 16)
+    for m in range(M):
+        _, dec = oracle.decode_step(np.ascontiguousarray(Q[:, :, m]), K, V, 20, 4, 16)
+        for b in range(B):
+            for h in range(Hq):
+                assert np.array_equal(np.sort(om[b][h][m]), np.sort(dec[b][h]))

@@ -50,6 +50,7 @@ struct ScoreParams {
 // from the scores, idx and V; both in one launch for the decode step.
 constexpr int kSaSelect = 1;
 constexpr int kSaAttend = 2;
+constexpr int kSaBuildHist = 4;        // with kSaSelect: build the digit-1 histogram from S first
 constexpr int kMaxCluster = 16;        // CTAs per query head at most
 constexpr int kMaxAttnSplit = 4;       // clusters per query head in the attention-only launch
 constexpr int kDigit2Shift = 10;       // digit 2 = bits [10, 21) of the order key
@@ -71,6 +72,19 @@ struct SaParams {
   int k, Hq, G, Hkv, mode;
   int nsplit;               // clusters per query head (grid z); > 1 only for attention alone
 };
+
+// Scores of prefill queries (rows (b, h, m) of Q [B, Hq, M, d]) against the keys of their KV
+// head, on the tensor cores.
+struct PfParams {
+  const __nv_bfloat16 *Q;   // [B, Hq, M, d]
+  const __nv_bfloat16 *K;   // [B, Hkv, cap, d]
+  float *S;                 // [B*Hq*M, ldS]
+  uint32_t *err;            // error word (bit kErrPrefillWait: a copy or the MMAs never landed)
+  long long N, cap, ldS;
+  int B, Hq, Hkv, G, M;
+  float scale;
+};
+constexpr uint32_t kErrPrefillWait = 8u;
 
 struct DenseParams {
   const __nv_bfloat16 *K, *V, *q;
@@ -113,6 +127,7 @@ int select_cluster_size(long long nC, int R, int d);
 int attn_split(long long nU, int R, int ncl, int d);
 cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s);
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
+cudaError_t launch_prefill_score(const PfParams &p, int d, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
 
 }  // namespace ra

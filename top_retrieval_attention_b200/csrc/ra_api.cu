@@ -311,6 +311,59 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
   return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws, cs);
 }
 
+// ---- prefill: exact top-k of a batch of queries (rows (b, h, m) of Q [B, Hq, M, d])
+
+// The prefill plan is the decode plan with one row per query: B * M "sequences" of Hq heads.
+static ra_status plan_prefill(const ra_kv *kv, int Hq, int M, int k, int n_sink, int n_window,
+                              void *ws, size_t ws_bytes, Step &st) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (M < 1) return RA_ERR_ARG;
+  if (static_cast<long long>(kv->B) * M > 65535) return RA_ERR_SHAPE;
+  s = plan_shape(kv->B * M, Hq, kv->Hkv, kv->N, kv->d, k, n_sink, n_window, st);
+  if (s != RA_OK) return s;
+  st.cap = kv->cap;
+  if (kv->N == 0) return RA_ERR_EMPTY;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return RA_ERR_WORKSPACE;
+  if (ws_bytes < st.total) return RA_ERR_WORKSPACE;
+  plan_clusters(st);
+  return RA_OK;
+}
+
+static ra_status run_prefill_score(const ra_kv *kv, const void *q, int Hq, int M, const Step &st,
+                                   void *ws, cudaStream_t stream) {
+  PfParams p{};
+  p.Q = static_cast<const __nv_bfloat16 *>(q);
+  p.K = static_cast<const __nv_bfloat16 *>(kv->K);
+  p.S = reinterpret_cast<float *>(at(ws, st.off_S));
+  p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+  p.N = st.N; p.cap = st.cap; p.ldS = st.ldS;
+  p.B = kv->B; p.Hq = Hq; p.Hkv = kv->Hkv; p.G = Hq / kv->Hkv; p.M = M;
+  p.scale = 1.0f / sqrtf(static_cast<float>(kv->d));
+  const cudaError_t e = launch_prefill_score(p, kv->d, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "prefill_score");
+}
+
+static ra_status run_prefill_select(const Step &st, int32_t *idx, void *ws, cudaStream_t stream) {
+  if (st.k == 0) return RA_OK;
+  SaParams p{};
+  p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
+  p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
+  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
+  p.idx = idx;
+  p.part = reinterpret_cast<float *>(at(ws, st.off_part));
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
+  p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+  p.ldS = st.ldS; p.ldL = st.ldL; p.cap = st.cap; p.N = st.N;
+  p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.nC = st.nC; p.k_eff = st.k_eff;
+  p.cbase = st.cbase; p.cper = st.cper;
+  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
+  p.mode = kSaSelect | kSaBuildHist;
+  p.nsplit = 1;
+  const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "prefill_select");
+}
+
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d) {
   if (B < 1 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
   if (N >= (1LL << 31) - 1) return 0;
@@ -367,6 +420,48 @@ ra_status ra_dense_decode(const ra_kv *kv, const void *q, int32_t Hq, float *out
   p.err = reinterpret_cast<uint32_t *>(at(ws, off_meta)) + kError;
   const cudaError_t e = launch_dense(p, kv->d, cs);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "dense_decode");
+}
+
+size_t ra_prefill_workspace_bytes(int32_t B, int32_t Hq, int32_t M, int64_t N, int32_t d,
+                                  int32_t k, int32_t n_sink, int32_t n_window) {
+  if (B < 1 || M < 1 || static_cast<long long>(B) * M > 65535) return 0;
+  Step st{};
+  if (plan_shape(B * M, Hq, Hq, N, d, k, n_sink, n_window, st) != RA_OK) return 0;
+  return st.total;
+}
+
+ra_status ra_prefill_score(const ra_kv *kv, const void *q, int32_t Hq, int32_t M, int32_t k,
+                           int32_t n_sink, int32_t n_window, void *ws, size_t ws_bytes,
+                           ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_prefill(kv, Hq, M, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q)) return RA_ERR_ARG;
+  return run_prefill_score(kv, q, Hq, M, st, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_prefill_select(const ra_kv *kv, int32_t Hq, int32_t M, int32_t k, int32_t n_sink,
+                            int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
+                            ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_prefill(kv, Hq, M, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  return run_prefill_select(st, idx, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ra_status ra_prefill_topk(const ra_kv *kv, const void *q, int32_t Hq, int32_t M, int32_t k,
+                          int32_t n_sink, int32_t n_window, int32_t *idx, void *ws,
+                          size_t ws_bytes, ra_stream_t stream) {
+  Step st{};
+  ra_status s = plan_prefill(kv, Hq, M, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  s = run_prefill_score(kv, q, Hq, M, st, ws, cs);
+  if (s != RA_OK) return s;
+  return run_prefill_select(st, idx, ws, cs);
 }
 
 }  // extern "C"

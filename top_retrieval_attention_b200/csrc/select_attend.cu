@@ -189,6 +189,16 @@ template <int D>
 __device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32_t want,
                                                int32_t *irow, uint32_t o0) {
   const int tid = threadIdx.x, lane = tid & 31;
+  if (n <= 32) {   // one key per lane: a key is taken when fewer than `want` keys exceed it
+    if (tid < 32) {
+      const unsigned long long x = static_cast<uint32_t>(lane) < n ? sm.fin[lane] : 0ull;
+      uint32_t above = 0;
+      for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, x, j) > x ? 1u : 0u;
+      if (static_cast<uint32_t>(lane) < n && above < want)
+        irow[o0 + above] = static_cast<int32_t>(composite_pos(x));
+    }
+    return;
+  }
   for (uint32_t i = n + tid; i < kFinish; i += kSaThreads) sm.fin[i] = 0ull;   // below every key
   __syncthreads();
   if (tid < 32) {
@@ -209,6 +219,40 @@ __device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32
     }
     for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = static_cast<int32_t>(composite_pos(sm.fin[i]));
   }
+}
+
+// The cluster-wide threshold of one digit: every CTA's sm.h holds its histogram of nb bins
+// (nb >= ncl) and the cluster has synchronised since.  Each CTA sums its slice of the CTAs'
+// histograms in place (through distributed shared memory) and sends the slice total to every
+// CTA; after a barrier every CTA finds the slice holding the want-th largest key (highest
+// slices first) and the bin inside it.  Returns the slice's first bin; sm.t_bin (relative to
+// it, -1 if the counts are inconsistent), sm.t_above (keys above that bin, cluster-wide) and
+// sm.t_cnt are set.  Other CTAs read this CTA's sm.h until the caller's next cluster barrier.
+template <int D>
+__device__ int cluster_thresh(SaSmem<D> &sm, cg::cluster_group &cl, int rank, int ncl, int nb,
+                              uint32_t want) {
+  const int tid = threadIdx.x;
+  const int sz = nb / ncl;
+  const int s0 = rank * sz;
+  uint32_t part = 0;
+  for (int bin = s0 + tid; bin < s0 + sz; bin += kSaThreads) {
+    uint32_t s = 0;
+    for (int c = 0; c < ncl; ++c) s += cl.map_shared_rank(sm.h, c)[bin];
+    sm.h[bin] = s;
+    part += s;
+  }
+  uint32_t tot, unused;
+  block_scan2(part, 0u, sm.warp_tot, tot, unused);
+  if (tid < ncl) cl.map_shared_rank(sm.x_tot, tid)[rank] = tot;
+  cl.sync();   // slices summed, slice totals exchanged
+  uint32_t above = 0;
+  int rs = ncl - 1;
+  for (; rs > 0; --rs) {
+    if (above + sm.x_tot[rs] >= want) break;
+    above += sm.x_tot[rs];
+  }
+  find_thresh<D, false>(sm, cl.map_shared_rank(sm.h, rs) + rs * sz, sz, want, above);
+  return rs * sz;
 }
 
 // Rounds below digit 1 over the keys of bin b1 (src): digit 2 first, whose histogram is already
@@ -238,33 +282,12 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
       cl.sync();   // every CTA's digit histogram is complete
     }
     have_hist = false;
-    // this CTA's slice of the cluster-summed histogram, in place; its total to every CTA
-    const int sz = nb / ncl;
-    const int s0 = rank * sz;
-    uint32_t part = 0;
-    for (int bin = s0 + tid; bin < s0 + sz; bin += kSaThreads) {
-      uint32_t s = 0;
-      for (int c = 0; c < ncl; ++c) s += cl.map_shared_rank(sm.h, c)[bin];
-      sm.h[bin] = s;
-      part += s;
-    }
-    uint32_t tot, unused;
-    block_scan2(part, 0u, sm.warp_tot, tot, unused);
-    if (tid < ncl) cl.map_shared_rank(sm.x_tot, tid)[rank] = tot;
-    cl.sync();   // slices summed, slice totals exchanged
-    // the slice holding the want-th largest key (highest slices first), then its digit
-    uint32_t above = 0;
-    int rs = ncl - 1;
-    for (; rs > 0; --rs) {
-      if (above + sm.x_tot[rs] >= want) break;
-      above += sm.x_tot[rs];
-    }
-    find_thresh<D, false>(sm, cl.map_shared_rank(sm.h, rs) + rs * sz, sz, want, above);
+    const int base_bin = cluster_thresh(sm, cl, rank, ncl, nb, want);
     if (sm.t_bin < 0) {   // inconsistent counts (never for a score row and its own histogram)
       if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);
       return;
     }
-    const uint32_t t = static_cast<uint32_t>(rs * sz + sm.t_bin);
+    const uint32_t t = static_cast<uint32_t>(base_bin + sm.t_bin);
     const uint32_t up = sm.t_above;   // keys of the prefix above digit t, cluster-wide
     const uint32_t eq = sm.t_cnt;     // keys of the prefix at digit t
     const uint32_t want2 = want - up; // 1 <= want2 <= eq
@@ -444,9 +467,26 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
     sm.n_sure = 0u;
     sm.n_list = 0u;
   }
-  // digit 1: the threshold bin of the score kernel's candidate histogram
-  find_thresh<D, true>(sm, h1, kHistBins, k_eff, 0u);
-  const int b1i = sm.t_bin;
+  const bool build = (p.mode & kSaBuildHist) != 0;
+  int b1i;
+  if (build) {
+    // digit 1 from the scores themselves: this CTA's histogram, then the cluster's threshold
+    __syncthreads();
+    ChunkSrc{srow, a0, lo, hi}.for_each([&](unsigned long long x) {
+      atomicAdd(&sm.h[static_cast<uint32_t>(x >> (64 - kHistBits))], 1u);
+    });
+    __syncthreads();
+    cl.sync();   // every CTA's digit-1 histogram is complete
+    b1i = cluster_thresh(sm, cl, rank, ncl, kHistBins, k_eff);
+    b1i = sm.t_bin < 0 ? -1 : b1i + sm.t_bin;
+    cl.sync();   // every CTA has read the slices it needed: the histograms can be cleared
+    for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
+    __syncthreads();
+  } else {
+    // digit 1: the threshold bin of the score kernel's candidate histogram
+    find_thresh<D, true>(sm, h1, kHistBins, k_eff, 0u);
+    b1i = sm.t_bin;
+  }
   const uint32_t above1 = sm.t_above;
   const uint32_t b1 = b1i < 0 ? 0u : static_cast<uint32_t>(b1i);
   uint2 *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - p.s1);
@@ -458,7 +498,7 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
     if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);
     return;
   }
-  if (rank == 0)
+  if (rank == 0 && !build)
     for (int i = tid; i < kHistBins; i += kSaThreads) h1[i] = 0u;   // left zero for the next call
   uint32_t off = 0;
   for (int c = 0; c < rank; ++c) off += sm.x_a[c];
@@ -669,10 +709,7 @@ __global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaPa
   pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
   if (p.mode & kSaSelect) select_phase<D>(p, sm, cl, rank, ncl, row);
   if (p.mode & kSaAttend) {
-    if (p.mode & kSaSelect) {
-      __threadfence();
-      cl.sync();   // Omega complete in idx and visible to the cluster
-    }
+    if (p.mode & kSaSelect) cl.sync();   // Omega complete in idx (release/acquire at cluster scope)
     attend_phase<D>(p, sm, cl, rank, ncl, row);
   } else {
     cl.sync();   // no CTA leaves while the cluster may still use its shared memory

@@ -21,7 +21,8 @@ RA_OK, RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_CAPACITY, RA_ERR_WORKSPACE, RA_ERR_CUDA,
 EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
            "ra_sparse_attn", "ra_select_attend", "ra_dense_workspace_bytes", "ra_dense_decode",
-           "ra_decode_step_static")
+           "ra_decode_step_static", "ra_prefill_workspace_bytes", "ra_prefill_topk",
+           "ra_prefill_score", "ra_prefill_select")
 
 
 class ra_kv(ctypes.Structure):
@@ -60,6 +61,14 @@ def lib() -> ctypes.CDLL:
             "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
             "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                                           c_void_p]),
+            "ra_prefill_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int64, c_int32,
+                                                      c_int32, c_int32, c_int32]),
+            "ra_prefill_topk": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                          c_void_p, c_void_p, c_size_t, c_void_p]),
+            "ra_prefill_score": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32,
+                                           c_void_p, c_size_t, c_void_p]),
+            "ra_prefill_select": (c_int32, [P, c_int32, c_int32, c_int32, c_int32, c_int32, c_void_p,
+                                            c_void_p, c_size_t, c_void_p]),
             "ra_decode_step_static": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32,
                                                 c_void_p, c_void_p, c_void_p]),
         }
@@ -209,6 +218,42 @@ def decode_step(cache: KVCache, q, k: int, n_sink: int, n_window: int, out=None,
                          idx.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
           "ra_decode_step")
     return out, idx[..., :k]
+
+
+def ra_prefill_workspace_bytes(B, Hq, M, N, d, k, n_sink, n_window) -> int:
+    return lib().ra_prefill_workspace_bytes(B, Hq, M, N, d, k, n_sink, n_window)
+
+
+def ra_prefill_topk(kv, q, Hq, M, k, n_sink, n_window, idx, ws, ws_bytes, stream):
+    return lib().ra_prefill_topk(ctypes.byref(kv), q, Hq, M, k, n_sink, n_window, idx, ws,
+                                 ws_bytes, stream)
+
+
+def ra_prefill_score(kv, q, Hq, M, k, n_sink, n_window, ws, ws_bytes, stream):
+    return lib().ra_prefill_score(ctypes.byref(kv), q, Hq, M, k, n_sink, n_window, ws, ws_bytes,
+                                  stream)
+
+
+def ra_prefill_select(kv, Hq, M, k, n_sink, n_window, idx, ws, ws_bytes, stream):
+    return lib().ra_prefill_select(ctypes.byref(kv), Hq, M, k, n_sink, n_window, idx, ws,
+                                   ws_bytes, stream)
+
+
+def prefill_topk(cache: KVCache, q, k: int, n_sink: int, n_window: int, idx=None, ws=None,
+                 stream=None):
+    """Exact top-k keys of every prefill query q [B, Hq, M, d].  Returns idx int32 [B, Hq, M, k]."""
+    import torch
+    B, Hq, M, d = q.shape
+    if idx is None:
+        idx = torch.empty((B, Hq, M, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        n = ra_prefill_workspace_bytes(B, Hq, M, cache.N, d, k, n_sink, n_window)
+        if n == 0:
+            raise RaError(RA_ERR_SHAPE, "ra_prefill_workspace_bytes")
+        ws = torch.empty(n, dtype=torch.uint8, device=q.device)
+    check(ra_prefill_topk(cache.kv, q.data_ptr(), Hq, M, k, n_sink, n_window, idx.data_ptr(),
+                          ws.data_ptr(), ws.numel(), _stream(stream)), "ra_prefill_topk")
+    return idx[..., :k]
 
 
 def dense_workspace(cache: KVCache, Hq: int):
