@@ -65,6 +65,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--prefill-queries", type=int, default=0,
+                    help="instead of decode steps: exact top-k of this many prefill queries per "
+                         "query head (tensor-core scores + cluster selection), one layer")
     return ap.parse_args()
 
 
@@ -505,6 +508,100 @@ def run_ours(args, w, rank, local_rank, world, dist):
     return result
 
 
+def run_prefill(args, w, rank, local_rank, world, dist):
+    """Exact top-k of M prefill queries per query head against one layer's cache: the
+    tcgen05 score GEMM (timed on its own for its roofline) and the cluster selection."""
+    import ctypes
+
+    import torch
+
+    import top_retrieval_attention_b200 as ra
+    from synth import device as sdev
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    M = args.prefill_queries
+    B, Hq, Hkv, d, N, k = w.B, w.Hq, w.Hkv, w.d, w.N, w.k
+    c = ra.KVCache(B, Hkv, d, N, device=dev)
+    sdev.device_layer(w, 0, c.K, c.V)
+    c.N = N
+    P = 4
+    qpool = torch.empty((P, B, Hq, M, d), dtype=torch.bfloat16, device=dev)
+    for s in range(P):
+        sdev.fill_q(qpool[s].view(B, Hq * M, d), w.seed + 7919 * s + 31)
+    n = ra.ra_prefill_workspace_bytes(B, Hq, M, N, d, k, w.n_sink, w.n_window)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    idx = torch.empty((B, Hq, M, max(k, 1)), dtype=torch.int32, device=dev)
+
+    def step(s, ev=None):
+        q = qpool[s % P].data_ptr()
+        if ev is not None:
+            ev[0].record(stream)
+        ra.check(ra.ra_prefill_score(c.kv, q, Hq, M, k, w.n_sink, w.n_window, ws.data_ptr(), n, sp),
+                 "prefill_score")
+        if ev is not None:
+            ev[1].record(stream)
+        ra.check(ra.ra_prefill_select(c.kv, Hq, M, k, w.n_sink, w.n_window, idx.data_ptr(),
+                                      ws.data_ptr(), n, sp), "prefill_select")
+        if ev is not None:
+            ev[2].record(stream)
+
+    for s in range(max(3, args.warmup)):
+        step(s)
+    torch.cuda.synchronize()
+    steps = args.steps if args.steps is not None else 20
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    clk = Clocks(uuid)
+    clk.start()
+    barrier(dist, local_rank)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        step(s, evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, local_rank)
+    clocks = clk.stop()
+    ms = max_over_ranks(dist, t0.elapsed_time(t1), dev) / steps
+    score_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    select_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    R = B * Hq * M
+    flops = 2.0 * R * N * d
+    s_bytes = 4.0 * R * N
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            peaks = json.load(fh)
+    except Exception:
+        peaks = {}
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    tflops_peak = float(peaks.get("bf16_tflops", 1590.0))
+    return {
+        "metric": "prefill exact top-k queries/s (tcgen05 scores + cluster select)",
+        "value": world * R / (ms / 1000.0), "unit": "queries/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 / Irwin-Hall normals, Llama-3-8B-shaped cache)",
+        "config": dict(workload_config(w), prefill_queries_per_head=M, rows=R),
+        "roofline": {"kernel": "prefill_score_kernel (tcgen05)", "bound": "hbm",
+                     "achieved": s_bytes / (score_ms / 1000.0) / 1e9, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": s_bytes / (score_ms / 1000.0) / 1e9 / hbm_peak,
+                     "traffic": None, "algorithmic_bytes_per_launch": s_bytes,
+                     "tensor_tflops": flops / (score_ms / 1000.0) / 1e12,
+                     "tensor_frac_of_bf16_peak": flops / (score_ms / 1000.0) / 1e12 / tflops_peak},
+        "score_kernel_us": 1000.0 * score_ms, "select_us": 1000.0 * select_ms,
+        "gpu_launches": 2 * steps, "clocks": clocks,
+    }
+
+
 def main():
     args = parse()
     rank, local_rank, world = dist_info()
@@ -518,7 +615,10 @@ def main():
         raise SystemExit("bench.py needs a CUDA device (the product has no CPU path)")
     dist = dist_init(world, True)
     try:
-        res = run_ours(args, w, rank, local_rank, world, dist)
+        if args.prefill_queries > 0:
+            res = run_prefill(args, w, rank, local_rank, world, dist)
+        else:
+            res = run_ours(args, w, rank, local_rank, world, dist)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
