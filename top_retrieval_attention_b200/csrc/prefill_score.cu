@@ -10,9 +10,16 @@
 //   * the same thread issues d / 16 tcgen05.mma (M 128, N 256, K 16, bf16 x bf16 -> fp32) into
 //     256 columns of tensor memory and commits them to a second mbarrier;
 //   * the four warps read their 32 tensor-memory lanes (one query row per thread) with
-//     tcgen05.ld, 16 columns at a time, scale, and store fp32 scores.
+//     tcgen05.ld, 32 columns at a time, scale, and write them into a 128-byte-swizzled
+//     [128 rows][32 columns] fp32 box in shared memory (the key tile's buffer, free once the
+//     products are done); one thread stores each box with a TMA tensor store (full lines; rows
+//     past the KV head's G * M and keys past N are clipped by the tensor map), two boxes in
+//     flight.
 // Every wait is bounded (an error bit and an orderly exit instead of a hang); the tensor memory
 // is freed on every path.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -34,10 +41,14 @@ struct PfCfg {
   static constexpr size_t smem_bytes() { return 1024 + kABytes + kBBytes + 64; }
 };
 
+constexpr int kPfCols = 32;                   // columns per stored box
+constexpr int kPfBox = kPfM * kPfCols * 4;    // 16 KB
+
 template <int D>
 __global__ void __launch_bounds__(kPfThreads, 2)
     prefill_score_kernel(const __grid_constant__ CUtensorMap tmQ,
-                         const __grid_constant__ CUtensorMap tmK, const PfParams p) {
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmS, const PfParams p) {
   using C = PfCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -105,35 +116,66 @@ __global__ void __launch_bounds__(kPfThreads, 2)
       mbar_wait(bar_load, 0);
     }
   } else {
-    const long long hrow = static_cast<long long>(qb) * kPfM + warp * 32 + lane;   // in the head
-    const bool row_ok = hrow < head_rows;
-    float *srow = p.S + (row0 + warp * 32 + lane) * p.ldS;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int r = warp * 32 + lane;   // this thread's row in the tile and in the stored box
 #pragma unroll 1
-    for (int c = 0; c < kPfN; c += 16) {
-      uint32_t r[16];
-      tmem_ld16(tmem + lane_base + static_cast<uint32_t>(c), r);
+    for (int ch = 0; ch < kPfN / kPfCols; ++ch) {
+      const uint32_t buf = sB + (ch & 1) * kPfBox;
+      if (ch >= 2 && tid == 0) bulk_wait_group_read<1>();   // box ch - 2 has left this buffer
+      __syncthreads();
+      uint32_t v0[16], v1[16];
+      tmem_ld16(tmem + lane_base + static_cast<uint32_t>(ch * kPfCols), v0);
+      tmem_ld16(tmem + lane_base + static_cast<uint32_t>(ch * kPfCols + 16), v1);
       tmem_wait_ld();
-      const long long kc = key0 + c;
-      if (row_ok && kc < p.N) {
-        float z[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) z[j] = canon_zero(__uint_as_float(r[j]) * p.scale);
-        if (kc + 16 <= p.N) {
-#pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4 *>(srow + kc + j) = make_float4(z[j], z[j + 1], z[j + 2], z[j + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (kc + j < p.N) srow[kc + j] = z[j];
-        }
+      for (int c = 0; c < 8; ++c) {   // 16-byte chunk c of the row, at swizzled chunk c ^ (r % 8)
+        const uint32_t *w = c < 4 ? v0 + 4 * c : v1 + 4 * (c - 4);
+        const float4 f = make_float4(canon_zero(__uint_as_float(w[0]) * p.scale),
+                                     canon_zero(__uint_as_float(w[1]) * p.scale),
+                                     canon_zero(__uint_as_float(w[2]) * p.scale),
+                                     canon_zero(__uint_as_float(w[3]) * p.scale));
+        const uint32_t dst = buf + r * 128 + ((c ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(dst), "f"(f.x), "f"(f.y),
+                     "f"(f.z), "f"(f.w)
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tma_store_3d(&tmS, buf, static_cast<int>(key0) + ch * kPfCols, qb * kPfM, bg);
+        bulk_commit_group();
       }
     }
+    if (tid == 0) bulk_wait_group<0>();   // every store has finished before the CTA leaves
   }
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kPfN);
+}
+
+// Host: 3-D fp32 tensor map over the scores viewed as [B * Hkv heads][G * M rows][N keys] (rows
+// ldS floats apart) with a box of [1][128][32] and the 128-byte swizzle.
+static bool encode_scores_tmap(CUtensorMap *out, float *S, long long heads, long long head_rows,
+                               long long N, long long ldS) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(head_rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ldS) * 4,
+                                 static_cast<cuuint64_t>(ldS) * 4 * head_rows};
+  const cuuint32_t box[3] = {kPfCols, kPfM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D>
@@ -152,10 +194,14 @@ static cudaError_t launch_prefill_t(const PfParams &p, cudaStream_t s) {
                         static_cast<uint64_t>(p.B) * p.Hkv, kPfN, static_cast<uint64_t>(p.cap)))
     return cudaErrorInvalidValue;
   const long long head_rows = static_cast<long long>(p.G) * p.M;
+  CUtensorMap ts;
+  if (!encode_scores_tmap(&ts, p.S, static_cast<long long>(p.B) * p.Hkv, head_rows, p.N, p.ldS))
+    return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((p.N + kPfN - 1) / kPfN),
                   static_cast<unsigned>((head_rows + kPfM - 1) / kPfM),
                   static_cast<unsigned>(p.B * p.Hkv));
-  return launch_pdl(prefill_score_kernel<D>, grid, dim3(kPfThreads), C::smem_bytes(), s, tq, tk, p);
+  return launch_pdl(prefill_score_kernel<D>, grid, dim3(kPfThreads), C::smem_bytes(), s, tq, tk,
+                    ts, p);
 }
 
 cudaError_t launch_prefill_score(const PfParams &p, int d, cudaStream_t s) {
