@@ -122,6 +122,31 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
                          ra_stream_t stream);
 
 /*
+ * ra_decode_step with the retrieval set cut at a softmax-weight threshold (Eq. (2), slide
+ * "Sparse attention renormalizes selected tokens"): Omega = the candidates i of C whose full
+ * softmax weight a_i = e^{z_i} / sum_{j < N} e^{z_j} exceeds eps, the k largest of them when
+ * more than k pass (k is the budget cap).  U = W u Omega as in ra_decode_step.
+ *   eps : 0 < eps < 1.   idx : entries past |Omega| are -1 (|Omega| <= min(k, |C|)).
+ *   ws  : the ra_decode_workspace_bytes(...) workspace of the same k.
+ * Errors: as ra_decode_step; RA_ERR_ARG for eps outside (0, 1); RA_ERR_EMPTY when W is empty
+ * (the threshold may keep no key at all).
+ */
+ra_status ra_decode_step_eps(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, float eps,
+                             int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
+                             void *ws, size_t ws_bytes, ra_stream_t stream);
+
+/*
+ * Per-layer retrieval budgets in the PyramidKV style (slide "Extra experiments show where
+ * budget matters": an adaptive layer budget): k_out[l], l < L, falls linearly from k_max at
+ * layer 0 to ratio * k_max at layer L - 1 with mean k_mean (k_max = 2 k_mean / (1 + ratio)),
+ * each rounded down and the remainder given one each to the lowest layers, so that the budgets
+ * sum to exactly L * k_mean.  Host only (no device work).  Pass k_out[l] as layer l's k.
+ *   ratio in (0, 1] (1: every layer gets k_mean).   k_out: int32 [L], host, caller-owned.
+ * Errors: RA_ERR_ARG.
+ */
+ra_status ra_pyramid_budgets(int32_t L, int32_t k_mean, double ratio, int32_t *k_out);
+
+/*
  * The phases of ra_decode_step, exposed so a caller can time or interleave them.  All take the
  * arguments of ra_decode_step and the same workspace, and must run as one of the complete
  * sequences  ra_score_gqa, ra_select_attend  (which is ra_decode_step)  or

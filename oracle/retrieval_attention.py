@@ -229,3 +229,49 @@ def prefill_topk(Q_bits: np.ndarray, K_bits: np.ndarray, k: int, n_sink: int,
             for m in range(M):
                 out[b][h][m] = select_topk(Z[m], C, k)
     return out
+
+
+# ------------------------------------------------------------------------------------
+# threshold budget (Eq. (2): I_{t,eps} = {i : a_{t,i} > eps}, slide "Sparse attention
+# renormalizes selected tokens")
+
+
+def select_threshold(z: np.ndarray, C: np.ndarray, k: int, eps: float) -> np.ndarray:
+    """Omega under a threshold: the candidates whose full softmax weight a_i (over all N
+    positions, Eq. (1)) exceeds eps, cut to the k largest by (z descending, position ascending)
+    when more than k pass."""
+    a = softmax_weights(z)
+    C = np.asarray(C, dtype=np.int64)
+    passing = C[a[C] > eps]
+    return select_topk(z, passing, k)
+
+
+def decode_head_eps(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray, k: int,
+                    eps: float, n_sink: int, n_window: int):
+    """One query head under the threshold budget: returns (o [d], Omega, z)."""
+    q = bf16_to_f64(q_bits)
+    K = bf16_to_f64(K_bits)
+    V = bf16_to_f64(V_bits)
+    N = K.shape[0]
+    z = scores(q, K)
+    W = static_set(N, n_sink, n_window)
+    omega = select_threshold(z, candidate_set(N, n_sink, n_window), k, eps)
+    U = np.concatenate([W, omega])
+    if U.size == 0:
+        raise ValueError("empty selected union")
+    return attend(z, V, U), omega, z
+
+
+def pyramid_budgets(L: int, k_mean: int, ratio: float) -> np.ndarray:
+    """Per-layer budgets in the PyramidKV style (slide "Extra experiments show where budget
+    matters": a layer budget that shrinks with depth): an arithmetic progression from k_max at
+    layer 0 to ratio * k_max at layer L - 1 whose mean is k_mean, rounded down, with the
+    remainder given one each to the lowest layers so that the total is exactly L * k_mean."""
+    if L == 1:
+        return np.array([k_mean], dtype=np.int64)
+    k_max = 2.0 * k_mean / (1.0 + ratio)
+    exact = [k_max * (1.0 - (1.0 - ratio) * l / (L - 1)) for l in range(L)]
+    base = np.array([math.floor(x) for x in exact], dtype=np.int64)
+    rem = L * k_mean - int(base.sum())
+    base[:rem] += 1
+    return base

@@ -10,6 +10,8 @@
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 import oracle
@@ -65,3 +67,26 @@ def check_head(q_bits, K_bits, V_bits, k, n_sink, n_window, out_gpu, idx_gpu):
 
 def check_dense_head(q_bits, K_bits, V_bits, out_gpu):
     return check_out(out_gpu, oracle.dense_head(q_bits, K_bits, V_bits), "dense")
+
+
+def check_omega_eps(got_row: np.ndarray, z: np.ndarray, N: int, n_sink: int, n_window: int,
+                    k: int, eps: float):
+    """The threshold budget's Omega: the oracle's set except near the threshold (scores within
+    TIE_REL of T = ln eps + logsumexp(z), where fp32 and fp64 may decide differently) or near
+    the cap's k-th score; entries past the GPU's count must be -1."""
+    C = oracle.candidate_set(N, n_sink, n_window)
+    got_row = np.asarray(got_row, dtype=np.int64)
+    n_gpu = int(np.sum(got_row[:k] >= 0))
+    om_gpu = got_row[:n_gpu]
+    assert np.all(got_row[n_gpu:k] == -1), "kept keys must come first, then -1"
+    assert np.unique(om_gpu).size == n_gpu, "duplicate positions"
+    assert np.all(np.isin(om_gpu, C)), "position outside the candidates"
+    om = oracle.select_threshold(z, C, k, eps)
+    zmax = z.max()
+    T = math.log(eps) + zmax + math.log(np.exp(z - zmax).sum())
+    near = lambda a, ref: abs(z[a] - ref) <= TIE_REL * max(1.0, abs(ref))
+    s_k = z[om[-1]] if om.size == k else None
+    diff = set(om_gpu.tolist()) ^ set(om.tolist())
+    bad = [a for a in diff if not (near(a, T) or (s_k is not None and near(a, s_k)))]
+    assert not bad, f"{len(bad)} positions differ beyond the tolerance, e.g. {bad[:5]}"
+    return om_gpu

@@ -150,3 +150,37 @@ def test_product_never_imports_the_oracle():
                 assert not re.search(r"^\s*(import|from)\s+oracle", text, re.M), f
                 assert "oracle/" not in text, f
 
+
+
+def test_pyramid_budgets_match_the_oracle_and_reject_bad_arguments():
+    import oracle
+    for L in (1, 2, 3, 7, 32, 80):
+        for km in (0, 1, 7, 100, 1310, 20971):
+            for r in (0.1, 0.25, 0.5, 0.9, 1.0):
+                assert ra.pyramid_budgets(L, km, r) == list(oracle.pyramid_budgets(L, km, r))
+    out = (ctypes.c_int32 * 4)()
+    assert ra.lib().ra_pyramid_budgets(0, 10, 0.5, out) == ra.RA_ERR_ARG
+    assert ra.lib().ra_pyramid_budgets(4, 10, 0.0, out) == ra.RA_ERR_ARG
+    assert ra.lib().ra_pyramid_budgets(4, 10, 1.5, out) == ra.RA_ERR_ARG
+
+
+def test_threshold_step_rejects_bad_arguments():
+    kv = _kv()
+    big = 1 << 30
+    f = ra.lib().ra_decode_step_eps
+    assert f(ctypes.byref(kv), FAKE, 4, 10, 0.0, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert f(ctypes.byref(kv), FAKE, 4, 10, 1.0, 4, 8, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert f(ctypes.byref(kv), FAKE, 4, 10, 1e-3, 0, 0, FAKE, FAKE, FAKE, big, None) == ra.RA_ERR_EMPTY
+    assert f(ctypes.byref(kv), FAKE, 4, 10, 1e-3, 4, 8, FAKE, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
+
+
+def test_prefill_rejects_bad_arguments():
+    kv = _kv()
+    big = 1 << 30
+    L = ra.lib()
+    assert L.ra_prefill_topk(ctypes.byref(kv), 0, 4, 8, 10, 4, 8, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert L.ra_prefill_topk(ctypes.byref(kv), FAKE, 4, 0, 10, 4, 8, FAKE, FAKE, big, None) == ra.RA_ERR_ARG
+    assert L.ra_prefill_topk(ctypes.byref(kv), FAKE, 3, 8, 10, 4, 8, FAKE, FAKE, big, None) == ra.RA_ERR_SHAPE
+    assert L.ra_prefill_topk(ctypes.byref(kv), FAKE, 4, 8, 10, 4, 8, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
+    assert ra.ra_prefill_workspace_bytes(1, 4, 8, 100, 128, 10, 4, 8) > 4 * 8 * 100 * 4
+    assert ra.ra_prefill_workspace_bytes(1, 4, 0, 100, 128, 10, 4, 8) == 0

@@ -436,3 +436,59 @@ def test_prefill_topk_rows_are_decode_selections():
         for b in range(B):
             for h in range(Hq):
                 assert np.array_equal(np.sort(om[b][h][m]), np.sort(dec[b][h]))
+
+
+# ---------------------------------------------------------------- threshold budget (Eq. 2)
+
+
+def test_threshold_two_keys_logistic_closed_form():
+    """Two keys with z = (x, 0): a_0 = sigma(x) (the logistic function); key 0 passes a
+    threshold eps exactly when sigma(x) > eps (no static set, generous k)."""
+    for x in (-3.0, -0.5, 0.0, 0.7, 2.5):
+        z = np.array([x, 0.0])
+        for eps in (0.05, 0.3, 0.5, 0.8):
+            om = set(oracle.select_threshold(z, np.arange(2), 5, eps).tolist())
+            assert (0 in om) == (expit(x) > eps)
+            assert (1 in om) == (expit(-x) > eps)
+
+
+def test_threshold_set_is_eq2_set_and_top_k_cap():
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal(400) * 2.0
+    C = oracle.candidate_set(400, 3, 20)
+    for eps in (1e-4, 1e-3, 1e-2):
+        I = set(oracle.threshold_set(z, eps).tolist()) & set(C.tolist())   # Eq. (2) within C
+        assert set(oracle.select_threshold(z, C, 10**6, eps).tolist()) == I
+        om = oracle.select_threshold(z, C, 5, eps)
+        assert om.size == min(5, len(I))
+        assert set(om.tolist()) <= I
+        if len(I) > 5:   # the cap keeps the largest scores
+            assert min(z[om]) >= max(z[list(I - set(om.tolist()))])
+    # a vanishing threshold is the plain top-k; no two keys can both exceed one half
+    assert np.array_equal(np.sort(oracle.select_threshold(z, C, 30, 1e-300)),
+                          np.sort(oracle.select_topk(z, C, 30)))
+    assert oracle.select_threshold(z, C, 30, 0.5).size <= 1
+
+
+def test_threshold_weights_use_the_full_softmax():
+    """The weights are Eq. (1)'s over all N positions, sinks and window included: raising a
+    window key's score lowers every candidate's weight."""
+    z = np.array([1.0, 1.0, 1.0, 1.0, 0.0])
+    C = oracle.candidate_set(5, 0, 1)                 # the window is position 4
+    a_before = 1.0 / (4.0 + math.exp(-1.0))          # weight of each of the four candidates
+    eps = a_before * 0.999
+    assert oracle.select_threshold(z, C, 10, eps).size == 4
+    z2 = z.copy()
+    z2[4] = 5.0                                       # the window key takes most of the mass
+    assert oracle.select_threshold(z2, C, 10, eps).size == 0
+
+
+def test_pyramid_budgets_shape():
+    for L, km, r in ((32, 2621, 0.25), (7, 100, 0.5), (5, 3, 1.0), (1, 9, 0.3), (80, 20971, 0.1)):
+        b = oracle.pyramid_budgets(L, km, r)
+        assert b.size == L and int(b.sum()) == L * km
+        assert np.all(np.diff(b) <= 0)                        # shrinks with depth
+        k_max = 2.0 * km / (1.0 + r)
+        if L > 1:
+            assert abs(b[0] - k_max) <= 1 and abs(b[-1] - r * k_max) <= 1
+    assert list(oracle.pyramid_budgets(6, 11, 1.0)) == [11] * 6

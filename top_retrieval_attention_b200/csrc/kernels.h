@@ -51,6 +51,7 @@ struct ScoreParams {
 constexpr int kSaSelect = 1;
 constexpr int kSaAttend = 2;
 constexpr int kSaBuildHist = 4;        // with kSaSelect: build the digit-1 histogram from S first
+constexpr int kSaEps = 8;              // with kSaSelect: keep only keys whose softmax weight > eps
 constexpr int kMaxCluster = 16;        // CTAs per query head at most
 constexpr int kMaxAttnSplit = 4;       // clusters per query head in the attention-only launch
 constexpr int kDigit2Shift = 10;       // digit 2 = bits [10, 21) of the order key
@@ -71,6 +72,7 @@ struct SaParams {
   long long cbase, cper;    // CTA r of a cluster owns candidates [cbase + r cper, + cper)
   int k, Hq, G, Hkv, mode;
   int nsplit;               // clusters per query head (grid z); > 1 only for attention alone
+  float log_eps;            // kSaEps: ln(eps)
 };
 
 // Scores of prefill queries (rows (b, h, m) of Q [B, Hq, M, d]) against the keys of their KV

@@ -2,6 +2,7 @@
 // Every check runs on the host before anything is enqueued; the library allocates nothing.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <math.h>
 #include <stdio.h>
 
 #include <algorithm>
@@ -129,7 +130,7 @@ static ra_status plan_step(const ra_kv *kv, int Hq, int k, int n_sink, int n_win
 static uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
 
 static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void *ws,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool hist = true) {
   ScoreParams p{};
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -141,7 +142,7 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   p.total_tiles = p.tiles_per_head * st.B * st.Hkv;
   p.B = st.B; p.Hkv = st.Hkv; p.G = st.G; p.Hq = st.Hq;
   p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
-  p.do_hist = st.k_eff > 0 && st.k_eff < st.nC;
+  p.do_hist = hist && st.k_eff > 0 && st.k_eff < st.nC;
   p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
   const cudaError_t e = launch_score(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
@@ -151,7 +152,8 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
 // attention is large enough to want more clusters per head than the selection uses (then it is
 // a second launch with nsplit clusters per head).
 static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, int32_t *idx,
-                                   float *out, void *ws, cudaStream_t stream) {
+                                   float *out, void *ws, cudaStream_t stream,
+                                   float log_eps = 0.f) {
   if (mode == kSaSelect && st.k == 0) return RA_OK;
   SaParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
@@ -167,15 +169,18 @@ static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, in
   p.s1 = st.s1; p.w0 = st.w0; p.nW = st.nW; p.nC = st.nC; p.k_eff = st.k_eff;
   p.cbase = st.cbase; p.cper = st.cper;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
+  p.log_eps = log_eps;
   const int split = (mode & kSaAttend) ? attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d) : 1;
   if (mode & kSaSelect) {
-    p.mode = split == 1 ? mode : kSaSelect;   // the attention joins the launch when it can
+    // the attention joins the launch when it can
+    p.mode = split == 1 ? mode : (mode & ~kSaAttend);
     p.nsplit = 1;
     const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend");
     if (p.mode == mode) return RA_OK;
   }
   p.mode = kSaAttend;
+  p.log_eps = 0.f;
   p.nsplit = split;
   const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "attend");
@@ -364,6 +369,22 @@ static ra_status run_prefill_select(const Step &st, int32_t *idx, void *ws, cuda
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "prefill_select");
 }
 
+ra_status ra_decode_step_eps(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, float eps,
+                             int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
+                             void *ws, size_t ws_bytes, ra_stream_t stream) {
+  if (!(eps > 0.0f && eps < 1.0f)) return RA_ERR_ARG;
+  Step st{};
+  ra_status s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+  if (s != RA_OK) return s;
+  if (st.nW == 0) return RA_ERR_EMPTY;   // the threshold may keep no key: W must be non-empty
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  s = run_score(kv, q, st, ws, cs, /*hist=*/false);   // the selection counts against the threshold
+  if (s != RA_OK) return s;
+  return run_select_attend(kv, st, kSaSelect | kSaAttend | kSaEps, idx, out, ws, cs, logf(eps));
+}
+
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d) {
   if (B < 1 || Hq < 1 || N < 0 || (d != 64 && d != 128)) return 0;
   if (N >= (1LL << 31) - 1) return 0;
@@ -462,6 +483,25 @@ ra_status ra_prefill_topk(const ra_kv *kv, const void *q, int32_t Hq, int32_t M,
   s = run_prefill_score(kv, q, Hq, M, st, ws, cs);
   if (s != RA_OK) return s;
   return run_prefill_select(st, idx, ws, cs);
+}
+
+ra_status ra_pyramid_budgets(int32_t L, int32_t k_mean, double ratio, int32_t *k_out) {
+  if (L < 1 || k_mean < 0 || !(ratio > 0.0 && ratio <= 1.0) || !k_out) return RA_ERR_ARG;
+  if (L == 1) {
+    k_out[0] = k_mean;
+    return RA_OK;
+  }
+  const double k_max = 2.0 * k_mean / (1.0 + ratio);
+  long long total = 0;
+  for (int32_t l = 0; l < L; ++l) {
+    const double x = k_max * (1.0 - (1.0 - ratio) * l / (L - 1));
+    k_out[l] = static_cast<int32_t>(floor(x));
+    total += k_out[l];
+  }
+  // the rounding remainder goes one by one to the lowest layers: the total is L * k_mean
+  const long long rem = static_cast<long long>(L) * k_mean - total;
+  for (long long l = 0; l < rem && l < L; ++l) k_out[l] += 1;
+  return RA_OK;
 }
 
 }  // extern "C"

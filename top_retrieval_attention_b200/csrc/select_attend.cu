@@ -57,6 +57,7 @@ struct __align__(16) SaSmem {
   uint32_t x_a[kMaxCluster];      // per-rank exchange slots (written remotely before a barrier)
   uint32_t x_b[kMaxCluster];
   uint32_t x_tot[kMaxCluster];
+  float x_m[kMaxCluster], x_s[kMaxCluster];   // per-rank (max, sum e^{z - max}) of a row
   uint32_t warp_tot[2 * kSaWarps];
   uint32_t n_sure, n_list;
   int t_bin;
@@ -262,9 +263,8 @@ __device__ int cluster_thresh(SaSmem<D> &sm, cg::cluster_group &cl, int rank, in
 template <int D, class Src>
 __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
                               int ncl, const Src &src, uint32_t b1, uint32_t want, uint32_t base,
-                              int32_t *irow) {
+                              int32_t *irow, uint32_t k_eff) {
   const int tid = threadIdx.x;
-  const uint32_t k_eff = static_cast<uint32_t>(p.k_eff);
   unsigned long long prefix = b1;
   int sh = 64 - kHistBits;   // composite bits below digit 1
   bool have_hist = true;
@@ -444,6 +444,56 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
   }
 }
 
+// ln sum_{j < N} e^{z_j} of one score row (the log of Eq. (1)'s softmax normaliser), cluster-
+// wide: each CTA folds its candidates [lo, hi) and its share of W into a running (max, sum),
+// the CTAs exchange theirs through distributed shared memory and all merge them.
+template <int D>
+__device__ float row_logsumexp(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
+                               int ncl, const float *srow, long long lo, long long hi) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float m = -INFINITY, s = 0.f;
+  auto add = [&](float z) {
+    if (z > m) {
+      s = s * expf(m - z) + 1.f;   // expf(-inf) = 0 for the first element
+      m = z;
+    } else {
+      s += expf(z - m);
+    }
+  };
+  for (long long i = lo + tid; i < hi; i += kSaThreads) add(__ldcg(srow + i));
+  const long long wper = (p.nW + ncl - 1) / ncl;
+  const long long w_hi = min(p.nW, (rank + 1) * wper);
+  for (long long e = rank * wper + tid; e < w_hi; e += kSaThreads)
+    add(__ldcg(srow + (e < p.s1 ? e : p.w0 + (e - p.s1))));
+  // merge (m, s) over the warp, then over the CTA's warps
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o), so = __shfl_xor_sync(0xffffffffu, s, o);
+    const float mn = fmaxf(m, mo);
+    s = (m == -INFINITY ? 0.f : s * expf(m - mn)) + (mo == -INFINITY ? 0.f : so * expf(mo - mn));
+    m = mn;
+  }
+  if (lane == 0) {
+    sm.wm[warp] = m;
+    sm.wz[warp] = s;
+  }
+  __syncthreads();
+  if (tid < ncl) {
+    float M = -INFINITY, Z = 0.f;
+    for (int w = 0; w < kSaWarps; ++w) M = fmaxf(M, sm.wm[w]);
+    for (int w = 0; w < kSaWarps; ++w)
+      if (sm.wm[w] != -INFINITY) Z += sm.wz[w] * expf(sm.wm[w] - M);
+    cl.map_shared_rank(sm.x_m, tid)[rank] = M;
+    cl.map_shared_rank(sm.x_s, tid)[rank] = Z;
+  }
+  cl.sync();   // every CTA's (max, sum) is in every CTA
+  float M = -INFINITY, Z = 0.f;
+  for (int c = 0; c < ncl; ++c) M = fmaxf(M, sm.x_m[c]);
+  for (int c = 0; c < ncl; ++c)
+    if (sm.x_m[c] != -INFINITY) Z += sm.x_s[c] * expf(sm.x_m[c] - M);
+  return M + logf(Z);
+}
+
 // Omega of one query head into irow (cluster-wide; every CTA takes the same branches).
 template <int D>
 __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
@@ -455,24 +505,56 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   if (p.k_eff == 0) return;
   const long long a0 = p.cbase + static_cast<long long>(rank) * p.cper;
   const long long lo = max(a0, p.s1), hi = min(a0 + p.cper, p.w0);
-  if (p.k_eff >= p.nC) {   // every candidate is selected
-    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - p.s1] = static_cast<int32_t>(i);
-    return;
-  }
-  const uint32_t k_eff = static_cast<uint32_t>(p.k_eff);
   const float *srow = p.S + static_cast<long long>(row) * p.ldS;
   uint32_t *h1 = p.hist + static_cast<long long>(row) * kHistBins;
+  const ChunkSrc chunk{srow, a0, lo, hi};
+  long long k_sel = p.k_eff;   // keys to select (the budget; fewer under a threshold)
   for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
   if (tid == 0) {
     sm.n_sure = 0u;
     sm.n_list = 0u;
   }
-  const bool build = (p.mode & kSaBuildHist) != 0;
-  int b1i;
-  if (build) {
+  const bool build = (p.mode & (kSaBuildHist | kSaEps)) != 0;
+  int b1i = -1;
+  if (p.mode & kSaEps) {
+    // Eq. (2)'s threshold: a_i > eps  <=>  z_i > T = ln(eps) + ln sum_j e^{z_j} (all N)
+    const float T = p.log_eps + row_logsumexp(p, sm, cl, rank, ncl, srow, lo, hi);
+    // this CTA's digit-1 histogram of its candidates and its count of z > T
+    uint32_t cnt = 0;
+    chunk.for_each([&](unsigned long long x) {
+      atomicAdd(&sm.h[static_cast<uint32_t>(x >> (64 - kHistBits))], 1u);
+      cnt += key_float(static_cast<uint32_t>(x >> 32)) > T ? 1u : 0u;
+    });
+    uint32_t tot, unused;
+    block_scan2(cnt, 0u, sm.warp_tot, tot, unused);
+    if (tid < ncl) cl.map_shared_rank(sm.x_b, tid)[rank] = tot;
+    __syncthreads();
+    cl.sync();   // histograms and counts complete
+    long long above_t = 0;
+    for (int c = 0; c < ncl; ++c) above_t += sm.x_b[c];
+    k_sel = min(k_sel, above_t);
+    if (rank == 0)
+      for (long long i = k_sel + tid; i < p.k_eff; i += kSaThreads) irow[i] = -1;
+    if (k_sel == 0) return;
+    if (k_sel < p.nC) {
+      b1i = cluster_thresh(sm, cl, rank, ncl, kHistBins, static_cast<uint32_t>(k_sel));
+      b1i = sm.t_bin < 0 ? -1 : b1i + sm.t_bin;
+    }
+    cl.sync();   // every CTA has read the slices it needed: the histograms can be cleared
+    for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
+    __syncthreads();
+  }
+  if (k_sel >= p.nC) {   // every candidate is selected
+    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - p.s1] = static_cast<int32_t>(i);
+    return;
+  }
+  const uint32_t k_eff = static_cast<uint32_t>(k_sel);
+  if (p.mode & kSaEps) {
+    // b1 found above
+  } else if (build) {
     // digit 1 from the scores themselves: this CTA's histogram, then the cluster's threshold
     __syncthreads();
-    ChunkSrc{srow, a0, lo, hi}.for_each([&](unsigned long long x) {
+    chunk.for_each([&](unsigned long long x) {
       atomicAdd(&sm.h[static_cast<uint32_t>(x >> (64 - kHistBits))], 1u);
     });
     __syncthreads();
@@ -502,7 +584,6 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
     for (int i = tid; i < kHistBins; i += kSaThreads) h1[i] = 0u;   // left zero for the next call
   uint32_t off = 0;
   for (int c = 0; c < rank; ++c) off += sm.x_a[c];
-  const ChunkSrc chunk{srow, a0, lo, hi};
   // the keys above b1 take idx slots [0, above1), CTA by CTA
   if (sm.n_sure <= static_cast<uint32_t>(kSureCap)) {
     for (uint32_t i = tid; i < sm.n_sure; i += kSaThreads)
@@ -522,7 +603,7 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   }
   // the keys of b1, from the CTAs' lists
   select_rounds(p, sm, cl, rank, ncl, ListSrc<D>{&sm, spill, sm.n_list}, b1, k_eff - above1,
-                above1, irow);
+                above1, irow, k_eff);
 }
 
 // Softmax attention of one query head over U = W u Omega (Omega read from idx), split across

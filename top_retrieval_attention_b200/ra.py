@@ -22,7 +22,7 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
            "ra_sparse_attn", "ra_select_attend", "ra_dense_workspace_bytes", "ra_dense_decode",
            "ra_decode_step_static", "ra_prefill_workspace_bytes", "ra_prefill_topk",
-           "ra_prefill_score", "ra_prefill_select")
+           "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets")
 
 
 class ra_kv(ctypes.Structure):
@@ -61,6 +61,11 @@ def lib() -> ctypes.CDLL:
             "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
             "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                                           c_void_p]),
+            "ra_pyramid_budgets": (c_int32, [c_int32, c_int32, ctypes.c_double,
+                                             ctypes.POINTER(c_int32)]),
+            "ra_decode_step_eps": (c_int32, [P, c_void_p, c_int32, c_int32, ctypes.c_float, c_int32,
+                                             c_int32, c_void_p, c_void_p, c_void_p, c_size_t,
+                                             c_void_p]),
             "ra_prefill_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int32, c_int64, c_int32,
                                                       c_int32, c_int32, c_int32]),
             "ra_prefill_topk": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32, c_int32,
@@ -254,6 +259,37 @@ def prefill_topk(cache: KVCache, q, k: int, n_sink: int, n_window: int, idx=None
     check(ra_prefill_topk(cache.kv, q.data_ptr(), Hq, M, k, n_sink, n_window, idx.data_ptr(),
                           ws.data_ptr(), ws.numel(), _stream(stream)), "ra_prefill_topk")
     return idx[..., :k]
+
+
+def pyramid_budgets(L: int, k_mean: int, ratio: float) -> list[int]:
+    """Per-layer budgets (ra_pyramid_budgets): a linear fall from layer 0 to layer L - 1 with
+    mean k_mean, summing to exactly L * k_mean."""
+    out = (c_int32 * L)()
+    check(lib().ra_pyramid_budgets(L, k_mean, ratio, out), "ra_pyramid_budgets")
+    return list(out)
+
+
+def ra_decode_step_eps(kv, q, Hq, k, eps, n_sink, n_window, out, idx, ws, ws_bytes, stream):
+    return lib().ra_decode_step_eps(ctypes.byref(kv), q, Hq, k, eps, n_sink, n_window, out, idx,
+                                    ws, ws_bytes, stream)
+
+
+def decode_step_eps(cache: KVCache, q, k: int, eps: float, n_sink: int, n_window: int, out=None,
+                    idx=None, ws=None, stream=None):
+    """Decode step keeping the candidates whose full softmax weight exceeds eps (at most k).
+    Returns (out fp32, idx int32 with -1 past the kept keys)."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = decode_workspace(cache, Hq, k, n_sink, n_window)
+    check(ra_decode_step_eps(cache.kv, q.data_ptr(), Hq, k, eps, n_sink, n_window, out.data_ptr(),
+                             idx.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+          "ra_decode_step_eps")
+    return out, idx[..., :k]
 
 
 def dense_workspace(cache: KVCache, Hq: int):
