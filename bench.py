@@ -65,6 +65,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--eps", type=float, default=0.0,
+                    help="threshold budget: keep candidates whose softmax weight exceeds eps "
+                         "(at most k per head; ra_decode_step_eps)")
+    ap.add_argument("--pyramid", type=float, default=0.0,
+                    help="per-layer budgets falling linearly with depth to this ratio of the "
+                         "first layer's, mean k (ra_pyramid_budgets)")
     ap.add_argument("--prefill-queries", type=int, default=0,
                     help="instead of decode steps: exact top-k of this many prefill queries per "
                          "query head (tensor-core scores + cluster selection), one layer")
@@ -292,24 +298,35 @@ def run_ours(args, w, rank, local_rank, world, dist):
     for s in range(P):
         for layer in range(L):
             sdev.fill_q(qpool[s, layer], w.seed + 7919 * s + 104729 * layer)
-    ws_bytes = ra.ra_decode_workspace_bytes(B, Hq, N, d, k, w.n_sink, w.n_window)
+    ks = ra.pyramid_budgets(L, k, args.pyramid) if args.pyramid > 0 else [k] * L
+    ws_bytes = ra.ra_decode_workspace_bytes(B, Hq, N, d, max(ks), w.n_sink, w.n_window)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     outs = [torch.empty((B, Hq, d), dtype=torch.float32, device=dev) for _ in range(L)]
-    idxs = [torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=dev) for _ in range(L)]
+    idxs = [torch.empty((B, Hq, max(kl, 1)), dtype=torch.int32, device=dev) for kl in ks]
     torch.cuda.synchronize()
 
     def phases(layer, qptr, ev=None):
         c = caches[layer]
         kv = c.kv
+        kl = ks[layer]
         if ev is not None:
             ev[0].record(stream)
         ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
         if ev is not None:
             ev[1].record(stream)
-        ra.check(ra.ra_score_gqa(kv, qptr, Hq, k, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
+        if args.eps > 0:   # the threshold step as one call (score, then select + attend)
+            ra.check(ra.ra_decode_step_eps(kv, qptr, Hq, kl, args.eps, w.n_sink, w.n_window,
+                                           outs[layer].data_ptr(), idxs[layer].data_ptr(),
+                                           ws.data_ptr(), ws_bytes, sp), "decode_step_eps")
+            if ev is not None:
+                ev[2].record(stream)
+                ev[3].record(stream)
+            c.N = N - 1
+            return
+        ra.check(ra.ra_score_gqa(kv, qptr, Hq, kl, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
         if ev is not None:
             ev[2].record(stream)
-        ra.check(ra.ra_select_attend(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+        ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window, idxs[layer].data_ptr(),
                                      outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "select_attend")
         if ev is not None:
             ev[3].record(stream)
@@ -324,12 +341,21 @@ def run_ours(args, w, rank, local_rank, world, dist):
         for layer in range(L):
             c = caches[layer]
             kv = c.kv
+            kl = ks[layer]
             qptr = qpool[s % P, layer].data_ptr()
             ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
+            if args.eps > 0:   # the score kernel runs inside the one call: time the whole call
+                ev[layer][0].record(stream)
+                ra.check(ra.ra_decode_step_eps(kv, qptr, Hq, kl, args.eps, w.n_sink, w.n_window,
+                                               outs[layer].data_ptr(), idxs[layer].data_ptr(),
+                                               ws.data_ptr(), ws_bytes, sp), "decode_step_eps")
+                ev[layer][1].record(stream)
+                c.N = N - 1
+                continue
             ev[layer][0].record(stream)
-            ra.check(ra.ra_score_gqa(kv, qptr, Hq, k, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
+            ra.check(ra.ra_score_gqa(kv, qptr, Hq, kl, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
             ev[layer][1].record(stream)
-            ra.check(ra.ra_select_attend(kv, Hq, k, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+            ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window, idxs[layer].data_ptr(),
                                          outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "select_attend")
             c.N = N - 1
 
@@ -397,16 +423,23 @@ def run_ours(args, w, rank, local_rank, world, dist):
     s1 = min(w.n_sink, N)
     w0 = max(s1, N - w.n_window)
     n_w = s1 + (N - w0)
-    k_eff = min(k, w0 - s1)
     k_bytes = B * Hkv * N * 2 * d
-    v_bytes = B * Hq * (n_w + k_eff) * 2 * d
+    if args.eps > 0:   # the keys the threshold kept (the last step's idx; every step alike)
+        kept = [int((t >= 0).sum().item()) for t in idxs]
+        v_bytes_all = sum(B * Hq * n_w * 2 * d + kl * 2 * d for kl in kept)
+    else:
+        kept = None
+        v_bytes_all = sum(B * Hq * (n_w + min(kl, w0 - s1)) * 2 * d for kl in ks)
     peak, peak_kind = measured_hbm_peak()
     score_s = statistics.mean(score_ms) / 1e3
     kscan_gbs = k_bytes / score_s / 1e9
-    step_gbs = L * (k_bytes + v_bytes) / (ms_per_step / 1000.0) / 1e9
+    step_gbs = (L * k_bytes + v_bytes_all) / (ms_per_step / 1000.0) / 1e9
     src_hash = score_source_hash()
     traffic = TRAFFIC.get((src_hash, w.name))
-    roofline = {"kernel": "score_gqa_kernel (K scan)", "bound": "hbm", "achieved": kscan_gbs,
+    if args.eps > 0:   # the score kernel is inside the one timed call: the roofline is the call's
+        kscan_gbs = (k_bytes + v_bytes_all / L) / score_s / 1e9
+    roofline = {"kernel": ("decode_step_eps (score + select + attend)" if args.eps > 0
+                           else "score_gqa_kernel (K scan)"), "bound": "hbm", "achieved": kscan_gbs,
                 "peak": peak, "unit": "GB/s", "frac": kscan_gbs / peak,
                 "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
                 "algorithmic_bytes_per_launch": k_bytes,
@@ -418,7 +451,8 @@ def run_ours(args, w, rank, local_rank, world, dist):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 / Irwin-Hall normals, Llama-3-8B-shaped caches)",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), **({"eps": args.eps} if args.eps > 0 else {}),
+                       **({"pyramid_ratio": args.pyramid, "k_per_layer": ks} if args.pyramid > 0 else {})),
         "roofline": roofline,
         "kscan_hbm_gbs": kscan_gbs,
         "step_algorithmic_gbs": step_gbs,
@@ -429,6 +463,9 @@ def run_ours(args, w, rank, local_rank, world, dist):
         "gpu_launches": launches_per_layer * L * steps,
         "clocks": clocks,
     }
+    if kept is not None:
+        result["kept_keys_per_head_mean"] = sum(kept) / (L * B * Hq)
+        result["roofline"]["traffic"] = None
 
     # dense flash-decode on the same cache (decode part only is compared)
     if not args.no_dense:
@@ -469,7 +506,7 @@ def run_ours(args, w, rank, local_rank, world, dist):
         dk = [torch.empty_like(t) for t in knew]
         dv = [torch.empty_like(t) for t in vnew]
         ho = torch.empty((L, B, Hq, d), dtype=torch.float32).pin_memory()
-        hi = torch.empty((L, B, Hq, max(k, 1)), dtype=torch.int32).pin_memory()
+        hi = [torch.empty((B, Hq, max(kl, 1)), dtype=torch.int32).pin_memory() for kl in ks]
 
         def e2e_step(s):
             dq.copy_(hq[s % P], non_blocking=True)
@@ -477,8 +514,12 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 dk[layer].copy_(hk[layer], non_blocking=True)
                 dv[layer].copy_(hv[layer], non_blocking=True)
                 ra.append_kv(caches[layer], dk[layer], dv[layer])
-                ra.decode_step(caches[layer], dq[layer], k, w.n_sink, w.n_window,
-                               out=outs[layer], idx=idxs[layer], ws=ws)
+                if args.eps > 0:
+                    ra.decode_step_eps(caches[layer], dq[layer], ks[layer], args.eps, w.n_sink,
+                                       w.n_window, out=outs[layer], idx=idxs[layer], ws=ws)
+                else:
+                    ra.decode_step(caches[layer], dq[layer], ks[layer], w.n_sink, w.n_window,
+                                   out=outs[layer], idx=idxs[layer], ws=ws)
                 caches[layer].N = N - 1
                 ho[layer].copy_(outs[layer], non_blocking=True)
                 hi[layer].copy_(idxs[layer], non_blocking=True)
@@ -495,7 +536,7 @@ def run_ours(args, w, rank, local_rank, world, dist):
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(dist, a.elapsed_time(b) / esteps, dev)
         h2d = L * (B * Hq * d * 2 + 2 * B * Hkv * d * 2)
-        d2h = L * (B * Hq * d * 4 + B * Hq * max(k, 1) * 4)
+        d2h = sum(B * Hq * d * 4 + B * Hq * max(kl, 1) * 4 for kl in ks)
         result["e2e"] = {"value": world * 1000.0 / e2e_ms, "unit": "steps/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": esteps,
                          "ms_per_step": e2e_ms,
