@@ -70,6 +70,26 @@ typedef struct {
   int64_t N;
 } ra_kv;
 
+/*
+ * A per-layer KV cache in pages (the serving layout: sequences of different lengths share one
+ * pool of fixed-size pages, a block table maps each sequence's token i to its page).
+ *   K, V        : bf16 page pools [num_pages, Hkv, 128, d], device, caller-owned.  Token i of
+ *                 sequence b, KV head g, is row i % 128 of page block_table[b * max_pages +
+ *                 i / 128] (pool row (page * Hkv + g) * 128 + i % 128).
+ *   block_table : int32 [B, max_pages], device, caller-owned; entries for the pages a
+ *                 sequence uses must be valid page indices (< num_pages).
+ *   seq_len     : int32 [B], HOST, caller-owned: tokens cached per sequence (>= 1 for a decode
+ *                 step, <= max_pages * 128); ra_paged_append_kv advances it.
+ *   B <= 256, d 64 or 128.
+ */
+typedef struct {
+  void *K;
+  void *V;
+  const int32_t *block_table;
+  int32_t *seq_len;
+  int32_t B, Hkv, d, max_pages, num_pages;
+} ra_paged_kv;
+
 /* Human-readable name of a status (static string). */
 const char *ra_status_str(ra_status s);
 
@@ -145,6 +165,25 @@ ra_status ra_decode_step_eps(const ra_kv *kv, const void *q, int32_t Hq, int32_t
  * Errors: RA_ERR_ARG.
  */
 ra_status ra_pyramid_budgets(int32_t L, int32_t k_mean, double ratio, int32_t *k_out);
+
+/*
+ * The decode step on a paged cache (ragged sequence lengths): per sequence b, exactly
+ * ra_decode_step over its seq_len[b] tokens (its own W, C and min(k, |C|)).
+ *   ra_paged_append_kv : token seq_len[b] + t of every sequence from k_new / v_new [B, Hkv, T, d]
+ *                        (bf16, device), then seq_len[b] += T on the host.  The pages must
+ *                        already be in the block table.  RA_ERR_CAPACITY past max_pages * 128.
+ *   ra_paged_workspace_bytes : the workspace of the longest sequence (max_N = max seq_len).
+ *   ra_paged_decode_step : q [B, Hq, d], out [B, Hq, d] fp32, idx [B, Hq, k] (-1 past each
+ *                        sequence's min(k, |C|)), ws as in ra_decode_step (zero-filled once).
+ * Errors: as ra_decode_step; RA_ERR_SHAPE for B > 256 or a length outside [1, max_pages * 128].
+ */
+ra_status ra_paged_append_kv(ra_paged_kv *kv, const void *k_new, const void *v_new, int32_t T,
+                             ra_stream_t stream);
+size_t ra_paged_workspace_bytes(int32_t B, int32_t Hq, int64_t max_N, int32_t d, int32_t k,
+                                int32_t n_sink, int32_t n_window);
+ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq, int32_t k,
+                               int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
+                               void *ws, size_t ws_bytes, ra_stream_t stream);
 
 /*
  * The phases of ra_decode_step, exposed so a caller can time or interleave them.  All take the

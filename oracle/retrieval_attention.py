@@ -275,3 +275,18 @@ def pyramid_budgets(L: int, k_mean: int, ratio: float) -> np.ndarray:
     rem = L * k_mean - int(base.sum())
     base[:rem] += 1
     return base
+
+
+# ------------------------------------------------------------------------------------
+# paged caches (the serving layout): token i of sequence b, KV head g, is row i % P of page
+# table[b][i // P] of the pool [num_pages, Hkv, P, d]
+
+
+def gather_paged(pool: np.ndarray, table: np.ndarray, lens) -> list:
+    """The dense [Hkv, N_b, d] cache of every sequence b, read out of a paged pool."""
+    P = pool.shape[2]
+    out = []
+    for b, n in enumerate(lens):
+        rows = [pool[table[b][i // P], :, i % P, :] for i in range(int(n))]
+        out.append(np.stack(rows, axis=1) if rows else pool[:0, :, 0, :].transpose(1, 0, 2))
+    return out

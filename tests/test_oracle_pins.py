@@ -492,3 +492,33 @@ def test_pyramid_budgets_shape():
         if L > 1:
             assert abs(b[0] - k_max) <= 1 and abs(b[-1] - r * k_max) <= 1
     assert list(oracle.pyramid_budgets(6, 11, 1.0)) == [11] * 6
+
+
+# ---------------------------------------------------------------- paged layout
+
+
+def test_gather_paged_inverts_a_scatter_by_the_definition():
+    """Scatter dense caches of ragged lengths into a shuffled page pool following the layout
+    (token i of sequence b in row i % 128 of page table[b][i // 128]); the gather must return
+    them exactly, for every sequence and KV head."""
+    rng = np.random.default_rng(9)
+    B, Hkv, d, P = 3, 2, 8, 128
+    lens = [1, 300, 129]
+    pages_needed = [(n + P - 1) // P for n in lens]
+    num_pages = sum(pages_needed) + 2
+    order = rng.permutation(num_pages)
+    table = np.full((B, 4), -1, dtype=np.int64)
+    pool = rng.integers(0, 2**16, size=(num_pages, Hkv, P, d)).astype(np.uint16)
+    dense = []
+    j = 0
+    for b, n in enumerate(lens):
+        X = rng.integers(0, 2**16, size=(Hkv, n, d)).astype(np.uint16)
+        dense.append(X)
+        for pg in range(pages_needed[b]):
+            table[b, pg] = order[j]
+            j += 1
+        for i in range(n):
+            pool[table[b, i // P], :, i % P, :] = X[:, i, :]
+    got = oracle.gather_paged(pool, table, lens)
+    for b in range(B):
+        assert np.array_equal(got[b], dense[b])

@@ -7,5 +7,6 @@ from .ra import (  # noqa: F401
     ra_decode_step_static, ra_dense_decode, ra_dense_workspace_bytes, ra_kv, ra_last_error, ra_score_gqa,
     ra_select_attend, ra_sparse_attn, ra_status_str, ra_topk_select, ra_version,
     ra_prefill_workspace_bytes, ra_prefill_topk, ra_prefill_score, ra_prefill_select, prefill_topk,
-    ra_decode_step_eps, decode_step_eps, pyramid_budgets,
+    ra_decode_step_eps, decode_step_eps, pyramid_budgets, ra_paged_kv, PagedKVCache,
+    paged_append_kv, paged_workspace, paged_decode_step,
 )

@@ -45,6 +45,19 @@ struct ScoreParams {
   uint32_t *err;            // error word (bit kErrScoreWait: a load never landed)
 };
 
+// Paged KV caches: K and V in pages of kPageSize tokens, [num_pages, Hkv, kPageSize, d]; sequence
+// b's token i lives in page block_table[b * max_pages + i / kPageSize].  The lengths travel in
+// the kernels' parameter blocks (at most kMaxPagedBatch sequences per call).
+constexpr int kPageSize = 128;
+constexpr int kMaxPagedBatch = 256;
+struct PagedInfo {
+  const int32_t *block_table;               // [B, max_pages], device
+  int max_pages, n_sink, n_window, k;
+  int32_t seq_len[kMaxPagedBatch];          // tokens of sequence b
+  int32_t tile_off[kMaxPagedBatch + 1];     // score tiles before sequence b (all its KV heads)
+};
+struct NoPaging {};   // the dense [B, Hkv, cap, d] layout
+
 // Top-k selection and sparse attention of one decode step, one thread-block cluster per query
 // head (row = b * Hq + h).  mode: kSaSelect writes idx from the scores; kSaAttend computes out
 // from the scores, idx and V; both in one launch for the decode step.
@@ -121,6 +134,8 @@ size_t counter_block_bytes(size_t rows);
 cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]);
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s);
+cudaError_t launch_score_paged(const ScoreParams &p, const PagedInfo &pg, long long num_pages, int d,
+                               cudaStream_t s);
 // Cluster size for one query head: a power of two <= kMaxCluster (16 only where the device
 // schedules 16-CTA clusters of this kernel), chunks of at most 64K scores, grown to fill the GPU.
 int select_cluster_size(long long nC, int R, int d);
@@ -128,8 +143,11 @@ int select_cluster_size(long long nC, int R, int d);
 // cluster takes at most 1024 entries, else up to kMaxAttnSplit while all clusters run in one wave.
 int attn_split(long long nU, int R, int ncl, int d);
 cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s);
+cudaError_t launch_select_attend_paged(const SaParams &p, const PagedInfo &pg, int d, int R, int ncl,
+                                       cudaStream_t s);
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
 cudaError_t launch_prefill_score(const PfParams &p, int d, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
+cudaError_t launch_append_paged(const AppendParams &p, const PagedInfo &pg, cudaStream_t s);
 
 }  // namespace ra

@@ -316,6 +316,39 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
   return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws, cs);
 }
 
+// ---- paged caches
+
+static ra_status check_paged(const ra_paged_kv *kv, long long *max_n) {
+  if (!kv || !kv->K || !kv->V || !kv->block_table || !kv->seq_len) return RA_ERR_ARG;
+  if (!aligned16(kv->K) || !aligned16(kv->V)) return RA_ERR_ARG;
+  if (kv->B < 1 || kv->Hkv < 1 || kv->max_pages < 1 || kv->num_pages < 1) return RA_ERR_ARG;
+  if (kv->B > kMaxPagedBatch) return RA_ERR_SHAPE;
+  if (kv->d != 64 && kv->d != 128) return RA_ERR_SHAPE;
+  long long m = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    if (kv->seq_len[b] < 0 || static_cast<long long>(kv->seq_len[b]) > 1LL * kv->max_pages * kPageSize)
+      return RA_ERR_SHAPE;
+    m = std::max<long long>(m, kv->seq_len[b]);
+  }
+  *max_n = m;
+  return RA_OK;
+}
+
+static void fill_paged_info(const ra_paged_kv *kv, int k, int n_sink, int n_window, PagedInfo &pg) {
+  pg.block_table = kv->block_table;
+  pg.max_pages = kv->max_pages;
+  pg.n_sink = n_sink;
+  pg.n_window = n_window;
+  pg.k = k;
+  int32_t off = 0;
+  for (int b = 0; b < kv->B; ++b) {
+    pg.seq_len[b] = kv->seq_len[b];
+    pg.tile_off[b] = off;
+    off += kv->Hkv * ((kv->seq_len[b] + kScoreTile - 1) / kScoreTile);
+  }
+  pg.tile_off[kv->B] = off;
+}
+
 // ---- prefill: exact top-k of a batch of queries (rows (b, h, m) of Q [B, Hq, M, d])
 
 // The prefill plan is the decode plan with one row per query: B * M "sequences" of Hq heads.
@@ -501,6 +534,104 @@ ra_status ra_pyramid_budgets(int32_t L, int32_t k_mean, double ratio, int32_t *k
   // the rounding remainder goes one by one to the lowest layers: the total is L * k_mean
   const long long rem = static_cast<long long>(L) * k_mean - total;
   for (long long l = 0; l < rem && l < L; ++l) k_out[l] += 1;
+  return RA_OK;
+}
+
+ra_status ra_paged_append_kv(ra_paged_kv *kv, const void *k_new, const void *v_new, int32_t T,
+                             ra_stream_t stream) {
+  long long max_n = 0;
+  ra_status s = check_paged(kv, &max_n);
+  if (s != RA_OK) return s;
+  if (T < 0) return RA_ERR_ARG;
+  if (T == 0) return RA_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return RA_ERR_ARG;
+  for (int b = 0; b < kv->B; ++b)
+    if (static_cast<long long>(kv->seq_len[b]) + T > 1LL * kv->max_pages * kPageSize)
+      return RA_ERR_CAPACITY;
+  AppendParams p{};
+  p.K = static_cast<__nv_bfloat16 *>(kv->K);
+  p.V = static_cast<__nv_bfloat16 *>(kv->V);
+  p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+  p.B = kv->B; p.Hkv = kv->Hkv; p.d = kv->d; p.T = T;
+  PagedInfo pg{};
+  fill_paged_info(kv, 0, 0, 0, pg);
+  const cudaError_t e = launch_append_paged(p, pg, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "paged_append");
+  for (int b = 0; b < kv->B; ++b) kv->seq_len[b] += T;
+  return RA_OK;
+}
+
+size_t ra_paged_workspace_bytes(int32_t B, int32_t Hq, int64_t max_N, int32_t d, int32_t k,
+                                int32_t n_sink, int32_t n_window) {
+  if (B > kMaxPagedBatch) return 0;
+  return ra_decode_workspace_bytes(B, Hq, max_N, d, k, n_sink, n_window);
+}
+
+ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq, int32_t k,
+                               int32_t n_sink, int32_t n_window, float *out, int32_t *idx,
+                               void *ws, size_t ws_bytes, ra_stream_t stream) {
+  long long max_n = 0;
+  ra_status s = check_paged(kv, &max_n);
+  if (s != RA_OK) return s;
+  for (int b = 0; b < kv->B; ++b)
+    if (kv->seq_len[b] < 1) return RA_ERR_EMPTY;
+  // the plan of the longest sequence bounds every row's (scores, lists, cluster split)
+  Step st{};
+  s = plan_shape(kv->B, Hq, kv->Hkv, max_n, kv->d, k, n_sink, n_window, st);
+  if (s != RA_OK) return s;
+  for (int b = 0; b < kv->B; ++b) {   // every row's union must be non-empty
+    const long long N = kv->seq_len[b];
+    const long long s1 = std::min<long long>(n_sink, N), w0 = std::max<long long>(s1, N - n_window);
+    if (s1 + (N - w0) + std::min<long long>(k, w0 - s1) == 0) return RA_ERR_EMPTY;
+  }
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < st.total)
+    return RA_ERR_WORKSPACE;
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  plan_clusters(st);
+  st.cap = 0;
+  PagedInfo pg{};
+  fill_paged_info(kv, k, n_sink, n_window, pg);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  {
+    ScoreParams p{};
+    p.K = static_cast<const __nv_bfloat16 *>(kv->K);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.S = reinterpret_cast<float *>(at(ws, st.off_S));
+    p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
+    p.N = st.N; p.cap = 0; p.ldS = st.ldS;
+    p.total_tiles = pg.tile_off[kv->B];
+    p.B = st.B; p.Hkv = st.Hkv; p.G = st.G; p.Hq = st.Hq;
+    p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
+    p.do_hist = k > 0;   // each head decides from its own length
+    p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+    const cudaError_t e = launch_score_paged(p, pg, kv->num_pages, st.d, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "paged_score");
+  }
+  SaParams p{};
+  p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
+  p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
+  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
+  p.V = static_cast<const __nv_bfloat16 *>(kv->V);
+  p.idx = idx;
+  p.out = out;
+  p.part = reinterpret_cast<float *>(at(ws, st.off_part));
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
+  p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+  p.ldS = st.ldS; p.ldL = st.ldL; p.cap = 0; p.N = st.N;
+  p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
+  const int split = attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d);
+  p.mode = split == 1 ? (kSaSelect | kSaAttend) : kSaSelect;
+  p.nsplit = 1;
+  cudaError_t e = launch_select_attend_paged(p, pg, st.d, st.R, st.ncl, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "paged_select_attend");
+  if (split > 1) {
+    p.mode = kSaAttend;
+    p.nsplit = split;
+    e = launch_select_attend_paged(p, pg, st.d, st.R, st.ncl, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "paged_attend");
+  }
   return RA_OK;
 }
 

@@ -35,9 +35,62 @@ struct ScoreCfg {
   }
 };
 
-template <int D>
+// ---- cache geometry: the dense [B, Hkv, cap, d] layout or 128-token pages (one tile each)
+
+// Tokens of the (b, g) head bg.
+__device__ __forceinline__ long long seq_n(const ScoreParams &p, const NoPaging &, long long) {
+  return p.N;
+}
+__device__ __forceinline__ long long seq_n(const ScoreParams &p, const PagedInfo &pg, long long bg) {
+  return pg.seq_len[bg / p.Hkv];
+}
+// The head and first key of flattened tile t (tiles ordered by head, then key).
+__device__ __forceinline__ void tile_start(const ScoreParams &p, const NoPaging &, long long t,
+                                           long long &bg, long long &key) {
+  bg = t / p.tiles_per_head;
+  key = (t - bg * p.tiles_per_head) * kScoreTile;
+}
+__device__ __forceinline__ void tile_start(const ScoreParams &p, const PagedInfo &pg, long long t,
+                                           long long &bg, long long &key) {
+  int b = 0;
+  while (b + 1 < p.B && pg.tile_off[b + 1] <= t) ++b;   // once per CTA
+  const long long per_head = (pg.seq_len[b] + kScoreTile - 1) / kScoreTile;
+  const long long r = t - pg.tile_off[b];
+  bg = static_cast<long long>(b) * p.Hkv + r / per_head;
+  key = (r % per_head) * kScoreTile;
+}
+// TMA coordinates (rows, plane) of the tile at (bg, key).
+__device__ __forceinline__ void tile_coords(const ScoreParams &, const NoPaging &, long long bg,
+                                            long long key, int &y, int &z) {
+  y = static_cast<int>(key);
+  z = static_cast<int>(bg);
+}
+__device__ __forceinline__ void tile_coords(const ScoreParams &p, const PagedInfo &pg, long long bg,
+                                            long long key, int &y, int &z) {
+  const long long b = bg / p.Hkv, g = bg - b * p.Hkv;
+  const int page = __ldg(pg.block_table + b * pg.max_pages + key / kPageSize);
+  y = static_cast<int>(key % kPageSize);
+  z = static_cast<int>(static_cast<long long>(page) * p.Hkv + g);
+}
+// The candidate range of head bg and whether its histogram is wanted.
+__device__ __forceinline__ void cand_range(const ScoreParams &p, const NoPaging &, long long,
+                                           long long &lo, long long &hi, bool &hist) {
+  lo = p.cand_lo;
+  hi = p.cand_hi;
+  hist = p.do_hist != 0;
+}
+__device__ __forceinline__ void cand_range(const ScoreParams &p, const PagedInfo &pg, long long bg,
+                                           long long &lo, long long &hi, bool &hist) {
+  const long long N = pg.seq_len[bg / p.Hkv];
+  lo = min(static_cast<long long>(pg.n_sink), N);
+  hi = max(lo, N - pg.n_window);
+  const long long k_eff = min(static_cast<long long>(pg.k), hi - lo);
+  hist = p.do_hist != 0 && k_eff > 0 && k_eff < hi - lo;
+}
+
+template <int D, class Pg>
 __global__ void __launch_bounds__(256, 1)
-    score_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const ScoreParams p) {
+    score_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const ScoreParams p, const Pg pg) {
   using C = ScoreCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -67,19 +120,21 @@ __global__ void __launch_bounds__(256, 1)
   pdl_wait();   // K (appended rows) and the score / histogram buffers belong to the predecessor
 
   // load cursor (thread 0 only) and compute cursor (all threads)
-  const long long bg0 = t_begin / p.tiles_per_head;
-  long long l_bg = bg0, l_key = (t_begin - bg0 * p.tiles_per_head) * C::kTile;
-  long long c_bg = bg0, c_key = l_key;
+  long long bg0, key0;
+  tile_start(p, pg, t_begin, bg0, key0);
+  long long l_bg = bg0, l_key = key0;
+  long long c_bg = bg0, c_key = key0;
   const uint64_t pol = policy_evict_first();
   auto issue = [&](int slot) {
     const uint32_t bar = bars + 8 * slot;
     mbar_arrive_expect_tx(bar, C::kTileBytes);
+    int ty, tz;
+    tile_coords(p, pg, l_bg, l_key, ty, tz);
 #pragma unroll
     for (int bx = 0; bx < C::kBoxes; ++bx)
-      tma_load_3d(tiles + slot * C::kTileBytes + bx * C::kBoxBytes, &tmK, bx * 64,
-                  static_cast<int>(l_key), static_cast<int>(l_bg), bar, pol);
+      tma_load_3d(tiles + slot * C::kTileBytes + bx * C::kBoxBytes, &tmK, bx * 64, ty, tz, bar, pol);
     l_key += C::kTile;
-    if (l_key >= p.N) {
+    if (l_key >= seq_n(p, pg, l_bg)) {
       l_key = 0;
       ++l_bg;
     }
@@ -102,6 +157,8 @@ __global__ void __launch_bounds__(256, 1)
 
   long long cur_bg = -1;
   long long rowbase = 0;
+  long long cur_lo = 0, cur_hi = 0, cur_n = 0;
+  bool cur_hist = false;
   uint32_t bq[D / 16][2];
   const int mat = lane >> 3;
   const int arow = warp * 16 + (lane & 7) + (mat & 1) * 8;   // ldmatrix source row
@@ -117,11 +174,13 @@ __global__ void __launch_bounds__(256, 1)
     if (tid == 0 && j + C::kStages - 1 < n_local) issue((j + C::kStages - 1) % C::kStages);
 
     if (c_bg != cur_bg) {
-      if (cur_bg >= 0 && p.do_hist) {
+      if (cur_bg >= 0 && cur_hist) {
         flush_hist(cur_bg);
         __syncthreads();
       }
       cur_bg = c_bg;
+      cand_range(p, pg, cur_bg, cur_lo, cur_hi, cur_hist);
+      cur_n = seq_n(p, pg, cur_bg);
       const long long b = c_bg / p.Hkv;
       const long long g = c_bg - b * p.Hkv;
       rowbase = b * p.Hq + g * p.G;
@@ -157,15 +216,15 @@ __global__ void __launch_bounds__(256, 1)
     for (int e = 0; e < 4; ++e) {
       const int h = 2 * t4 + (e & 1);
       const long long key = c_key + warp * 16 + g4 + (e >> 1) * 8;
-      if (h < p.G && key < p.N) {
+      if (h < p.G && key < cur_n) {
         const float z = canon_zero((acc0[e] + acc1[e]) * p.scale);
         p.S[(rowbase + h) * p.ldS + key] = z;
-        if (p.do_hist && key >= p.cand_lo && key < p.cand_hi)
+        if (cur_hist && key >= cur_lo && key < cur_hi)
           atomicAdd(&hist_s[h * kHistBins + (order_key(z) >> (32 - kHistBits))], 1u);
       }
     }
     c_key += C::kTile;
-    if (c_key >= p.N) {
+    if (c_key >= cur_n) {
       c_key = 0;
       ++c_bg;
     }
@@ -181,29 +240,41 @@ __global__ void __launch_bounds__(256, 1)
     return;
   }
   __syncthreads();
-  if (cur_bg >= 0 && p.do_hist) flush_hist(cur_bg);
+  if (cur_bg >= 0 && cur_hist) flush_hist(cur_bg);
 }
 
-template <int D>
-static cudaError_t launch_score_t(const ScoreParams &p, cudaStream_t s) {
+template <int D, class Pg>
+static cudaError_t launch_score_t(const ScoreParams &p, const Pg &pg, long long num_pages,
+                                  cudaStream_t s) {
   using C = ScoreCfg<D>;
   static bool done[64] = {};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D>),
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D, Pg>),
                                     static_cast<int>(C::smem_bytes(kMaxGroup)), done);
   if (e != cudaSuccess) return e;
   CUtensorMap tm;
-  if (!encode_rows_tmap(&tm, p.K, D, static_cast<uint64_t>(p.N),
-                        static_cast<uint64_t>(p.B) * p.Hkv, C::kTile, static_cast<uint64_t>(p.cap)))
+  const bool paged = num_pages > 0;
+  // dense: [B * Hkv planes][N rows (cap apart)][d]; paged: [pages * Hkv planes][128 rows][d]
+  if (!encode_rows_tmap(&tm, p.K, D, paged ? kPageSize : static_cast<uint64_t>(p.N),
+                        paged ? static_cast<uint64_t>(num_pages) * p.Hkv
+                              : static_cast<uint64_t>(p.B) * p.Hkv,
+                        C::kTile, paged ? kPageSize : static_cast<uint64_t>(p.cap)))
     return cudaErrorInvalidValue;
   long long grid = num_sms();
   if (grid > p.total_tiles) grid = p.total_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(score_gqa_kernel<D>, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads),
-                    C::smem_bytes(p.G), s, tm, p);
+  return launch_pdl(score_gqa_kernel<D, Pg>, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads),
+                    C::smem_bytes(p.G), s, tm, p, pg);
 }
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s) {
-  return d == 128 ? launch_score_t<128>(p, s) : launch_score_t<64>(p, s);
+  const NoPaging pg{};
+  return d == 128 ? launch_score_t<128>(p, pg, 0, s) : launch_score_t<64>(p, pg, 0, s);
+}
+
+cudaError_t launch_score_paged(const ScoreParams &p, const PagedInfo &pg, long long num_pages, int d,
+                               cudaStream_t s) {
+  return d == 128 ? launch_score_t<128>(p, pg, num_pages, s)
+                  : launch_score_t<64>(p, pg, num_pages, s);
 }
 
 }  // namespace ra

@@ -444,11 +444,54 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
   }
 }
 
+// The per-row geometry of the step: N, W = [0, s1) u [w0, N), C = [s1, w0), the budget k_eff
+// and the cluster's chunking of C.  Dense caches share one geometry (from the parameters);
+// paged caches derive it from the row's sequence length.
+struct RowGeo {
+  long long N, s1, w0, nW, nC, k_eff, cbase, cper;
+};
+__device__ __forceinline__ RowGeo row_geo(const SaParams &p, const NoPaging &, int, int) {
+  return RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, p.k_eff, p.cbase, p.cper};
+}
+__device__ __forceinline__ RowGeo row_geo(const SaParams &p, const PagedInfo &pg, int row, int ncl) {
+  RowGeo g;
+  g.N = pg.seq_len[row / p.Hq];
+  g.s1 = min(static_cast<long long>(pg.n_sink), g.N);
+  g.w0 = max(g.s1, g.N - pg.n_window);
+  g.nW = g.s1 + (g.N - g.w0);
+  g.nC = g.w0 - g.s1;
+  g.k_eff = min(static_cast<long long>(pg.k), g.nC);
+  g.cbase = g.s1 & ~3LL;
+  const long long span = max(g.w0 - g.cbase, 1LL);
+  g.cper = ((span + ncl - 1) / ncl + 3) / 4 * 4;
+  return g;
+}
+// Where token `pos` of sequence b, KV head gk, sits in V: v_base(...) + v_index(...) * d.
+// Dense caches: the (b, gk) plane and the position; paged caches: the pool and the pool row
+// of the token's page.
+template <int D>
+__device__ __forceinline__ const __nv_bfloat16 *v_base(const SaParams &p, const NoPaging &, int b,
+                                                       int gk) {
+  return p.V + (static_cast<long long>(b) * p.Hkv + gk) * p.cap * D;
+}
+template <int D>
+__device__ __forceinline__ const __nv_bfloat16 *v_base(const SaParams &p, const PagedInfo &, int,
+                                                       int) {
+  return p.V;
+}
+__device__ __forceinline__ int v_index(const SaParams &, const NoPaging &, int, int, int pos) {
+  return pos;
+}
+__device__ __forceinline__ int v_index(const SaParams &p, const PagedInfo &pg, int b, int gk, int pos) {
+  const int page = __ldg(pg.block_table + static_cast<long long>(b) * pg.max_pages + pos / kPageSize);
+  return (page * p.Hkv + gk) * kPageSize + pos % kPageSize;
+}
+
 // ln sum_{j < N} e^{z_j} of one score row (the log of Eq. (1)'s softmax normaliser), cluster-
 // wide: each CTA folds its candidates [lo, hi) and its share of W into a running (max, sum),
 // the CTAs exchange theirs through distributed shared memory and all merge them.
 template <int D>
-__device__ float row_logsumexp(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
+__device__ float row_logsumexp(const RowGeo &gm, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
                                int ncl, const float *srow, long long lo, long long hi) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float m = -INFINITY, s = 0.f;
@@ -461,10 +504,10 @@ __device__ float row_logsumexp(const SaParams &p, SaSmem<D> &sm, cg::cluster_gro
     }
   };
   for (long long i = lo + tid; i < hi; i += kSaThreads) add(__ldcg(srow + i));
-  const long long wper = (p.nW + ncl - 1) / ncl;
-  const long long w_hi = min(p.nW, (rank + 1) * wper);
+  const long long wper = (gm.nW + ncl - 1) / ncl;
+  const long long w_hi = min(gm.nW, (rank + 1) * wper);
   for (long long e = rank * wper + tid; e < w_hi; e += kSaThreads)
-    add(__ldcg(srow + (e < p.s1 ? e : p.w0 + (e - p.s1))));
+    add(__ldcg(srow + (e < gm.s1 ? e : gm.w0 + (e - gm.s1))));
   // merge (m, s) over the warp, then over the CTA's warps
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -496,19 +539,19 @@ __device__ float row_logsumexp(const SaParams &p, SaSmem<D> &sm, cg::cluster_gro
 
 // Omega of one query head into irow (cluster-wide; every CTA takes the same branches).
 template <int D>
-__device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
-                             int ncl, int row) {
+__device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
+                             cg::cluster_group &cl, int rank, int ncl, int row) {
   const int tid = threadIdx.x;
   int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   if (rank == 0)
-    for (long long i = p.k_eff + tid; i < p.k; i += kSaThreads) irow[i] = -1;
-  if (p.k_eff == 0) return;
-  const long long a0 = p.cbase + static_cast<long long>(rank) * p.cper;
-  const long long lo = max(a0, p.s1), hi = min(a0 + p.cper, p.w0);
+    for (long long i = gm.k_eff + tid; i < p.k; i += kSaThreads) irow[i] = -1;
+  if (gm.k_eff == 0) return;
+  const long long a0 = gm.cbase + static_cast<long long>(rank) * gm.cper;
+  const long long lo = max(a0, gm.s1), hi = min(a0 + gm.cper, gm.w0);
   const float *srow = p.S + static_cast<long long>(row) * p.ldS;
   uint32_t *h1 = p.hist + static_cast<long long>(row) * kHistBins;
   const ChunkSrc chunk{srow, a0, lo, hi};
-  long long k_sel = p.k_eff;   // keys to select (the budget; fewer under a threshold)
+  long long k_sel = gm.k_eff;   // keys to select (the budget; fewer under a threshold)
   for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
   if (tid == 0) {
     sm.n_sure = 0u;
@@ -518,7 +561,7 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   int b1i = -1;
   if (p.mode & kSaEps) {
     // Eq. (2)'s threshold: a_i > eps  <=>  z_i > T = ln(eps) + ln sum_j e^{z_j} (all N)
-    const float T = p.log_eps + row_logsumexp(p, sm, cl, rank, ncl, srow, lo, hi);
+    const float T = p.log_eps + row_logsumexp(gm, sm, cl, rank, ncl, srow, lo, hi);
     // this CTA's digit-1 histogram of its candidates and its count of z > T
     uint32_t cnt = 0;
     chunk.for_each([&](unsigned long long x) {
@@ -534,9 +577,9 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
     for (int c = 0; c < ncl; ++c) above_t += sm.x_b[c];
     k_sel = min(k_sel, above_t);
     if (rank == 0)
-      for (long long i = k_sel + tid; i < p.k_eff; i += kSaThreads) irow[i] = -1;
+      for (long long i = k_sel + tid; i < gm.k_eff; i += kSaThreads) irow[i] = -1;
     if (k_sel == 0) return;
-    if (k_sel < p.nC) {
+    if (k_sel < gm.nC) {
       b1i = cluster_thresh(sm, cl, rank, ncl, kHistBins, static_cast<uint32_t>(k_sel));
       b1i = sm.t_bin < 0 ? -1 : b1i + sm.t_bin;
     }
@@ -544,8 +587,8 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
     for (int i = tid; i < kHistBins; i += kSaThreads) sm.h[i] = 0u;
     __syncthreads();
   }
-  if (k_sel >= p.nC) {   // every candidate is selected
-    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - p.s1] = static_cast<int32_t>(i);
+  if (k_sel >= gm.nC) {   // every candidate is selected
+    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - gm.s1] = static_cast<int32_t>(i);
     return;
   }
   const uint32_t k_eff = static_cast<uint32_t>(k_sel);
@@ -571,7 +614,7 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   }
   const uint32_t above1 = sm.t_above;
   const uint32_t b1 = b1i < 0 ? 0u : static_cast<uint32_t>(b1i);
-  uint2 *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - p.s1);
+  uint2 *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - gm.s1);
   if (b1i >= 0) stream_chunk(sm, srow, spill, a0, lo, hi, b1);
   __syncthreads();
   if (tid < ncl) cl.map_shared_rank(sm.x_a, tid)[rank] = sm.n_sure;
@@ -614,22 +657,22 @@ __device__ void select_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
 constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
 constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
 
-template <int D>
-__device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
-                             int ncl, int row) {
+template <int D, class Pg>
+__device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, SaSmem<D> &sm,
+                             cg::cluster_group &cl, int rank, int ncl, int row) {
   constexpr int CPL = D / 32;   // channels per lane
   constexpr int kPer = kStage / kSaThreads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long nU = p.nW + p.k_eff;
+  const long long nU = gm.nW + gm.k_eff;
   const long long parts = static_cast<long long>(ncl) * p.nsplit;
   const long long per = (nU + parts - 1) / parts;
   const long long e_lo = (static_cast<long long>(blockIdx.z) * ncl + rank) * per;
   const long long e_hi = min(nU, e_lo + per);
   const int b = row / p.Hq, h = row - b * p.Hq;
-  const __nv_bfloat16 *Vh = p.V + (static_cast<long long>(b) * p.Hkv + h / p.G) * p.cap * D;
+  const __nv_bfloat16 *Vb = v_base<D>(p, pg, b, h / p.G);
   const float *srow = p.S + static_cast<long long>(row) * p.ldS;
   const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
-  int *spos = reinterpret_cast<int *>(sm.sure);
+  int *spos = reinterpret_cast<int *>(sm.sure);   // staged: the entry's V row (-1: none)
   float *sz = reinterpret_cast<float *>(sm.sure + kStage);
   float m = -INFINITY, zs = 0.f, acc[CPL];
 #pragma unroll
@@ -643,15 +686,15 @@ __device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
       const int i = tid + j * kSaThreads;
       const long long e = blk + i;
       long long pos = -1;
-      if (i < nb) pos = e < p.nW ? (e < p.s1 ? e : p.w0 + (e - p.s1)) : __ldcg(irow + (e - p.nW));
-      pp[j] = (pos >= 0 && pos < p.N) ? static_cast<int>(pos) : -1;   // always, for a complete idx
+      if (i < nb) pos = e < gm.nW ? (e < gm.s1 ? e : gm.w0 + (e - gm.s1)) : __ldcg(irow + (e - gm.nW));
+      pp[j] = (pos >= 0 && pos < gm.N) ? static_cast<int>(pos) : -1;   // always, for a complete idx
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int i = tid + j * kSaThreads;
       const float z = pp[j] >= 0 ? __ldcg(srow + pp[j]) : -INFINITY;
       if (i < nb) {
-        spos[i] = pp[j];
+        spos[i] = pp[j] >= 0 ? v_index(p, pg, b, h / p.G, pp[j]) : -1;
         sz[i] = z;
       }
     }
@@ -665,7 +708,7 @@ __device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
       for (int j = 0; j < kAttnRows; ++j) {
         const int pj = __shfl_sync(0xffffffffu, pos, j);
         if (pj >= 0) {
-          const __nv_bfloat16 *vr = Vh + static_cast<long long>(pj) * D;
+          const __nv_bfloat16 *vr = Vb + static_cast<long long>(pj) * D;
           if constexpr (CPL == 4) {
             const uint2 v = __ldg(reinterpret_cast<const uint2 *>(vr) + lane);
             wv[j][0] = v.x;
@@ -779,19 +822,20 @@ __device__ void attend_phase(const SaParams &p, SaSmem<D> &sm, cg::cluster_group
   cl.sync();   // the first CTA has read every partial state
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaParams p) {
+template <int D, class Pg>
+__global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaParams p, const Pg pg) {
   __shared__ SaSmem<D> sm;
   cg::cluster_group cl = cg::this_cluster();
   const int ncl = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
   const int row = blockIdx.y;
+  const RowGeo gm = row_geo(p, pg, row, ncl);
   pdl_trigger();
   pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
-  if (p.mode & kSaSelect) select_phase<D>(p, sm, cl, rank, ncl, row);
+  if (p.mode & kSaSelect) select_phase<D>(p, gm, sm, cl, rank, ncl, row);
   if (p.mode & kSaAttend) {
     if (p.mode & kSaSelect) cl.sync();   // Omega complete in idx (release/acquire at cluster scope)
-    attend_phase<D>(p, sm, cl, rank, ncl, row);
+    attend_phase<D>(p, gm, pg, sm, cl, rank, ncl, row);
   } else {
     cl.sync();   // no CTA leaves while the cluster may still use its shared memory
   }
@@ -811,7 +855,7 @@ static int active_clusters_t(int ncl) {
   while ((1 << li) < ncl) ++li;
   if (!done[dev][li]) {
     if (ncl > 8)
-      (void)cudaFuncSetAttribute(select_attend_kernel<D>,
+      (void)cudaFuncSetAttribute(select_attend_kernel<D, NoPaging>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(ncl), 1);
@@ -824,7 +868,8 @@ static int active_clusters_t(int ncl) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, select_attend_kernel<D>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, select_attend_kernel<D, NoPaging>, &cfg) != cudaSuccess)
+      n = 0;
     (void)cudaGetLastError();   // a refused query leaves no error behind
     cache[dev][li] = n;
     done[dev][li] = true;
@@ -846,8 +891,16 @@ int select_cluster_size(long long nC, int R, int d) {
   return n;
 }
 
-template <int D>
-static cudaError_t launch_sa_t(const SaParams &p, int R, int ncl, cudaStream_t s) {
+template <int D, class Pg>
+static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (ncl > 8 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !attr_done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg>,
+                                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ncl), static_cast<unsigned>(R),
                      static_cast<unsigned>(p.nsplit < 1 ? 1 : p.nsplit));
@@ -863,7 +916,7 @@ static cudaError_t launch_sa_t(const SaParams &p, int R, int ncl, cudaStream_t s
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D>, p);
+  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D, Pg>, p, pg);
 }
 
 int attn_split(long long nU, int R, int ncl, int d) {
@@ -874,11 +927,21 @@ int attn_split(long long nU, int R, int ncl, int d) {
   return n;
 }
 
+static bool valid_launch(const SaParams &p, int ncl) {
+  if (ncl < 1 || ncl > kMaxCluster || (ncl & (ncl - 1)) != 0) return false;
+  return p.nsplit >= 1 && p.nsplit <= kMaxAttnSplit && !(p.nsplit > 1 && (p.mode & kSaSelect));
+}
+
 cudaError_t launch_select_attend(const SaParams &p, int d, int R, int ncl, cudaStream_t s) {
-  if (ncl < 1 || ncl > kMaxCluster || (ncl & (ncl - 1)) != 0) return cudaErrorInvalidValue;
-  if (p.nsplit < 1 || p.nsplit > kMaxAttnSplit || (p.nsplit > 1 && (p.mode & kSaSelect)))
-    return cudaErrorInvalidValue;
-  return d == 128 ? launch_sa_t<128>(p, R, ncl, s) : launch_sa_t<64>(p, R, ncl, s);
+  if (!valid_launch(p, ncl)) return cudaErrorInvalidValue;
+  const NoPaging pg{};
+  return d == 128 ? launch_sa_t<128>(p, pg, R, ncl, s) : launch_sa_t<64>(p, pg, R, ncl, s);
+}
+
+cudaError_t launch_select_attend_paged(const SaParams &p, const PagedInfo &pg, int d, int R, int ncl,
+                                       cudaStream_t s) {
+  if (!valid_launch(p, ncl)) return cudaErrorInvalidValue;
+  return d == 128 ? launch_sa_t<128>(p, pg, R, ncl, s) : launch_sa_t<64>(p, pg, R, ncl, s);
 }
 
 }  // namespace ra

@@ -22,12 +22,19 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_decode_workspace_bytes", "ra_decode_step", "ra_score_gqa", "ra_topk_select",
            "ra_sparse_attn", "ra_select_attend", "ra_dense_workspace_bytes", "ra_dense_decode",
            "ra_decode_step_static", "ra_prefill_workspace_bytes", "ra_prefill_topk",
-           "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets")
+           "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets",
+           "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step")
 
 
 class ra_kv(ctypes.Structure):
     _fields_ = [("K", c_void_p), ("V", c_void_p), ("B", c_int32), ("Hkv", c_int32),
                 ("d", c_int32), ("cap", c_int32), ("N", c_int64)]
+
+
+class ra_paged_kv(ctypes.Structure):
+    _fields_ = [("K", c_void_p), ("V", c_void_p), ("block_table", c_void_p),
+                ("seq_len", ctypes.POINTER(c_int32)), ("B", c_int32), ("Hkv", c_int32),
+                ("d", c_int32), ("max_pages", c_int32), ("num_pages", c_int32)]
 
 
 _lib = None
@@ -61,6 +68,13 @@ def lib() -> ctypes.CDLL:
             "ra_dense_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32]),
             "ra_dense_decode": (c_int32, [P, c_void_p, c_int32, c_void_p, c_void_p, c_size_t,
                                           c_void_p]),
+            "ra_paged_append_kv": (c_int32, [ctypes.POINTER(ra_paged_kv), c_void_p, c_void_p,
+                                             c_int32, c_void_p]),
+            "ra_paged_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32, c_int32,
+                                                    c_int32, c_int32]),
+            "ra_paged_decode_step": (c_int32, [ctypes.POINTER(ra_paged_kv), c_void_p, c_int32, c_int32,
+                                               c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                               c_size_t, c_void_p]),
             "ra_pyramid_budgets": (c_int32, [c_int32, c_int32, ctypes.c_double,
                                              ctypes.POINTER(c_int32)]),
             "ra_decode_step_eps": (c_int32, [P, c_void_p, c_int32, c_int32, ctypes.c_float, c_int32,
@@ -289,6 +303,64 @@ def decode_step_eps(cache: KVCache, q, k: int, eps: float, n_sink: int, n_window
     check(ra_decode_step_eps(cache.kv, q.data_ptr(), Hq, k, eps, n_sink, n_window, out.data_ptr(),
                              idx.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
           "ra_decode_step_eps")
+    return out, idx[..., :k]
+
+
+PAGE = 128
+
+
+class PagedKVCache:
+    """A paged layer cache: torch-allocated page pools [num_pages, Hkv, 128, d] (bf16), a device
+    block table [B, max_pages] (int32) and host lengths; `kv` is the C struct over them."""
+
+    def __init__(self, B: int, Hkv: int, d: int, num_pages: int, max_pages: int, device="cuda"):
+        import torch
+        self.B, self.Hkv, self.d = B, Hkv, d
+        self.num_pages, self.max_pages = num_pages, max_pages
+        self.K = torch.empty((num_pages, Hkv, PAGE, d), dtype=torch.bfloat16, device=device)
+        self.V = torch.empty_like(self.K)
+        self.block_table = torch.zeros((B, max_pages), dtype=torch.int32, device=device)
+        self._lens = (c_int32 * B)()
+        self.kv = ra_paged_kv(self.K.data_ptr(), self.V.data_ptr(), self.block_table.data_ptr(),
+                              self._lens, B, Hkv, d, max_pages, num_pages)
+
+    @property
+    def seq_len(self) -> list[int]:
+        return list(self._lens)
+
+    def set_lengths(self, lens) -> None:
+        for b, n in enumerate(lens):
+            self._lens[b] = int(n)
+
+
+def paged_append_kv(cache: PagedKVCache, k_new, v_new, stream=None) -> None:
+    """Append T tokens per sequence (k_new / v_new bf16 [B, Hkv, T, d])."""
+    check(lib().ra_paged_append_kv(ctypes.byref(cache.kv), k_new.data_ptr(), v_new.data_ptr(),
+                                   k_new.shape[2], _stream(stream)), "ra_paged_append_kv")
+
+
+def paged_workspace(cache: PagedKVCache, Hq: int, k: int, n_sink: int, n_window: int):
+    import torch
+    n = lib().ra_paged_workspace_bytes(cache.B, Hq, max(cache.seq_len), cache.d, k, n_sink, n_window)
+    if n == 0:
+        raise RaError(RA_ERR_SHAPE, "ra_paged_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=cache.K.device)
+
+
+def paged_decode_step(cache: PagedKVCache, q, k: int, n_sink: int, n_window: int, out=None,
+                      idx=None, ws=None, stream=None):
+    """The decode step on a paged cache with per-sequence lengths.  Returns (out, idx)."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        ws = paged_workspace(cache, Hq, k, n_sink, n_window)
+    check(lib().ra_paged_decode_step(ctypes.byref(cache.kv), q.data_ptr(), Hq, k, n_sink, n_window,
+                                     out.data_ptr(), idx.data_ptr(), ws.data_ptr(), ws.numel(),
+                                     _stream(stream)), "ra_paged_decode_step")
     return out, idx[..., :k]
 
 
