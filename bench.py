@@ -43,7 +43,7 @@ FALLBACK_HBM_GBS = 6650.0
 # keyed by the sha256 of the score kernel's own sources (score.cu and its TMA helpers) it was
 # taken on, so a changed kernel reports null until it is captured again.  Values are per launch
 # of the named workload (profiles/score_gqa_l8b_128k.md).
-TRAFFIC = {("063948ee6f144422", "l8b_128k_k1pct"): 275.65e6}
+TRAFFIC = {("7d70c406e21ebd58", "l8b_128k_k1pct"): 275.46e6}
 
 
 def score_source_hash() -> str:
@@ -71,6 +71,9 @@ def parse():
     ap.add_argument("--pyramid", type=float, default=0.0,
                     help="per-layer budgets falling linearly with depth to this ratio of the "
                          "first layer's, mean k (ra_pyramid_budgets)")
+    ap.add_argument("--paged", action="store_true",
+                    help="paged cache (128-token pages, shuffled) with ragged lengths falling "
+                         "linearly from N to N/2 over the batch (ra_paged_decode_step)")
     ap.add_argument("--prefill-queries", type=int, default=0,
                     help="instead of decode steps: exact top-k of this many prefill queries per "
                          "query head (tensor-core scores + cluster selection), one layer")
@@ -549,6 +552,112 @@ def run_ours(args, w, rank, local_rank, world, dist):
     return result
 
 
+def run_paged(args, w, rank, local_rank, world, dist):
+    """Decode steps on a paged cache with ragged lengths: sequence b holds
+    N - (N / 2) * b / (B - 1) tokens (rounded down to a multiple of 4), pages shuffled over the
+    pool; each step appends one token per sequence and decodes (one layer)."""
+    import ctypes
+
+    import torch
+
+    import top_retrieval_attention_b200 as ra
+    from synth import device as sdev
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    B, Hq, Hkv, d, N, k = w.B, w.Hq, w.Hkv, w.d, w.N, w.k
+    PAGE = 128
+    lens = [max(1, (N - (N // 2) * b // max(B - 1, 1)) // 4 * 4) for b in range(B)]
+    need = [(n + 1 + PAGE - 1) // PAGE for n in lens]            # room for the appended token
+    num_pages, max_pages = sum(need), max(need)
+    cache = ra.PagedKVCache(B, Hkv, d, num_pages, max_pages, device=dev)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    order = torch.randperm(num_pages, generator=g).to(torch.int32)
+    table = torch.zeros((B, max_pages), dtype=torch.int32)
+    j = 0
+    for b in range(B):
+        table[b, :need[b]] = order[j:j + need[b]]
+        j += need[b]
+    cache.block_table.copy_(table)
+    # fill: each sequence's dense rows from the generator, scattered into its pages
+    for b in range(B):
+        rows = need[b] * PAGE
+        Kd = torch.empty((1, Hkv, rows, d), dtype=torch.bfloat16, device=dev)
+        Vd = torch.empty_like(Kd)
+        sdev.fill_kv(Kd, Vd, 0, rows, w.seed + b, 0, with_offset=True)
+        pages = table[b, :need[b]].to(dev).long()
+        cache.K[pages] = Kd[0].view(Hkv, need[b], PAGE, d).permute(1, 0, 2, 3)
+        cache.V[pages] = Vd[0].view(Hkv, need[b], PAGE, d).permute(1, 0, 2, 3)
+        del Kd, Vd
+    cache.set_lengths(lens)
+    P = 16
+    qpool = torch.empty((P, B, Hq, d), dtype=torch.bfloat16, device=dev)
+    for s in range(P):
+        sdev.fill_q(qpool[s], w.seed + 7919 * s)
+    knew = torch.zeros((B, Hkv, 1, d), dtype=torch.bfloat16, device=dev)
+    vnew = torch.zeros_like(knew)
+    ws_bytes = ra.lib().ra_paged_workspace_bytes(B, Hq, max(lens) + 1, d, k, w.n_sink, w.n_window)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hq, k), dtype=torch.int32, device=dev)
+
+    def step(s):
+        ra.check(ra.lib().ra_paged_append_kv(ctypes.byref(cache.kv), knew.data_ptr(),
+                                             vnew.data_ptr(), 1, sp), "paged_append")
+        ra.check(ra.lib().ra_paged_decode_step(ctypes.byref(cache.kv), qpool[s % P].data_ptr(), Hq,
+                                               k, w.n_sink, w.n_window, out.data_ptr(),
+                                               idx.data_ptr(), ws.data_ptr(), ws_bytes, sp),
+                 "paged_decode")
+        cache.set_lengths(lens)   # the next step re-appends into the same slot
+
+    for s in range(max(3, args.warmup)):
+        step(s)
+    torch.cuda.synchronize()
+    steps = args.steps if args.steps is not None else 200
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    clk = Clocks(uuid)
+    clk.start()
+    barrier(dist, local_rank)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        step(s)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, local_rank)
+    clocks = clk.stop()
+    ms = max_over_ranks(dist, t0.elapsed_time(t1), dev) / steps
+    n1 = [n + 1 for n in lens]
+    k_bytes = sum(Hkv * n * 2 * d for n in n1)
+    v_bytes = 0
+    for n in n1:
+        s1 = min(w.n_sink, n)
+        w0 = max(s1, n - w.n_window)
+        v_bytes += Hq * (s1 + n - w0 + min(k, w0 - s1)) * 2 * d
+    peak, peak_kind = measured_hbm_peak()
+    gbs = (k_bytes + v_bytes) / (ms / 1000.0) / 1e9
+    return {
+        "metric": METRIC + " (paged, ragged lengths)", "value": world * 1000.0 / ms,
+        "unit": "steps/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 / Irwin-Hall normals), pages shuffled",
+        "config": dict(workload_config(w), paged=True, page_tokens=PAGE, lengths=lens),
+        "roofline": {"kernel": "paged decode step (score + select + attend)", "bound": "hbm",
+                     "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": k_bytes + v_bytes},
+        "gpu_launches": 3 * steps, "clocks": clocks,
+    }
+
+
 def run_prefill(args, w, rank, local_rank, world, dist):
     """Exact top-k of M prefill queries per query head against one layer's cache: the
     tcgen05 score GEMM (timed on its own for its roofline) and the cluster selection."""
@@ -658,6 +767,8 @@ def main():
     try:
         if args.prefill_queries > 0:
             res = run_prefill(args, w, rank, local_rank, world, dist)
+        elif args.paged:
+            res = run_paged(args, w, rank, local_rank, world, dist)
         else:
             res = run_ours(args, w, rank, local_rank, world, dist)
         if rank == 0:
