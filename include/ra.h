@@ -260,6 +260,56 @@ ra_status ra_prefill_select(const ra_kv *kv, int32_t Hq, int32_t M, int32_t k, i
                             int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
                             ra_stream_t stream);
 
+/*
+ * Device-side approximate retrieval: an inverted-file (IVF) index of one layer's keys (the
+ * pages' IVF baseline over the keys, probed with the decode query; slide "Available GPU memory
+ * changes the comparison"), built and searched on the GPU.  Not exact: a key of a cluster that
+ * is not probed is never retrieved.
+ *   Ksorted   : bf16 [B, Hkv, N, d], the keys ordered by cluster.
+ *   pos       : int32 [B, Hkv, N], the cache position of each sorted key.
+ *   offsets   : int32 [B, Hkv, nlist + 1], cluster c's keys are sorted entries
+ *               [offsets[c], offsets[c + 1]).
+ *   centroids : bf16 [B, Hkv, nlist, d], unit-norm (spherical k-means: keys are assigned to the
+ *               centroid of largest inner product, ties to the lower index).
+ *   All device, caller-owned.  N is the number of keys indexed; 1 <= nlist <= 4096.
+ */
+typedef struct {
+  void *Ksorted;
+  int32_t *pos;
+  int32_t *offsets;
+  void *centroids;
+  int32_t B, Hkv, d, nlist;
+  int64_t N;
+} ra_ivf;
+
+/*
+ * Build the index of kv's first ix->N keys (ix->N <= kv->N; B, Hkv, d as kv's): `iters` Lloyd
+ * iterations of spherical k-means from centroids at evenly spaced keys (the key-centroid scores
+ * on the tcgen05 tensor cores), then the final assignment and the sort by cluster.
+ *   ws : at least ra_ivf_build_workspace_bytes(...) bytes, 256-byte aligned.
+ * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_WORKSPACE, RA_ERR_CUDA.
+ */
+size_t ra_ivf_build_workspace_bytes(int32_t B, int32_t Hkv, int64_t N, int32_t d, int32_t nlist);
+ra_status ra_ivf_build(const ra_kv *kv, ra_ivf *ix, int32_t iters, void *ws, size_t ws_bytes,
+                       ra_stream_t stream);
+
+/*
+ * A decode step that retrieves through the index: per query head, the nprobe clusters whose
+ * centroids score highest, the exact top-k of their keys outside W (ties to the lower position),
+ * and softmax attention over W u Omega as ra_decode_step.  Keys appended after the build are
+ * only attended through the window: kv->N - ix->N <= n_window is required.
+ *   nprobe : 1 <= nprobe <= min(nlist, 64).   idx : -1 past the keys retrieved.
+ *   ws     : at least ra_ivf_search_workspace_bytes(...) bytes, 256-byte aligned, zero-filled
+ *            once (it holds a decode workspace's counter block).
+ * Errors: as ra_decode_step; RA_ERR_ARG for nprobe or an index that does not cover the cache.
+ */
+size_t ra_ivf_search_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, int32_t k,
+                                     int32_t nprobe);
+ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, int32_t Hq,
+                             int32_t k, int32_t nprobe, int32_t n_sink, int32_t n_window,
+                             float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                             ra_stream_t stream);
+
 /* Workspace bytes for ra_dense_decode (split partial states).  0 for an invalid shape. */
 size_t ra_dense_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d);
 

@@ -290,3 +290,34 @@ def gather_paged(pool: np.ndarray, table: np.ndarray, lens) -> list:
         rows = [pool[table[b][i // P], :, i % P, :] for i in range(int(n))]
         out.append(np.stack(rows, axis=1) if rows else pool[:0, :, 0, :].transpose(1, 0, 2))
     return out
+
+
+# ------------------------------------------------------------------------------------
+# IVF retrieval (the pages' IVF baseline over the keys, slide "Available GPU memory changes
+# the comparison"): given an index (keys grouped by cluster, unit-norm centroids), probe the
+# nprobe clusters whose centroids score highest and take the exact top-k of their keys
+
+
+def ivf_probe(q: np.ndarray, centroids: np.ndarray, nprobe: int) -> np.ndarray:
+    """The nprobe clusters with the largest q . c (ties to the lower cluster index)."""
+    zc = centroids @ q
+    order = np.lexsort((np.arange(zc.size), -zc))
+    return order[:nprobe]
+
+
+def ivf_decode_head(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray,
+                    pos: np.ndarray, offsets: np.ndarray, cent_bits: np.ndarray, k: int,
+                    nprobe: int, n_sink: int, n_window: int):
+    """One query head through an IVF index of its KV head: returns (o [d], Omega, z, probe).
+    pos [N_ix] are the cache positions grouped by cluster, offsets [nlist + 1] the groups."""
+    q = bf16_to_f64(q_bits)
+    K = bf16_to_f64(K_bits)
+    V = bf16_to_f64(V_bits)
+    N = K.shape[0]
+    z = scores(q, K)
+    probe = ivf_probe(q, bf16_to_f64(cent_bits), nprobe)
+    cand = np.concatenate([pos[offsets[c]:offsets[c + 1]] for c in probe]).astype(np.int64)
+    C = np.intersect1d(cand, candidate_set(N, n_sink, n_window))
+    omega = select_topk(z, C, k)
+    U = np.concatenate([static_set(N, n_sink, n_window), omega])
+    return attend(z, V, U), omega, z, probe

@@ -522,3 +522,42 @@ def test_gather_paged_inverts_a_scatter_by_the_definition():
     got = oracle.gather_paged(pool, table, lens)
     for b in range(B):
         assert np.array_equal(got[b], dense[b])
+
+
+# ---------------------------------------------------------------- IVF retrieval
+
+
+def test_ivf_probing_every_cluster_is_exact_retrieval():
+    """With every cluster probed, IVF retrieval is the exact top-k step, for any partition of
+    the keys into clusters (the index only restricts the candidates)."""
+    rng = np.random.default_rng(21)
+    N, d, nlist, k = 500, 64, 7, 40
+    q, K, V = rand_bf16(d), rand_bf16((N, d)), rand_bf16((N, d))
+    assign = rng.integers(0, nlist, size=N)
+    pos = np.argsort(assign, kind="stable")
+    offsets = np.concatenate([[0], np.cumsum(np.bincount(assign, minlength=nlist))])
+    cent = rand_bf16((nlist, d))
+    o_ivf, om_ivf, _, probe = oracle.ivf_decode_head(q, K, V, pos, offsets, cent, k, nlist, 4, 32)
+    o, om, _ = oracle.decode_head(q, K, V, k, 4, 32)
+    assert sorted(probe.tolist()) == list(range(nlist))
+    assert np.array_equal(np.sort(om_ivf), np.sort(om))
+    assert np.allclose(o_ivf, o, rtol=0, atol=1e-12)
+
+
+def test_ivf_candidates_are_the_probed_clusters():
+    """Keys of unprobed clusters are never retrieved; the probe is the top-nprobe centroids by
+    q . c with ties to the lower index."""
+    d, N = 64, 300
+    q = gen.f64_to_bf16_bits(np.eye(d)[0] * 1.0)                     # q = e_0
+    cent = gen.f64_to_bf16_bits(np.array([np.eye(d)[i % d] * (1.0 if i != 3 else 2.0)
+                                          for i in range(6)]))        # c_3 scores 0, c_0 1
+    cent[2] = cent[0]                                                 # c_0 and c_2 tie
+    probe = oracle.ivf_probe(oracle.bf16_to_f64(q), oracle.bf16_to_f64(cent), 2)
+    assert list(probe) == [0, 2]
+    rng = np.random.default_rng(3)
+    K, V = rand_bf16((N, d)), rand_bf16((N, d))
+    assign = np.arange(N) % 6
+    pos = np.argsort(assign, kind="stable")
+    offsets = np.concatenate([[0], np.cumsum(np.bincount(assign, minlength=6))])
+    _, om, _, _ = oracle.ivf_decode_head(q, K, V, pos, offsets, cent, 1000, 2, 0, 0)
+    assert set(om.tolist()) == {i for i in range(N) if i % 6 in (0, 2)}

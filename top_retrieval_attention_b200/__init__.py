@@ -8,5 +8,6 @@ from .ra import (  # noqa: F401
     ra_select_attend, ra_sparse_attn, ra_status_str, ra_topk_select, ra_version,
     ra_prefill_workspace_bytes, ra_prefill_topk, ra_prefill_score, ra_prefill_select, prefill_topk,
     ra_decode_step_eps, decode_step_eps, pyramid_budgets, ra_paged_kv, PagedKVCache,
-    paged_append_kv, paged_workspace, paged_decode_step,
+    paged_append_kv, paged_workspace, paged_decode_step, ra_ivf, IvfIndex, ivf_build,
+    ivf_decode_step,
 )

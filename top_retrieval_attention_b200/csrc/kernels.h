@@ -86,6 +86,8 @@ struct SaParams {
   int k, Hq, G, Hkv, mode;
   int nsplit;               // clusters per query head (grid z); > 1 only for attention alone
   float log_eps;            // kSaEps: ln(eps)
+  const int32_t *row_n;     // if set: row r's candidates are [0, row_n[r]) of its score row,
+                            // with no static set (the IVF candidate lists)
 };
 
 // Scores of prefill queries (rows (b, h, m) of Q [B, Hq, M, d]) against the keys of their KV
@@ -96,10 +98,41 @@ struct PfParams {
   float *S;                 // [B*Hq*M, ldS]
   uint32_t *err;            // error word (bit kErrPrefillWait: a copy or the MMAs never landed)
   long long N, cap, ldS;
+  long long q_plane_rows;   // rows between KV heads' query blocks in Q (0: G * M, contiguous)
   int B, Hq, Hkv, G, M;
   float scale;
 };
 constexpr uint32_t kErrPrefillWait = 8u;
+
+// IVF index build over one layer's keys (per KV head, bg = b * Hkv + g).
+struct IvfParams {
+  const __nv_bfloat16 *K;   // cache keys [BH, cap, d]
+  __nv_bfloat16 *cent;      // [BH, nlist, d] unit-norm centroids
+  const float *A;           // [BH * N, ldA] key-centroid scores of the current iteration
+  float *sums;              // [BH, nlist, d]
+  uint32_t *count, *cursor; // [BH, nlist]
+  int32_t *assign;          // [BH * N]
+  int32_t *offsets;         // [BH, nlist + 1]
+  int32_t *pos;             // [BH, N] cache position of each sorted key
+  __nv_bfloat16 *Ksorted;   // [BH, N, d]
+  long long N, cap, ldA;
+  int BH, nlist, d;
+};
+
+// IVF search of one decode step (rows = b * Hq + h).
+struct IvfSearchParams {
+  const __nv_bfloat16 *q, *K, *Ksorted, *cent;
+  const int32_t *pos, *offsets;
+  int32_t *probe, *cand_off, *n_cand;   // [R, nprobe], [R, nprobe + 1], [R]
+  float *S;                 // [R, ldS] full-length score rows (written at candidate and W positions)
+  float *S_cand;            // [R, ldC] candidate scores (-inf: a W key)
+  int32_t *pos_cand;        // [R, ldC]
+  const int32_t *idx_cand;  // [R, k] selected candidate indices
+  int32_t *idx;             // [R, k] their cache positions
+  long long N, cap, ldS, ldC, s1, w0, nW;
+  int R, Hq, Hkv, G, d, nlist, nprobe, k;
+  float scale;
+};
 
 struct DenseParams {
   const __nv_bfloat16 *K, *V, *q;
@@ -147,6 +180,13 @@ cudaError_t launch_select_attend_paged(const SaParams &p, const PagedInfo &pg, i
                                        cudaStream_t s);
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
 cudaError_t launch_prefill_score(const PfParams &p, int d, cudaStream_t s);
+cudaError_t launch_ivf_init(const IvfParams &p, cudaStream_t s);
+cudaError_t launch_ivf_assign(const IvfParams &p, bool accumulate, cudaStream_t s);
+cudaError_t launch_ivf_update(const IvfParams &p, cudaStream_t s);
+cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s);
+cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s);
+cudaError_t launch_ivf_cand(const IvfSearchParams &p, int d, cudaStream_t s);
+cudaError_t launch_ivf_map(const IvfSearchParams &p, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
 cudaError_t launch_append_paged(const AppendParams &p, const PagedInfo &pg, cudaStream_t s);
 

@@ -63,10 +63,6 @@ __global__ void __launch_bounds__(kPfThreads, 2)
   const long long key0 = static_cast<long long>(blockIdx.x) * kPfN;
   const int qb = blockIdx.y;                               // 128-row block of the head's rows
   const int bg = blockIdx.z;                               // b * Hkv + g
-  const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-  const long long head_rows = static_cast<long long>(p.G) * p.M;
-  const long long row0 = (static_cast<long long>(b) * p.Hq + static_cast<long long>(g) * p.G) * p.M +
-                         static_cast<long long>(qb) * kPfM;   // first flattened query row
 
   pdl_trigger();
   if (warp == 0) tmem_alloc(slot, kPfN);
@@ -88,7 +84,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
     mbar_arrive_expect_tx(bar_load, C::kABytes + C::kBBytes);
 #pragma unroll
     for (int bx = 0; bx < C::kBoxes; ++bx) {
-      tma_load_3d(sA + bx * C::kABox, &tmQ, bx * 64, static_cast<int>(row0), 0, bar_load, pol);
+      tma_load_3d(sA + bx * C::kABox, &tmQ, bx * 64, qb * kPfM, bg, bar_load, pol);
       tma_load_3d(sB + bx * C::kBBox, &tmK, bx * 64, static_cast<int>(key0), bg, bar_load, pol);
     }
     if (mbar_wait(bar_load, 0)) {
@@ -185,10 +181,13 @@ static cudaError_t launch_prefill_t(const PfParams &p, cudaStream_t s) {
   cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(prefill_score_kernel<D>),
                                     static_cast<int>(C::smem_bytes()), done);
   if (e != cudaSuccess) return e;
-  const long long q_rows = static_cast<long long>(p.B) * p.Hq * p.M;
+  // queries as [B * Hkv planes][G * M rows][d] (planes q_plane_rows rows apart): the G * M rows
+  // of a KV head's query heads are contiguous in [B, Hq, M, d]; rows past G * M read as zeros
+  const long long head_rows_q = static_cast<long long>(p.G) * p.M;
   CUtensorMap tq, tk;
-  if (!encode_rows_tmap(&tq, p.Q, D, static_cast<uint64_t>(q_rows), 1, kPfM,
-                        static_cast<uint64_t>(q_rows)))
+  if (!encode_rows_tmap(&tq, p.Q, D, static_cast<uint64_t>(head_rows_q),
+                        static_cast<uint64_t>(p.B) * p.Hkv, kPfM,
+                        static_cast<uint64_t>(p.q_plane_rows > 0 ? p.q_plane_rows : head_rows_q)))
     return cudaErrorInvalidValue;
   if (!encode_rows_tmap(&tk, p.K, D, static_cast<uint64_t>(p.N),
                         static_cast<uint64_t>(p.B) * p.Hkv, kPfN, static_cast<uint64_t>(p.cap)))

@@ -635,4 +635,186 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
   return RA_OK;
 }
 
+// ---- IVF index
+
+struct IvfBuildLayout {
+  size_t off_A, off_sums, off_count, off_cursor, off_assign, off_err, total;
+  long long ldA;
+};
+static bool ivf_build_layout(int B, int Hkv, long long N, int d, int nlist, IvfBuildLayout &L) {
+  if (B < 1 || Hkv < 1 || N < 1 || (d != 64 && d != 128) || nlist < 1 || nlist > 4096) return false;
+  const size_t BH = static_cast<size_t>(B) * Hkv;
+  L.ldA = round4(nlist);
+  size_t off = 0;
+  L.off_A = off;      off = align_up(off + BH * N * L.ldA * 4);
+  L.off_sums = off;   off = align_up(off + BH * nlist * d * 4);
+  L.off_count = off;  off = align_up(off + BH * nlist * 4);
+  L.off_cursor = off; off = align_up(off + BH * nlist * 4);
+  L.off_assign = off; off = align_up(off + BH * N * 4);
+  L.off_err = off;    off = align_up(off + 4);
+  L.total = off;
+  return true;
+}
+
+size_t ra_ivf_build_workspace_bytes(int32_t B, int32_t Hkv, int64_t N, int32_t d, int32_t nlist) {
+  IvfBuildLayout L{};
+  return ivf_build_layout(B, Hkv, N, d, nlist, L) ? L.total : 0;
+}
+
+ra_status ra_ivf_build(const ra_kv *kv, ra_ivf *ix, int32_t iters, void *ws, size_t ws_bytes,
+                       ra_stream_t stream) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (!ix || !ix->Ksorted || !ix->pos || !ix->offsets || !ix->centroids || iters < 0) return RA_ERR_ARG;
+  if (!aligned16(ix->Ksorted) || !aligned16(ix->centroids)) return RA_ERR_ARG;
+  if (ix->B != kv->B || ix->Hkv != kv->Hkv || ix->d != kv->d || ix->N < 1 || ix->N > kv->N)
+    return RA_ERR_SHAPE;
+  IvfBuildLayout L{};
+  if (!ivf_build_layout(kv->B, kv->Hkv, ix->N, kv->d, ix->nlist, L)) return RA_ERR_SHAPE;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < L.total)
+    return RA_ERR_WORKSPACE;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  IvfParams p{};
+  p.K = static_cast<const __nv_bfloat16 *>(kv->K);
+  p.cent = static_cast<__nv_bfloat16 *>(ix->centroids);
+  p.A = reinterpret_cast<const float *>(at(ws, L.off_A));
+  p.sums = reinterpret_cast<float *>(at(ws, L.off_sums));
+  p.count = reinterpret_cast<uint32_t *>(at(ws, L.off_count));
+  p.cursor = reinterpret_cast<uint32_t *>(at(ws, L.off_cursor));
+  p.assign = reinterpret_cast<int32_t *>(at(ws, L.off_assign));
+  p.offsets = ix->offsets;
+  p.pos = ix->pos;
+  p.Ksorted = static_cast<__nv_bfloat16 *>(ix->Ksorted);
+  p.N = ix->N; p.cap = kv->cap; p.ldA = L.ldA;
+  p.BH = kv->B * kv->Hkv; p.nlist = ix->nlist; p.d = kv->d;
+  // the key-centroid scores: the keys as the query rows of the tensor-core score kernel
+  PfParams f{};
+  f.Q = static_cast<const __nv_bfloat16 *>(kv->K);
+  f.K = p.cent;
+  f.S = reinterpret_cast<float *>(at(ws, L.off_A));
+  f.err = reinterpret_cast<uint32_t *>(at(ws, L.off_err));
+  f.N = ix->nlist; f.cap = ix->nlist; f.ldS = L.ldA; f.q_plane_rows = kv->cap;
+  f.B = kv->B; f.Hq = kv->Hkv; f.Hkv = kv->Hkv; f.G = 1; f.M = static_cast<int>(ix->N);
+  f.scale = 1.0f;
+  cudaError_t e = cudaMemsetAsync(at(ws, L.off_sums), 0, L.off_assign - L.off_sums, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at(ws, L.off_err), 0, 4, cs);
+  if (e == cudaSuccess) e = launch_ivf_init(p, cs);
+  for (int it = 0; it <= iters && e == cudaSuccess; ++it) {
+    e = launch_prefill_score(f, kv->d, cs);
+    if (e == cudaSuccess) e = launch_ivf_assign(p, it < iters, cs);
+    if (e == cudaSuccess && it < iters) e = launch_ivf_update(p, cs);
+  }
+  if (e == cudaSuccess) e = launch_ivf_sort(p, cs);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "ivf_build");
+}
+
+struct IvfSearchLayout {
+  Step st;                  // the selection's plan over candidate rows of up to N entries
+  size_t off_Sfull, off_poscand, off_probe, off_candoff, off_ncand, off_idxc, total;
+};
+static bool ivf_search_layout(int B, int Hq, long long N, int d, int k, int nprobe,
+                              IvfSearchLayout &L) {
+  if (nprobe < 1 || nprobe > 64) return false;
+  if (plan_shape(B, Hq, Hq, N, d, k, 0, 0, L.st) != RA_OK) return false;
+  const size_t R = static_cast<size_t>(B) * Hq;
+  size_t off = L.st.total;
+  L.off_Sfull = off;   off = align_up(off + R * L.st.ldS * 4);
+  L.off_poscand = off; off = align_up(off + R * L.st.ldS * 4);
+  L.off_probe = off;   off = align_up(off + R * nprobe * 4);
+  L.off_candoff = off; off = align_up(off + R * (nprobe + 1) * 4);
+  L.off_ncand = off;   off = align_up(off + R * 4);
+  L.off_idxc = off;    off = align_up(off + R * std::max(k, 1) * 4);
+  L.total = off;
+  return true;
+}
+
+size_t ra_ivf_search_workspace_bytes(int32_t B, int32_t Hq, int64_t N, int32_t d, int32_t k,
+                                     int32_t nprobe) {
+  IvfSearchLayout L{};
+  return ivf_search_layout(B, Hq, N, d, k, nprobe, L) ? L.total : 0;
+}
+
+ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, int32_t Hq,
+                             int32_t k, int32_t nprobe, int32_t n_sink, int32_t n_window,
+                             float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                             ra_stream_t stream) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (!ix || !ix->Ksorted || !ix->pos || !ix->offsets || !ix->centroids) return RA_ERR_ARG;
+  if (ix->B != kv->B || ix->Hkv != kv->Hkv || ix->d != kv->d) return RA_ERR_SHAPE;
+  if (nprobe < 1 || nprobe > 64 || nprobe > ix->nlist || ix->nlist > 4096) return RA_ERR_ARG;
+  if (ix->N < 1 || ix->N > kv->N || kv->N - ix->N > n_window) return RA_ERR_ARG;
+  Step dec{};   // the step's own geometry (W, C, the attention)
+  s = plan_step(kv, Hq, k, n_sink, n_window, ws, ws_bytes, dec);
+  if (s != RA_OK && s != RA_ERR_WORKSPACE) return s;
+  IvfSearchLayout L{};
+  if (!ivf_search_layout(kv->B, Hq, kv->N, kv->d, k, nprobe, L)) return RA_ERR_SHAPE;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < L.total)
+    return RA_ERR_WORKSPACE;
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  plan_clusters(dec);
+  plan_clusters(L.st);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  IvfSearchParams v{};
+  v.q = static_cast<const __nv_bfloat16 *>(q);
+  v.K = static_cast<const __nv_bfloat16 *>(kv->K);
+  v.Ksorted = static_cast<const __nv_bfloat16 *>(ix->Ksorted);
+  v.cent = static_cast<const __nv_bfloat16 *>(ix->centroids);
+  v.pos = ix->pos;
+  v.offsets = ix->offsets;
+  v.probe = reinterpret_cast<int32_t *>(at(ws, L.off_probe));
+  v.cand_off = reinterpret_cast<int32_t *>(at(ws, L.off_candoff));
+  v.n_cand = reinterpret_cast<int32_t *>(at(ws, L.off_ncand));
+  v.S = reinterpret_cast<float *>(at(ws, L.off_Sfull));
+  v.S_cand = reinterpret_cast<float *>(at(ws, L.st.off_S));
+  v.pos_cand = reinterpret_cast<int32_t *>(at(ws, L.off_poscand));
+  int32_t *idx_cand = reinterpret_cast<int32_t *>(at(ws, L.off_idxc));
+  v.idx_cand = idx_cand;
+  v.idx = idx;
+  v.N = ix->N; v.cap = kv->cap; v.ldS = L.st.ldS; v.ldC = L.st.ldS;
+  v.s1 = dec.s1; v.w0 = dec.w0; v.nW = dec.nW;
+  v.R = dec.R; v.Hq = Hq; v.Hkv = kv->Hkv; v.G = Hq / kv->Hkv; v.d = kv->d;
+  v.nlist = ix->nlist; v.nprobe = nprobe; v.k = k;
+  v.scale = 1.0f / sqrtf(static_cast<float>(kv->d));
+  cudaError_t e = launch_ivf_probe(v, cs);
+  if (e == cudaSuccess) e = launch_ivf_cand(v, kv->d, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "ivf_search");
+  if (k > 0) {   // exact top-k of each row's candidates, then their cache positions
+    SaParams p{};
+    p.S = v.S_cand;
+    p.hist = reinterpret_cast<uint32_t *>(at(ws, L.st.off_hist));
+    p.list = reinterpret_cast<uint2 *>(at(ws, L.st.off_list));
+    p.idx = idx_cand;
+    p.part = reinterpret_cast<float *>(at(ws, L.st.off_part));
+    p.meta = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta));
+    p.err = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta)) + kError;
+    p.ldS = L.st.ldS; p.ldL = L.st.ldL; p.N = L.st.N;
+    p.k = k; p.Hq = Hq; p.G = v.G; p.Hkv = kv->Hkv;
+    p.mode = kSaSelect | kSaBuildHist;
+    p.nsplit = 1;
+    p.row_n = v.n_cand;
+    e = launch_select_attend(p, kv->d, L.st.R, L.st.ncl, cs);
+    if (e == cudaSuccess) e = launch_ivf_map(v, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "ivf_select");
+  }
+  // softmax attention over W u Omega from the full-length score rows
+  SaParams a{};
+  a.S = v.S;
+  a.V = static_cast<const __nv_bfloat16 *>(kv->V);
+  a.idx = idx;
+  a.out = out;
+  a.part = reinterpret_cast<float *>(at(ws, L.st.off_part));
+  a.meta = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta));
+  a.err = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta)) + kError;
+  a.ldS = L.st.ldS; a.cap = kv->cap; a.N = dec.N;
+  a.s1 = dec.s1; a.w0 = dec.w0; a.nW = dec.nW; a.nC = dec.nC; a.k_eff = dec.k_eff;
+  a.cbase = dec.cbase; a.cper = dec.cper;
+  a.k = k; a.Hq = Hq; a.G = dec.G; a.Hkv = dec.Hkv;
+  a.mode = kSaAttend;
+  a.nsplit = attn_split(dec.nW + dec.k_eff, dec.R, dec.ncl, dec.d);
+  e = launch_select_attend(a, kv->d, dec.R, dec.ncl, cs);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "ivf_attend");
+}
+
 }  // extern "C"

@@ -450,7 +450,19 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
 struct RowGeo {
   long long N, s1, w0, nW, nC, k_eff, cbase, cper;
 };
-__device__ __forceinline__ RowGeo row_geo(const SaParams &p, const NoPaging &, int, int) {
+__device__ __forceinline__ RowGeo row_geo(const SaParams &p, const NoPaging &, int row, int ncl) {
+  if (p.row_n) {   // a candidate list of its own length, no static set
+    RowGeo g;
+    g.N = p.row_n[row];
+    g.s1 = 0;
+    g.w0 = g.N;
+    g.nW = 0;
+    g.nC = g.N;
+    g.k_eff = min(static_cast<long long>(p.k), g.N);
+    g.cbase = 0;
+    g.cper = ((max(g.N, 1LL) + ncl - 1) / ncl + 3) / 4 * 4;
+    return g;
+  }
   return RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, p.k_eff, p.cbase, p.cper};
 }
 __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const PagedInfo &pg, int row, int ncl) {

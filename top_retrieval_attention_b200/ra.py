@@ -23,7 +23,9 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_sparse_attn", "ra_select_attend", "ra_dense_workspace_bytes", "ra_dense_decode",
            "ra_decode_step_static", "ra_prefill_workspace_bytes", "ra_prefill_topk",
            "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets",
-           "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step")
+           "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step",
+           "ra_ivf_build_workspace_bytes", "ra_ivf_build", "ra_ivf_search_workspace_bytes",
+           "ra_ivf_decode_step")
 
 
 class ra_kv(ctypes.Structure):
@@ -35,6 +37,12 @@ class ra_paged_kv(ctypes.Structure):
     _fields_ = [("K", c_void_p), ("V", c_void_p), ("block_table", c_void_p),
                 ("seq_len", ctypes.POINTER(c_int32)), ("B", c_int32), ("Hkv", c_int32),
                 ("d", c_int32), ("max_pages", c_int32), ("num_pages", c_int32)]
+
+
+class ra_ivf(ctypes.Structure):
+    _fields_ = [("Ksorted", c_void_p), ("pos", c_void_p), ("offsets", c_void_p),
+                ("centroids", c_void_p), ("B", c_int32), ("Hkv", c_int32), ("d", c_int32),
+                ("nlist", c_int32), ("N", c_int64)]
 
 
 _lib = None
@@ -75,6 +83,14 @@ def lib() -> ctypes.CDLL:
             "ra_paged_decode_step": (c_int32, [ctypes.POINTER(ra_paged_kv), c_void_p, c_int32, c_int32,
                                                c_int32, c_int32, c_void_p, c_void_p, c_void_p,
                                                c_size_t, c_void_p]),
+            "ra_ivf_build_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32, c_int32]),
+            "ra_ivf_build": (c_int32, [P, ctypes.POINTER(ra_ivf), c_int32, c_void_p, c_size_t,
+                                       c_void_p]),
+            "ra_ivf_search_workspace_bytes": (c_size_t, [c_int32, c_int32, c_int64, c_int32,
+                                                         c_int32, c_int32]),
+            "ra_ivf_decode_step": (c_int32, [P, ctypes.POINTER(ra_ivf), c_void_p, c_int32, c_int32,
+                                             c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                             c_void_p, c_size_t, c_void_p]),
             "ra_pyramid_budgets": (c_int32, [c_int32, c_int32, ctypes.c_double,
                                              ctypes.POINTER(c_int32)]),
             "ra_decode_step_eps": (c_int32, [P, c_void_p, c_int32, c_int32, ctypes.c_float, c_int32,
@@ -361,6 +377,58 @@ def paged_decode_step(cache: PagedKVCache, q, k: int, n_sink: int, n_window: int
     check(lib().ra_paged_decode_step(ctypes.byref(cache.kv), q.data_ptr(), Hq, k, n_sink, n_window,
                                      out.data_ptr(), idx.data_ptr(), ws.data_ptr(), ws.numel(),
                                      _stream(stream)), "ra_paged_decode_step")
+    return out, idx[..., :k]
+
+
+class IvfIndex:
+    """An IVF index of a layer cache's first N keys: torch-allocated sorted keys, positions,
+    offsets and centroids; `ix` is the C struct over them."""
+
+    def __init__(self, cache: KVCache, nlist: int, N: int | None = None):
+        import torch
+        self.N = cache.N if N is None else N
+        dev = cache.K.device
+        B, Hkv, d = cache.B, cache.Hkv, cache.d
+        self.nlist = nlist
+        self.Ksorted = torch.empty((B, Hkv, self.N, d), dtype=torch.bfloat16, device=dev)
+        self.pos = torch.empty((B, Hkv, self.N), dtype=torch.int32, device=dev)
+        self.offsets = torch.empty((B, Hkv, nlist + 1), dtype=torch.int32, device=dev)
+        self.centroids = torch.empty((B, Hkv, nlist, d), dtype=torch.bfloat16, device=dev)
+        self.ix = ra_ivf(self.Ksorted.data_ptr(), self.pos.data_ptr(), self.offsets.data_ptr(),
+                         self.centroids.data_ptr(), B, Hkv, d, nlist, self.N)
+
+
+def ivf_build(cache: KVCache, nlist: int, iters: int = 4, N: int | None = None, stream=None):
+    """Spherical k-means IVF index of the cache's first N keys (all by default)."""
+    import torch
+    ix = IvfIndex(cache, nlist, N)
+    n = lib().ra_ivf_build_workspace_bytes(cache.B, cache.Hkv, ix.N, cache.d, nlist)
+    if n == 0:
+        raise RaError(RA_ERR_SHAPE, "ra_ivf_build_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=cache.K.device)
+    check(lib().ra_ivf_build(ctypes.byref(cache.kv), ctypes.byref(ix.ix), iters, ws.data_ptr(), n,
+                             _stream(stream)), "ra_ivf_build")
+    return ix
+
+
+def ivf_decode_step(cache: KVCache, ix: IvfIndex, q, k: int, nprobe: int, n_sink: int,
+                    n_window: int, out=None, idx=None, ws=None, stream=None):
+    """Decode step retrieving through the IVF index.  Returns (out fp32, idx int32)."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        n = lib().ra_ivf_search_workspace_bytes(B, Hq, cache.N, d, k, nprobe)
+        if n == 0:
+            raise RaError(RA_ERR_SHAPE, "ra_ivf_search_workspace_bytes")
+        ws = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    check(lib().ra_ivf_decode_step(ctypes.byref(cache.kv), ctypes.byref(ix.ix), q.data_ptr(), Hq, k,
+                                   nprobe, n_sink, n_window, out.data_ptr(), idx.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), _stream(stream)),
+          "ra_ivf_decode_step")
     return out, idx[..., :k]
 
 
