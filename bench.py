@@ -74,6 +74,11 @@ def parse():
     ap.add_argument("--paged", action="store_true",
                     help="paged cache (128-token pages, shuffled) with ragged lengths falling "
                          "linearly from N to N/2 over the batch (ra_paged_decode_step)")
+    ap.add_argument("--ivf", type=int, default=0, metavar="NLIST",
+                    help="decode through a device-built IVF index of NLIST clusters per KV head "
+                         "(one layer); reports Recall@k against the exact top-k")
+    ap.add_argument("--nprobe", type=int, default=32, help="IVF clusters probed per query head")
+    ap.add_argument("--ivf-iters", type=int, default=4, help="k-means iterations of the IVF build")
     ap.add_argument("--prefill-queries", type=int, default=0,
                     help="instead of decode steps: exact top-k of this many prefill queries per "
                          "query head (tensor-core scores + cluster selection), one layer")
@@ -658,6 +663,152 @@ def run_paged(args, w, rank, local_rank, world, dist):
     }
 
 
+def run_ivf(args, w, rank, local_rank, world, dist):
+    """Decode steps retrieving through an IVF index of the keys built on the device (spherical
+    k-means, `--ivf` clusters per KV head, `--nprobe` probed per query head), one layer of the
+    workload.  The index covers the N - 1 cached keys; each step appends the N-th token (served by
+    the window) and decodes.  Beside the throughput: the build time, the fraction of candidate
+    keys scored, and Recall@k of the IVF selection against the exact top-k of the same step."""
+    import ctypes
+
+    import torch
+
+    import top_retrieval_attention_b200 as ra
+    from synth import device as sdev
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    B, Hq, Hkv, d, N, k, G = w.B, w.Hq, w.Hkv, w.d, w.N, w.k, w.G
+    nlist, nprobe = args.ivf, args.nprobe
+    c = ra.KVCache(B, Hkv, d, N, device=dev)
+    sdev.device_layer(w, 0, c.K, c.V)
+    knew = c.K[:, :, N - 1:N].clone()
+    vnew = c.V[:, :, N - 1:N].clone()
+    c.N = N - 1
+    P = 16
+    qpool = torch.empty((P, B, Hq, d), dtype=torch.bfloat16, device=dev)
+    for s in range(P):
+        sdev.fill_q(qpool[s], w.seed + 7919 * s)
+
+    # the build: once untimed (kernel loading), then timed with events
+    ix = ra.ivf_build(c, nlist, args.ivf_iters)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    ix = ra.ivf_build(c, nlist, args.ivf_iters)
+    b.record(stream)
+    torch.cuda.synchronize()
+    build_ms = a.elapsed_time(b)
+
+    n = ra.lib().ra_ivf_search_workspace_bytes(B, Hq, N, d, k, nprobe)
+    if n == 0:
+        raise SystemExit(f"IVF search shape rejected (nprobe {nprobe}, nlist {nlist})")
+    ws = torch.zeros(n, dtype=torch.uint8, device=dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=dev)
+
+    def step(s):
+        ra.check(ra.ra_append_kv(c.kv, knew.data_ptr(), vnew.data_ptr(), 1, sp), "append")
+        ra.check(ra.lib().ra_ivf_decode_step(ctypes.byref(c.kv), ctypes.byref(ix.ix),
+                                             qpool[s % P].data_ptr(), Hq, k, nprobe, w.n_sink,
+                                             w.n_window, out.data_ptr(), idx.data_ptr(),
+                                             ws.data_ptr(), n, sp), "ivf_decode")
+        c.N = N - 1
+
+    # quality: Recall@k of every query of the pool against the exact step's selection, and the
+    # keys each query head scores (its probed clusters' sizes; diagnostic arithmetic in torch)
+    ews = torch.zeros(ra.ra_decode_workspace_bytes(B, Hq, N, d, k, w.n_sink, w.n_window),
+                      dtype=torch.uint8, device=dev)
+    hits = total = 0
+    scanned = []
+    sizes = (ix.offsets[..., 1:] - ix.offsets[..., :-1]).float()            # [B, Hkv, nlist]
+    for s in range(P):
+        step(s)
+        ra.check(ra.ra_append_kv(c.kv, knew.data_ptr(), vnew.data_ptr(), 1, sp), "append")
+        _, ex = ra.decode_step(c, qpool[s], k, w.n_sink, w.n_window, ws=ews)
+        c.N = N - 1
+        got = idx[..., :k]
+        for bb in range(B):
+            for h in range(Hq):
+                e = ex[bb, h][ex[bb, h] >= 0]
+                hits += int(torch.isin(e, got[bb, h]).sum().item())
+                total += int(e.numel())
+        zc = torch.einsum("bgcd,bghd->bghc", ix.centroids.float(),
+                          qpool[s].float().view(B, Hkv, G, d))
+        top = zc.topk(nprobe, dim=-1).indices                                # [B, Hkv, G, nprobe]
+        sz = torch.gather(sizes.unsqueeze(2).expand(B, Hkv, G, nlist), 3, top).sum(-1)
+        scanned.append(sz.mean().item())
+    torch.cuda.synchronize()
+    recall = hits / max(total, 1)
+    cand_per_head = statistics.mean(scanned)
+
+    for s in range(max(3, args.warmup)):
+        step(s)
+    torch.cuda.synchronize()
+    steps = args.steps if args.steps is not None else 1000
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    clk = Clocks(uuid)
+    clk.start()
+    barrier(dist, local_rank)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(steps):
+        step(s)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, local_rank)
+    clocks = clk.stop()
+    ms = max_over_ranks(dist, t0.elapsed_time(t1), dev) / steps
+
+    # the exact step on the same cache, for the speedup
+    for s in range(5):
+        ra.check(ra.ra_append_kv(c.kv, knew.data_ptr(), vnew.data_ptr(), 1, sp), "append")
+        ra.decode_step(c, qpool[s % P], k, w.n_sink, w.n_window, ws=ews)
+        c.N = N - 1
+    a.record(stream)
+    for s in range(steps):
+        ra.check(ra.ra_append_kv(c.kv, knew.data_ptr(), vnew.data_ptr(), 1, sp), "append")
+        ra.decode_step(c, qpool[s % P], k, w.n_sink, w.n_window, ws=ews)
+        c.N = N - 1
+    b.record(stream)
+    torch.cuda.synchronize()
+    exact_ms = max_over_ranks(dist, a.elapsed_time(b), dev) / steps
+
+    # algorithmic bytes per step, per query head: the centroids, the probed clusters' keys, the
+    # static set's keys, and the V rows of U
+    s1 = min(w.n_sink, N)
+    w0 = max(s1, N - w.n_window)
+    n_w = s1 + (N - w0)
+    row = 2 * d
+    alg = B * Hq * (nlist * row + cand_per_head * row + n_w * row + (n_w + min(k, w0 - s1)) * row)
+    peak, peak_kind = measured_hbm_peak()
+    gbs = alg / (ms / 1000.0) / 1e9
+    return {
+        "metric": "IVF-retrieval decode steps/s (device-built index, probed top-k)",
+        "value": world * 1000.0 / ms, "unit": "steps/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 / Irwin-Hall normals, Llama-3-8B-shaped cache)",
+        "config": dict(workload_config(w), layers=1, nlist=nlist, nprobe=nprobe,
+                       kmeans_iters=args.ivf_iters),
+        "roofline": {"kernel": "IVF decode step (probe + candidate scores + select + attend)",
+                     "bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": alg},
+        "recall_at_k": recall, "scanned_fraction": cand_per_head / N,
+        "candidates_per_query_head": cand_per_head, "build_ms": build_ms,
+        "exact_step_ms": exact_ms, "speedup_over_exact": exact_ms / ms,
+        "gpu_launches": 6 * steps, "clocks": clocks,
+    }
+
+
 def run_prefill(args, w, rank, local_rank, world, dist):
     """Exact top-k of M prefill queries per query head against one layer's cache: the
     tcgen05 score GEMM (timed on its own for its roofline) and the cluster selection."""
@@ -767,6 +918,8 @@ def main():
     try:
         if args.prefill_queries > 0:
             res = run_prefill(args, w, rank, local_rank, world, dist)
+        elif args.ivf > 0:
+            res = run_ivf(args, w, rank, local_rank, world, dist)
         elif args.paged:
             res = run_paged(args, w, rank, local_rank, world, dist)
         else:
