@@ -295,10 +295,15 @@ ra_status ra_ivf_build(const ra_kv *kv, ra_ivf *ix, int32_t iters, void *ws, siz
 
 /*
  * A decode step that retrieves through the index: per query head, the nprobe clusters whose
- * centroids score highest, the exact top-k of their keys outside W (ties to the lower position),
- * and softmax attention over W u Omega as ra_decode_step.  Keys appended after the build are
- * only attended through the window: kv->N - ix->N <= n_window is required.
- *   nprobe : 1 <= nprobe <= min(nlist, 64).   idx : -1 past the keys retrieved.
+ * centroids score highest (ties to the lower cluster), the exact top-k of their keys outside W,
+ * and softmax attention over W u Omega as ra_decode_step.  Keys of equal score are taken in
+ * candidate order (probe order, then the order inside a cluster), not by position.  Keys
+ * appended after the build are only attended through the window: kv->N - ix->N <= n_window is
+ * required.  Three launches: the centroid probe, the candidate scores, and the selection fused
+ * with the attention (a fourth when the attention is split across several clusters per head).
+ *   nprobe : 1 <= nprobe <= min(nlist, 64).
+ *   idx    : int32 [B, Hq, k], cache positions; -1 in slots that retrieve nothing (when the
+ *            probed clusters hold fewer than k keys outside W).
  *   ws     : at least ra_ivf_search_workspace_bytes(...) bytes, 256-byte aligned, zero-filled
  *            once (it holds a decode workspace's counter block).
  * Errors: as ra_decode_step; RA_ERR_ARG for nprobe or an index that does not cover the cache.

@@ -10,10 +10,10 @@
 // normalised into the next centroids.  A final assignment, a count per cluster, an exclusive
 // scan and a scatter give the keys sorted by cluster (with their positions) and the cluster
 // offsets.
-// Search, per query head: the scores of the nlist centroids, the nprobe best (bitonic sort of
-// (order key, id) in shared memory), the exact scores of every key of the probed clusters
-// (read contiguously from the sorted copy; static-set positions excluded) and of the static
-// set; the cluster kernel then selects the exact top-k of the probed candidates and attends.
+// Search, per query head: the scores of the nlist centroids and the nprobe best, the exact
+// scores of every key of the probed clusters (read contiguously from the sorted copy; static-set
+// positions excluded) and of the static set; the cluster kernel then selects the exact top-k of
+// the probed candidates (reporting their cache positions) and attends over W and Omega.
 #include <math.h>
 
 #include <algorithm>
@@ -169,131 +169,263 @@ __global__ void __launch_bounds__(256) ivf_scatter_kernel(const IvfParams p) {
 
 // ---- search
 
-constexpr int kIvfMaxList = 4096;   // clusters per head at most (the probe sorts them in smem)
+constexpr int kIvfMaxList = 4096;    // clusters per head at most
+constexpr int kProbeThreads = 512;
+constexpr int kProbeCollect = 512;   // keys at or above the threshold bin ranked directly
 
-// One CTA per query head row: centroid scores, the nprobe best clusters, their candidate offsets.
-__global__ void __launch_bounds__(256) ivf_probe_kernel(const IvfSearchParams p) {
+// Exclusive prefix (from thread 0 up) of one value per thread of a kProbeThreads block, and the
+// block total.  wsum holds kProbeThreads / 32 words.
+__device__ __forceinline__ uint32_t probe_scan(uint32_t v, uint32_t *wsum, uint32_t &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  uint32_t before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kProbeThreads / 32; ++w) {
+    const uint32_t t = wsum[w];
+    before += w < warp ? t : 0u;
+    total += t;
+  }
+  __syncthreads();
+  return before + x - v;
+}
+
+// One CTA per query head row: the scores of its KV head's nlist centroids, the nprobe best
+// (largest score first, ties to the lower cluster), their clusters' offsets in the row's
+// candidate list.  The selection: an 11-bit histogram of the score keys gives the bin of the
+// nprobe-th largest; the keys at or above it are gathered and each is ranked by counting the
+// gathered keys above it.  Should that bin hold more keys than the gather takes, every key is
+// sorted instead (bitonic, in shared memory).
+__global__ void __launch_bounds__(kProbeThreads) ivf_probe_kernel(const IvfSearchParams p) {
   __shared__ unsigned long long keys[kIvfMaxList];
+  __shared__ unsigned long long coll[kProbeCollect];
+  __shared__ uint32_t hist[kHistBins];
   __shared__ float qs[128];
+  __shared__ int32_t sel[64];
+  __shared__ uint32_t wsum[kProbeThreads / 32];
+  __shared__ int t_bin;
+  __shared__ uint32_t n_coll;
   const int row = blockIdx.x, tid = threadIdx.x;
   const int b = row / p.Hq, h = row - b * p.Hq;
   const long long bg = static_cast<long long>(b) * p.Hkv + h / p.G;
+  pdl_trigger();
+  pdl_wait();   // the query and the cache may come from earlier kernels of the stream
   if (tid < p.d) qs[tid] = __bfloat162float(p.q[static_cast<long long>(row) * p.d + tid]);
-  int np2 = 1;
-  while (np2 < p.nlist) np2 <<= 1;
-  __syncthreads();
-  for (int c = tid; c < np2; c += 256) {
-    unsigned long long key = 0ull;   // below every real key
-    if (c < p.nlist) {
-      const __nv_bfloat16 *cent = p.cent + (bg * p.nlist + c) * p.d;
-      float z = 0.f;
-      for (int j = 0; j < p.d; j += 2) {
-        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(cent + j);
-        z += qs[j] * __low2float(v) + qs[j + 1] * __high2float(v);
-      }
-      key = (static_cast<unsigned long long>(order_key(canon_zero(z))) << 32) |
-            (0xFFFFFFFFu - static_cast<uint32_t>(c));
-    }
-    keys[c] = key;
-  }
-  __syncthreads();
-  // bitonic sort, descending
-  for (int size = 2; size <= np2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < np2 / 2; i += 256) {
-        const int lo = 2 * stride * (i / stride) + (i % stride);
-        const int hi = lo + stride;
-        const unsigned long long a = keys[lo], bb = keys[hi];
-        const bool desc = (lo & size) == 0;
-        if (desc ? (a < bb) : (a > bb)) {
-          keys[lo] = bb;
-          keys[hi] = a;
-        }
-      }
-      __syncthreads();
-    }
-  }
+  for (int i = tid; i < kHistBins; i += kProbeThreads) hist[i] = 0u;
+  if (tid < 64) sel[tid] = 0;   // a valid cluster in every slot whatever happens below
   if (tid == 0) {
+    t_bin = -1;
+    n_coll = 0u;
+  }
+  __syncthreads();
+  // a thread per centroid, its row read in 16-byte pieces
+  for (int c = tid; c < p.nlist; c += kProbeThreads) {
+    const uint4 *cr = reinterpret_cast<const uint4 *>(p.cent + (bg * p.nlist + c) * p.d);
+    float z = 0.f;
+    for (int j = 0; j < p.d / 8; ++j) {
+      const uint4 v = __ldg(cr + j);
+      const float *qq = qs + 8 * j;
+      z += qq[0] * bf16_lo(v.x) + qq[1] * bf16_hi(v.x) + qq[2] * bf16_lo(v.y) +
+           qq[3] * bf16_hi(v.y) + qq[4] * bf16_lo(v.z) + qq[5] * bf16_hi(v.z) +
+           qq[6] * bf16_lo(v.w) + qq[7] * bf16_hi(v.w);
+    }
+    const uint32_t okey = order_key(canon_zero(z));
+    keys[c] = (static_cast<unsigned long long>(okey) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(c));
+    atomicAdd(&hist[okey >> (32 - kHistBits)], 1u);
+  }
+  __syncthreads();
+  // the bin of the nprobe-th largest key: thread t owns bins [2048 - 4 (t + 1), 2048 - 4 t)
+  {
+    constexpr int per = kHistBins / kProbeThreads;
+    uint32_t loc[per], s = 0;
+#pragma unroll
+    for (int i = 0; i < per; ++i) {
+      loc[i] = hist[kHistBins - per * (tid + 1) + (per - 1 - i)];
+      s += loc[i];
+    }
+    uint32_t total;
+    const uint32_t before = probe_scan(s, wsum, total);
+    const uint32_t want = static_cast<uint32_t>(p.nprobe);
+    if (before < want && want <= before + s) {
+      uint32_t cum = before;
+#pragma unroll
+      for (int i = 0; i < per; ++i) {
+        if (cum + loc[i] >= want) {
+          t_bin = kHistBins - per * (tid + 1) + (per - 1 - i);
+          break;
+        }
+        cum += loc[i];
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t tb = static_cast<uint32_t>(t_bin);   // found: nprobe <= nlist keys exist
+  for (int c = tid; c < p.nlist; c += kProbeThreads) {
+    const unsigned long long x = keys[c];
+    if (static_cast<uint32_t>(x >> (64 - kHistBits)) >= tb) {
+      const uint32_t slot = atomicAdd(&n_coll, 1u);
+      if (slot < static_cast<uint32_t>(kProbeCollect)) coll[slot] = x;
+    }
+  }
+  __syncthreads();
+  const uint32_t m = n_coll;
+  if (m <= static_cast<uint32_t>(kProbeCollect)) {
+    for (uint32_t i = tid; i < m; i += kProbeThreads) {
+      const unsigned long long x = coll[i];
+      uint32_t r = 0;
+      for (uint32_t j = 0; j < m; ++j) r += coll[j] > x ? 1u : 0u;
+      if (r < static_cast<uint32_t>(p.nprobe))
+        sel[r] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(x));
+    }
+  } else {   // a crowded bin: sort all keys, descending
+    int np2 = 1;
+    while (np2 < p.nlist) np2 <<= 1;
+    for (int c = p.nlist + tid; c < np2; c += kProbeThreads) keys[c] = 0ull;   // below every key
+    __syncthreads();
+    for (int size = 2; size <= np2; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < np2 / 2; i += kProbeThreads) {
+          const int lo = 2 * stride * (i / stride) + (i % stride);
+          const int hi = lo + stride;
+          const unsigned long long a = keys[lo], bb = keys[hi];
+          const bool desc = (lo & size) == 0;
+          if (desc ? (a < bb) : (a > bb)) {
+            keys[lo] = bb;
+            keys[hi] = a;
+          }
+        }
+        __syncthreads();
+      }
+    }
+    if (tid < p.nprobe) sel[tid] = static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(keys[tid]));
+  }
+  __syncthreads();
+  // the probed clusters' sizes -> offsets in the candidate list (lane l: slots 2l and 2l + 1)
+  if (tid < 32) {
+    const int32_t *offs = p.offsets + bg * (p.nlist + 1);
+    const int j0 = 2 * tid, j1 = j0 + 1;
+    const int32_t s0 = j0 < p.nprobe ? offs[sel[j0] + 1] - offs[sel[j0]] : 0;
+    const int32_t s1 = j1 < p.nprobe ? offs[sel[j1] + 1] - offs[sel[j1]] : 0;
+    int32_t x = s0 + s1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (tid >= o) x += y;
+    }
+    const int32_t excl = x - s0 - s1;
+    const int32_t total = __shfl_sync(0xffffffffu, x, 31);
     int32_t *probe = p.probe + static_cast<long long>(row) * p.nprobe;
     int32_t *off = p.cand_off + static_cast<long long>(row) * (p.nprobe + 1);
-    const int32_t *offs = p.offsets + bg * (p.nlist + 1);
-    int32_t acc = 0;
-    for (int j = 0; j < p.nprobe; ++j) {
-      const int c = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(keys[j]));
-      probe[j] = c;
-      off[j] = acc;
-      acc += offs[c + 1] - offs[c];
+    if (j0 < p.nprobe) {
+      probe[j0] = sel[j0];
+      off[j0] = excl;
     }
-    off[p.nprobe] = acc;
-    p.n_cand[row] = acc;
+    if (j1 < p.nprobe) {
+      probe[j1] = sel[j1];
+      off[j1] = excl + s0;
+    }
+    if (tid == 0) {
+      off[p.nprobe] = total;
+      p.n_cand[row] = total;
+    }
   }
 }
 
-// Exact scores of the probed candidates (into S_cand, positions into pos_cand, and into the
-// row's full score row at their positions) and of the static set (full score row).  Static-set
-// positions among the candidates get -inf in S_cand (W is attended anyway).  One warp per key.
+// Exact scores of the probed candidates (into S_cand, the candidate -> cache position map into
+// pos_cand, and into the row's full score row at their positions) and of the static set (full
+// score row).  Static-set keys among the candidates get -inf in S_cand and -1 in pos_cand (W is
+// attended anyway).  Four lanes per key, each with a quarter of the channels in 16-byte loads;
+// a warp scores eight keys at a time.
 template <int D>
 __global__ void __launch_bounds__(256) ivf_cand_kernel(const IvfSearchParams p) {
-  constexpr int CPL = D / 32;
-  const int row = blockIdx.y, lane = threadIdx.x & 31;
+  constexpr int CPG = D / 4;    // channels per lane
+  constexpr int NV = CPG / 8;   // 16-byte loads per lane
+  __shared__ long long sbase[64];
+  __shared__ int32_t soff[65];
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane & 3, gi = lane >> 2;
   const int b = row / p.Hq, h = row - b * p.Hq;
   const long long bg = static_cast<long long>(b) * p.Hkv + h / p.G;
-  float qv[CPL];
+  pdl_trigger();
+  pdl_wait();   // the probe's lists (and, before it, the appended keys)
+  if (tid <= p.nprobe) {
+    soff[tid] = p.cand_off[static_cast<long long>(row) * (p.nprobe + 1) + tid];
+    if (tid < p.nprobe) {
+      const int c = p.probe[static_cast<long long>(row) * p.nprobe + tid];
+      sbase[tid] = bg * p.N + p.offsets[bg * (p.nlist + 1) + c];
+    }
+  }
+  float qv[CPG];
+  {
+    const uint4 *qr = reinterpret_cast<const uint4 *>(p.q + static_cast<long long>(row) * D + sub * CPG);
 #pragma unroll
-  for (int c = 0; c < CPL; ++c)
-    qv[c] = __bfloat162float(p.q[static_cast<long long>(row) * D + lane * CPL + c]);
-  const int32_t *off = p.cand_off + static_cast<long long>(row) * (p.nprobe + 1);
-  const int32_t *probe = p.probe + static_cast<long long>(row) * p.nprobe;
-  const int32_t *offs = p.offsets + bg * (p.nlist + 1);
-  const long long n_cand = off[p.nprobe];
+    for (int v = 0; v < NV; ++v) {
+      const uint4 w = __ldg(qr + v);
+      qv[8 * v + 0] = bf16_lo(w.x); qv[8 * v + 1] = bf16_hi(w.x);
+      qv[8 * v + 2] = bf16_lo(w.y); qv[8 * v + 3] = bf16_hi(w.y);
+      qv[8 * v + 4] = bf16_lo(w.z); qv[8 * v + 5] = bf16_hi(w.z);
+      qv[8 * v + 6] = bf16_lo(w.w); qv[8 * v + 7] = bf16_hi(w.w);
+    }
+  }
+  __syncthreads();
+  const long long n_cand = soff[p.nprobe];
   const long long total = n_cand + p.nW;
   float *srow = p.S + static_cast<long long>(row) * p.ldS;
-  const long long warps = static_cast<long long>(gridDim.x) * 8;
-  for (long long e = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); e < total; e += warps) {
-    const __nv_bfloat16 *krow;
-    long long pos;
-    if (e < n_cand) {
-      int j = 0;   // the probe slot holding candidate e
-      while (j + 1 < p.nprobe && off[j + 1] <= e) ++j;
-      const long long si = bg * p.N + offs[probe[j]] + (e - off[j]);
-      pos = p.pos[si];
-      krow = p.Ksorted + si * D;
-    } else {
-      const long long wi = e - n_cand;
-      pos = wi < p.s1 ? wi : p.w0 + (wi - p.s1);
-      krow = p.K + (bg * p.cap + pos) * D;
+  const long long step = static_cast<long long>(gridDim.x) * 64;
+  for (long long e0 = (static_cast<long long>(blockIdx.x) * 8 + warp) * 8; e0 < total; e0 += step) {
+    const long long e = e0 + gi;
+    const bool valid = e < total;
+    const __nv_bfloat16 *krow = nullptr;
+    long long si = -1, pos = 0;
+    if (valid) {
+      if (e < n_cand) {
+        int lo = 0, hi = p.nprobe - 1;   // the last probe slot starting at or before e
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (soff[mid] <= e) lo = mid;
+          else hi = mid - 1;
+        }
+        si = sbase[lo] + (e - soff[lo]);
+        krow = p.Ksorted + si * D;
+      } else {
+        const long long wi = e - n_cand;
+        pos = wi < p.s1 ? wi : p.w0 + (wi - p.s1);
+        krow = p.K + (bg * p.cap + pos) * D;
+      }
     }
     float z = 0.f;
-    if constexpr (CPL == 4) {
-      const uint2 v = *reinterpret_cast<const uint2 *>(krow + lane * 4);
-      z = qv[0] * bf16_lo(v.x) + qv[1] * bf16_hi(v.x) + qv[2] * bf16_lo(v.y) + qv[3] * bf16_hi(v.y);
-    } else {
-      const uint32_t v = *reinterpret_cast<const uint32_t *>(krow + lane * 2);
-      z = qv[0] * bf16_lo(v) + qv[1] * bf16_hi(v);
+    if (valid) {
+      const uint4 *kr = reinterpret_cast<const uint4 *>(krow + sub * CPG);
+      uint4 kv[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) kv[v] = __ldg(kr + v);
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        z += qv[8 * v + 0] * bf16_lo(kv[v].x) + qv[8 * v + 1] * bf16_hi(kv[v].x) +
+             qv[8 * v + 2] * bf16_lo(kv[v].y) + qv[8 * v + 3] * bf16_hi(kv[v].y) +
+             qv[8 * v + 4] * bf16_lo(kv[v].z) + qv[8 * v + 5] * bf16_hi(kv[v].z) +
+             qv[8 * v + 6] * bf16_lo(kv[v].w) + qv[8 * v + 7] * bf16_hi(kv[v].w);
+      }
     }
-    z = canon_zero(warp_sum(z) * p.scale);
-    if (lane == 0) {
+    z += __shfl_xor_sync(0xffffffffu, z, 1);
+    z += __shfl_xor_sync(0xffffffffu, z, 2);
+    if (valid && sub == 0) {
+      z = canon_zero(z * p.scale);
+      if (si >= 0) pos = p.pos[si];
       srow[pos] = z;
       if (e < n_cand) {
         const bool in_w = pos < p.s1 || pos >= p.w0;
         p.S_cand[static_cast<long long>(row) * p.ldC + e] = in_w ? -INFINITY : z;
-        p.pos_cand[static_cast<long long>(row) * p.ldC + e] = static_cast<int32_t>(pos);
+        p.pos_cand[static_cast<long long>(row) * p.ldC + e] = in_w ? -1 : static_cast<int32_t>(pos);
       }
     }
-  }
-}
-
-// Candidate indices chosen by the selection -> cache positions (-1 for none or a W key).
-__global__ void __launch_bounds__(256) ivf_map_kernel(const IvfSearchParams p) {
-  const long long n = static_cast<long long>(p.R) * p.k;
-  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256) {
-    const long long row = i / p.k;
-    const int32_t e = p.idx_cand[i];
-    int32_t pos = -1;
-    if (e >= 0 && e < p.n_cand[row] &&
-        p.S_cand[row * p.ldC + e] != -INFINITY)
-      pos = p.pos_cand[row * p.ldC + e];
-    p.idx[i] = pos;
   }
 }
 
@@ -319,20 +451,16 @@ cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s) {
-  ivf_probe_kernel<<<p.R, 256, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(ivf_probe_kernel, dim3(static_cast<unsigned>(p.R)), dim3(kProbeThreads), 0, s, p);
 }
 cudaError_t launch_ivf_cand(const IvfSearchParams &p, int d, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>(std::max<long long>(1, std::min<long long>(64, (p.N + 2047) / 2048))),
-                  static_cast<unsigned>(p.R));
-  if (d == 128) ivf_cand_kernel<128><<<grid, 256, 0, s>>>(p);
-  else ivf_cand_kernel<64><<<grid, 256, 0, s>>>(p);
-  return cudaGetLastError();
-}
-cudaError_t launch_ivf_map(const IvfSearchParams &p, cudaStream_t s) {
-  const long long n = static_cast<long long>(p.R) * p.k;
-  ivf_map_kernel<<<static_cast<unsigned>(std::max<long long>(1, std::min<long long>(1024, (n + 255) / 256))), 256, 0, s>>>(p);
-  return cudaGetLastError();
+  // CTAs per row from the expected candidate count (twice the mean cluster share); the grid-
+  // stride loop covers any count
+  const long long expect = 2 * p.N * p.nprobe / std::max(p.nlist, 1) + p.nW;
+  const long long x = std::max<long long>(4, std::min<long long>(128, (expect + 511) / 512));
+  const dim3 grid(static_cast<unsigned>(x), static_cast<unsigned>(p.R));
+  if (d == 128) return launch_pdl(ivf_cand_kernel<128>, grid, dim3(256), 0, s, p);
+  return launch_pdl(ivf_cand_kernel<64>, grid, dim3(256), 0, s, p);
 }
 
 }  // namespace ra

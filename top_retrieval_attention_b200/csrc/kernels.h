@@ -88,6 +88,9 @@ struct SaParams {
   float log_eps;            // kSaEps: ln(eps)
   const int32_t *row_n;     // if set: row r's candidates are [0, row_n[r]) of its score row,
                             // with no static set (the IVF candidate lists)
+  const int32_t *pos_map;   // with row_n: [B*Hq, ldS] cache position of each candidate (-1: a
+                            // static-set key); idx reports these positions
+  const float *S_att;       // with row_n: [B*Hq, ldS] full-length score rows for the attention
 };
 
 // Scores of prefill queries (rows (b, h, m) of Q [B, Hq, M, d]) against the keys of their KV
@@ -126,9 +129,7 @@ struct IvfSearchParams {
   int32_t *probe, *cand_off, *n_cand;   // [R, nprobe], [R, nprobe + 1], [R]
   float *S;                 // [R, ldS] full-length score rows (written at candidate and W positions)
   float *S_cand;            // [R, ldC] candidate scores (-inf: a W key)
-  int32_t *pos_cand;        // [R, ldC]
-  const int32_t *idx_cand;  // [R, k] selected candidate indices
-  int32_t *idx;             // [R, k] their cache positions
+  int32_t *pos_cand;        // [R, ldC] cache position of each candidate (-1: a W key)
   long long N, cap, ldS, ldC, s1, w0, nW;
   int R, Hq, Hkv, G, d, nlist, nprobe, k;
   float scale;
@@ -186,7 +187,6 @@ cudaError_t launch_ivf_update(const IvfParams &p, cudaStream_t s);
 cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s);
 cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s);
 cudaError_t launch_ivf_cand(const IvfSearchParams &p, int d, cudaStream_t s);
-cudaError_t launch_ivf_map(const IvfSearchParams &p, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);
 cudaError_t launch_append_paged(const AppendParams &p, const PagedInfo &pg, cudaStream_t s);
 

@@ -710,7 +710,7 @@ ra_status ra_ivf_build(const ra_kv *kv, ra_ivf *ix, int32_t iters, void *ws, siz
 
 struct IvfSearchLayout {
   Step st;                  // the selection's plan over candidate rows of up to N entries
-  size_t off_Sfull, off_poscand, off_probe, off_candoff, off_ncand, off_idxc, total;
+  size_t off_Sfull, off_poscand, off_probe, off_candoff, off_ncand, total;
 };
 static bool ivf_search_layout(int B, int Hq, long long N, int d, int k, int nprobe,
                               IvfSearchLayout &L) {
@@ -723,7 +723,6 @@ static bool ivf_search_layout(int B, int Hq, long long N, int d, int k, int npro
   L.off_probe = off;   off = align_up(off + R * nprobe * 4);
   L.off_candoff = off; off = align_up(off + R * (nprobe + 1) * 4);
   L.off_ncand = off;   off = align_up(off + R * 4);
-  L.off_idxc = off;    off = align_up(off + R * std::max(k, 1) * 4);
   L.total = off;
   return true;
 }
@@ -741,6 +740,7 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
   ra_status s = check_kv(kv);
   if (s != RA_OK) return s;
   if (!ix || !ix->Ksorted || !ix->pos || !ix->offsets || !ix->centroids) return RA_ERR_ARG;
+  if (!aligned16(ix->Ksorted) || !aligned16(ix->centroids)) return RA_ERR_ARG;
   if (ix->B != kv->B || ix->Hkv != kv->Hkv || ix->d != kv->d) return RA_ERR_SHAPE;
   if (nprobe < 1 || nprobe > 64 || nprobe > ix->nlist || ix->nlist > 4096) return RA_ERR_ARG;
   if (ix->N < 1 || ix->N > kv->N || kv->N - ix->N > n_window) return RA_ERR_ARG;
@@ -753,8 +753,14 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
     return RA_ERR_WORKSPACE;
   if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
   if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
-  plan_clusters(dec);
-  plan_clusters(L.st);
+  // one cluster size for the selection and the attention, sized for the expected candidates
+  // (twice the probed clusters' mean share; rows with more take longer chunks) and grown until
+  // a CTA attends over at most 256 entries of U
+  const long long expect = std::min<long long>(
+      ix->N, std::max<long long>(4096, 2 * ix->N * nprobe / ix->nlist));
+  int ncl = select_cluster_size(expect, dec.R, dec.d);
+  const long long nU = dec.nW + std::min<long long>(k, expect);
+  while (ncl < 8 && nU > 256LL * ncl) ncl *= 2;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   IvfSearchParams v{};
   v.q = static_cast<const __nv_bfloat16 *>(q);
@@ -769,9 +775,6 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
   v.S = reinterpret_cast<float *>(at(ws, L.off_Sfull));
   v.S_cand = reinterpret_cast<float *>(at(ws, L.st.off_S));
   v.pos_cand = reinterpret_cast<int32_t *>(at(ws, L.off_poscand));
-  int32_t *idx_cand = reinterpret_cast<int32_t *>(at(ws, L.off_idxc));
-  v.idx_cand = idx_cand;
-  v.idx = idx;
   v.N = ix->N; v.cap = kv->cap; v.ldS = L.st.ldS; v.ldC = L.st.ldS;
   v.s1 = dec.s1; v.w0 = dec.w0; v.nW = dec.nW;
   v.R = dec.R; v.Hq = Hq; v.Hkv = kv->Hkv; v.G = Hq / kv->Hkv; v.d = kv->d;
@@ -780,40 +783,37 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
   cudaError_t e = launch_ivf_probe(v, cs);
   if (e == cudaSuccess) e = launch_ivf_cand(v, kv->d, cs);
   if (e != cudaSuccess) return cuda_fail(e, "ivf_search");
-  if (k > 0) {   // exact top-k of each row's candidates, then their cache positions
-    SaParams p{};
-    p.S = v.S_cand;
-    p.hist = reinterpret_cast<uint32_t *>(at(ws, L.st.off_hist));
-    p.list = reinterpret_cast<uint2 *>(at(ws, L.st.off_list));
-    p.idx = idx_cand;
-    p.part = reinterpret_cast<float *>(at(ws, L.st.off_part));
-    p.meta = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta));
-    p.err = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta)) + kError;
-    p.ldS = L.st.ldS; p.ldL = L.st.ldL; p.N = L.st.N;
-    p.k = k; p.Hq = Hq; p.G = v.G; p.Hkv = kv->Hkv;
-    p.mode = kSaSelect | kSaBuildHist;
+  // the exact top-k of each row's candidates (idx: their cache positions), then softmax
+  // attention over W u Omega from the full-length score rows; one launch unless the attention
+  // wants more clusters per head than the selection has
+  SaParams p{};
+  p.S = v.S_cand;
+  p.S_att = v.S;
+  p.pos_map = v.pos_cand;
+  p.row_n = v.n_cand;
+  p.hist = reinterpret_cast<uint32_t *>(at(ws, L.st.off_hist));
+  p.list = reinterpret_cast<uint2 *>(at(ws, L.st.off_list));
+  p.V = static_cast<const __nv_bfloat16 *>(kv->V);
+  p.idx = idx;
+  p.out = out;
+  p.part = reinterpret_cast<float *>(at(ws, L.st.off_part));
+  p.meta = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta));
+  p.err = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta)) + kError;
+  p.ldS = L.st.ldS; p.ldL = L.st.ldL; p.cap = kv->cap; p.N = dec.N;
+  p.s1 = dec.s1; p.w0 = dec.w0; p.nW = dec.nW; p.nC = dec.nC; p.k_eff = dec.k_eff;
+  p.cbase = dec.cbase; p.cper = dec.cper;
+  p.k = k; p.Hq = Hq; p.G = dec.G; p.Hkv = dec.Hkv;
+  const int split = attn_split(nU, dec.R, ncl, dec.d);
+  if (k > 0) {
+    p.mode = kSaSelect | kSaBuildHist | (split == 1 ? kSaAttend : 0);
     p.nsplit = 1;
-    p.row_n = v.n_cand;
-    e = launch_select_attend(p, kv->d, L.st.R, L.st.ncl, cs);
-    if (e == cudaSuccess) e = launch_ivf_map(v, cs);
-    if (e != cudaSuccess) return cuda_fail(e, "ivf_select");
+    e = launch_select_attend(p, kv->d, dec.R, ncl, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "ivf_select_attend");
+    if (split == 1) return RA_OK;
   }
-  // softmax attention over W u Omega from the full-length score rows
-  SaParams a{};
-  a.S = v.S;
-  a.V = static_cast<const __nv_bfloat16 *>(kv->V);
-  a.idx = idx;
-  a.out = out;
-  a.part = reinterpret_cast<float *>(at(ws, L.st.off_part));
-  a.meta = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta));
-  a.err = reinterpret_cast<uint32_t *>(at(ws, L.st.off_meta)) + kError;
-  a.ldS = L.st.ldS; a.cap = kv->cap; a.N = dec.N;
-  a.s1 = dec.s1; a.w0 = dec.w0; a.nW = dec.nW; a.nC = dec.nC; a.k_eff = dec.k_eff;
-  a.cbase = dec.cbase; a.cper = dec.cper;
-  a.k = k; a.Hq = Hq; a.G = dec.G; a.Hkv = dec.Hkv;
-  a.mode = kSaAttend;
-  a.nsplit = attn_split(dec.nW + dec.k_eff, dec.R, dec.ncl, dec.d);
-  e = launch_select_attend(a, kv->d, dec.R, dec.ncl, cs);
+  p.mode = kSaAttend;
+  p.nsplit = split;
+  e = launch_select_attend(p, kv->d, dec.R, ncl, cs);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "ivf_attend");
 }
 

@@ -64,6 +64,14 @@ struct __align__(16) SaSmem {
   uint32_t t_above, t_cnt;
 };
 
+// The index a selected entry e of row blockIdx.y is reported as in idx: its position in the
+// score row, or, for a candidate list (pos_map set), the cache position the list maps it to (-1:
+// a static-set key).  Read from the parameter block, so it costs the callers no registers.
+__device__ __forceinline__ int32_t idx_of(const SaParams &p, uint32_t e) {
+  return p.pos_map ? __ldcg(p.pos_map + static_cast<long long>(blockIdx.y) * p.ldS + e)
+                   : static_cast<int32_t>(e);
+}
+
 __device__ __forceinline__ unsigned long long composite(uint32_t key, uint32_t pos) {
   return (static_cast<unsigned long long>(key) << 32) | (0xFFFFFFFFu - pos);
 }
@@ -187,8 +195,8 @@ struct ChunkSrc {
 // Bitonic finish in the first CTA: the n <= kFinish keys in sm.fin, the `want` largest written
 // to irow[o0 ..].  One warp.
 template <int D>
-__device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32_t want,
-                                               int32_t *irow, uint32_t o0) {
+__device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm, uint32_t n,
+                                               uint32_t want, int32_t *irow, uint32_t o0) {
   const int tid = threadIdx.x, lane = tid & 31;
   if (n <= 32) {   // one key per lane: a key is taken when fewer than `want` keys exceed it
     if (tid < 32) {
@@ -196,7 +204,7 @@ __device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32
       uint32_t above = 0;
       for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, x, j) > x ? 1u : 0u;
       if (static_cast<uint32_t>(lane) < n && above < want)
-        irow[o0 + above] = static_cast<int32_t>(composite_pos(x));
+        irow[o0 + above] = idx_of(p, composite_pos(x));
     }
     return;
   }
@@ -218,7 +226,7 @@ __device__ __forceinline__ void bitonic_finish(SaSmem<D> &sm, uint32_t n, uint32
         __syncwarp();
       }
     }
-    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = static_cast<int32_t>(composite_pos(sm.fin[i]));
+    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = idx_of(p, composite_pos(sm.fin[i]));
   }
 }
 
@@ -320,11 +328,11 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
       if ((x >> sh) != prefix) return;
       const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
       if (dg > t) {
-        if (ou < k_eff) irow[ou] = static_cast<int32_t>(composite_pos(x));
+        if (ou < k_eff) irow[ou] = idx_of(p, composite_pos(x));
         ++ou;
       } else if (dg == t) {
         if (take_eq) {
-          if (base + up + oe < k_eff) irow[base + up + oe] = static_cast<int32_t>(composite_pos(x));
+          if (base + up + oe < k_eff) irow[base + up + oe] = idx_of(p, composite_pos(x));
         } else if (fin && oe < static_cast<uint32_t>(kFinish)) {
           fin0[oe] = x;
         }
@@ -334,7 +342,8 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
     if (take_eq) return;
     if (fin) {
       cl.sync();   // the final bucket is complete in the first CTA
-      if (rank == 0) bitonic_finish(sm, eq, min(want2, k_eff - min(k_eff, base + up)), irow, base + up);
+      if (rank == 0)
+        bitonic_finish(p, sm, eq, min(want2, k_eff - min(k_eff, base + up)), irow, base + up);
       return;
     }
     // next digit: every remote read of sm.h came before the last barrier
@@ -478,6 +487,14 @@ __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const PagedInfo &pg
   g.cper = ((span + ncl - 1) / ncl + 3) / 4 * 4;
   return g;
 }
+// The geometry the attention uses: the row's own, except that a candidate list's Omega (the
+// min(k, candidates) entries of idx) is attended together with the cache's static set.
+template <class Pg>
+__device__ __forceinline__ RowGeo attend_geo(const SaParams &p, const Pg &pg, int row, int ncl) {
+  RowGeo g = row_geo(p, pg, row, ncl);
+  if (p.row_n) g = RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, g.k_eff, p.cbase, p.cper};
+  return g;
+}
 // Where token `pos` of sequence b, KV head gk, sits in V: v_base(...) + v_index(...) * d.
 // Dense caches: the (b, gk) plane and the position; paged caches: the pool and the pool row
 // of the token's page.
@@ -600,7 +617,8 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     __syncthreads();
   }
   if (k_sel >= gm.nC) {   // every candidate is selected
-    for (long long i = lo + tid; i < hi; i += kSaThreads) irow[i - gm.s1] = static_cast<int32_t>(i);
+    for (long long i = lo + tid; i < hi; i += kSaThreads)
+      irow[i - gm.s1] = idx_of(p, static_cast<uint32_t>(i));
     return;
   }
   const uint32_t k_eff = static_cast<uint32_t>(k_sel);
@@ -642,7 +660,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   // the keys above b1 take idx slots [0, above1), CTA by CTA
   if (sm.n_sure <= static_cast<uint32_t>(kSureCap)) {
     for (uint32_t i = tid; i < sm.n_sure; i += kSaThreads)
-      if (off + i < k_eff) irow[off + i] = static_cast<int32_t>(sm.sure[i]);
+      if (off + i < k_eff) irow[off + i] = idx_of(p, sm.sure[i]);
   } else {   // more sure keys than sm.sure holds: from the chunk again
     uint32_t cu = 0;
     chunk.for_each([&](unsigned long long x) { cu += (x >> (64 - kHistBits)) > b1 ? 1u : 0u; });
@@ -651,7 +669,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     uint32_t o = off + inc.x - cu;
     chunk.for_each([&](unsigned long long x) {
       if ((x >> (64 - kHistBits)) > b1) {
-        if (o < k_eff) irow[o] = static_cast<int32_t>(composite_pos(x));
+        if (o < k_eff) irow[o] = idx_of(p, composite_pos(x));
         ++o;
       }
     });
@@ -682,7 +700,7 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   const long long e_hi = min(nU, e_lo + per);
   const int b = row / p.Hq, h = row - b * p.Hq;
   const __nv_bfloat16 *Vb = v_base<D>(p, pg, b, h / p.G);
-  const float *srow = p.S + static_cast<long long>(row) * p.ldS;
+  const float *srow = (p.S_att ? p.S_att : p.S) + static_cast<long long>(row) * p.ldS;
   const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   int *spos = reinterpret_cast<int *>(sm.sure);   // staged: the entry's V row (-1: none)
   float *sz = reinterpret_cast<float *>(sm.sure + kStage);
@@ -841,13 +859,13 @@ __global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaPa
   const int ncl = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
   const int row = blockIdx.y;
-  const RowGeo gm = row_geo(p, pg, row, ncl);
   pdl_trigger();
   pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
-  if (p.mode & kSaSelect) select_phase<D>(p, gm, sm, cl, rank, ncl, row);
+  // each phase computes the row geometry afresh (nothing stays live across the selection)
+  if (p.mode & kSaSelect) select_phase<D>(p, row_geo(p, pg, row, ncl), sm, cl, rank, ncl, row);
   if (p.mode & kSaAttend) {
     if (p.mode & kSaSelect) cl.sync();   // Omega complete in idx (release/acquire at cluster scope)
-    attend_phase<D>(p, gm, pg, sm, cl, rank, ncl, row);
+    attend_phase<D>(p, attend_geo(p, pg, row, ncl), pg, sm, cl, rank, ncl, row);
   } else {
     cl.sync();   // no CTA leaves while the cluster may still use its shared memory
   }
