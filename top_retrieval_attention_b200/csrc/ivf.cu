@@ -203,6 +203,7 @@ __device__ __forceinline__ uint32_t probe_scan(uint32_t v, uint32_t *wsum, uint3
 // nprobe-th largest; the keys at or above it are gathered and each is ranked by counting the
 // gathered keys above it.  Should that bin hold more keys than the gather takes, every key is
 // sorted instead (bitonic, in shared memory).
+template <int D>
 __global__ void __launch_bounds__(kProbeThreads) ivf_probe_kernel(const IvfSearchParams p) {
   __shared__ unsigned long long keys[kIvfMaxList];
   __shared__ unsigned long long coll[kProbeCollect];
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kProbeThreads) ivf_probe_kernel(const IvfSearc
   const long long bg = static_cast<long long>(b) * p.Hkv + h / p.G;
   pdl_trigger();
   pdl_wait();   // the query and the cache may come from earlier kernels of the stream
-  if (tid < p.d) qs[tid] = __bfloat162float(p.q[static_cast<long long>(row) * p.d + tid]);
+  if (tid < D) qs[tid] = __bfloat162float(p.q[static_cast<long long>(row) * D + tid]);
   for (int i = tid; i < kHistBins; i += kProbeThreads) hist[i] = 0u;
   if (tid < 64) sel[tid] = 0;   // a valid cluster in every slot whatever happens below
   if (tid == 0) {
@@ -225,12 +226,16 @@ __global__ void __launch_bounds__(kProbeThreads) ivf_probe_kernel(const IvfSearc
     n_coll = 0u;
   }
   __syncthreads();
-  // a thread per centroid, its row read in 16-byte pieces
+  // a thread per centroid, its row read in 16-byte pieces (all in flight together)
   for (int c = tid; c < p.nlist; c += kProbeThreads) {
-    const uint4 *cr = reinterpret_cast<const uint4 *>(p.cent + (bg * p.nlist + c) * p.d);
+    const uint4 *cr = reinterpret_cast<const uint4 *>(p.cent + (bg * p.nlist + c) * D);
+    uint4 row_v[D / 8];
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) row_v[j] = __ldg(cr + j);
     float z = 0.f;
-    for (int j = 0; j < p.d / 8; ++j) {
-      const uint4 v = __ldg(cr + j);
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      const uint4 v = row_v[j];
       const float *qq = qs + 8 * j;
       z += qq[0] * bf16_lo(v.x) + qq[1] * bf16_hi(v.x) + qq[2] * bf16_lo(v.y) +
            qq[3] * bf16_hi(v.y) + qq[4] * bf16_lo(v.z) + qq[5] * bf16_hi(v.z) +
@@ -394,6 +399,7 @@ __global__ void __launch_bounds__(256) ivf_cand_kernel(const IvfSearchParams p) 
         }
         si = sbase[lo] + (e - soff[lo]);
         krow = p.Ksorted + si * D;
+        if (sub == 0) pos = __ldg(p.pos + si);   // in flight with the key's loads
       } else {
         const long long wi = e - n_cand;
         pos = wi < p.s1 ? wi : p.w0 + (wi - p.s1);
@@ -418,7 +424,6 @@ __global__ void __launch_bounds__(256) ivf_cand_kernel(const IvfSearchParams p) 
     z += __shfl_xor_sync(0xffffffffu, z, 2);
     if (valid && sub == 0) {
       z = canon_zero(z * p.scale);
-      if (si >= 0) pos = p.pos[si];
       srow[pos] = z;
       if (e < n_cand) {
         const bool in_w = pos < p.s1 || pos >= p.w0;
@@ -451,13 +456,15 @@ cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s) {
   return cudaGetLastError();
 }
 cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s) {
-  return launch_pdl(ivf_probe_kernel, dim3(static_cast<unsigned>(p.R)), dim3(kProbeThreads), 0, s, p);
+  const dim3 grid(static_cast<unsigned>(p.R));
+  if (p.d == 128) return launch_pdl(ivf_probe_kernel<128>, grid, dim3(kProbeThreads), 0, s, p);
+  return launch_pdl(ivf_probe_kernel<64>, grid, dim3(kProbeThreads), 0, s, p);
 }
 cudaError_t launch_ivf_cand(const IvfSearchParams &p, int d, cudaStream_t s) {
-  // CTAs per row from the expected candidate count (twice the mean cluster share); the grid-
-  // stride loop covers any count
+  // CTAs per row from the expected candidate count (twice the mean cluster share), one key per
+  // lane group at that count; the grid-stride loop covers any count
   const long long expect = 2 * p.N * p.nprobe / std::max(p.nlist, 1) + p.nW;
-  const long long x = std::max<long long>(4, std::min<long long>(128, (expect + 511) / 512));
+  const long long x = std::max<long long>(4, std::min<long long>(256, (expect + 255) / 256));
   const dim3 grid(static_cast<unsigned>(x), static_cast<unsigned>(p.R));
   if (d == 128) return launch_pdl(ivf_cand_kernel<128>, grid, dim3(256), 0, s, p);
   return launch_pdl(ivf_cand_kernel<64>, grid, dim3(256), 0, s, p);

@@ -44,6 +44,10 @@ constexpr int kListSmem = 1536;   // keys in b1 kept in shared memory per CTA (t
 constexpr int kFinish = 64;       // bitonic finish size (one warp)
 constexpr int kStreamVec = 8;     // float4 score loads per thread in flight
 
+// The first CTA's threshold list doubles as the attention's exchange area: one D-float
+// numerator per CTA of the cluster.
+static_assert(kMaxCluster * 128 * sizeof(float) <= kListSmem * sizeof(uint2), "exchange area");
+
 template <int D>
 struct __align__(16) SaSmem {
   uint32_t sure[kSureCap];
@@ -51,13 +55,12 @@ struct __align__(16) SaSmem {
   float wacc[kSaWarps * D];       // attention: per-warp numerators
   uint32_t h[kHistBins];          // digit histogram of the current round (slice reduced in place)
   unsigned long long fin[kFinish];  // first CTA: keys of the final bucket
-  float pacc[D];                  // this CTA's partial state (read by the first CTA)
-  float pm, pz;
   float wm[kSaWarps], wz[kSaWarps];
   uint32_t x_a[kMaxCluster];      // per-rank exchange slots (written remotely before a barrier)
   uint32_t x_b[kMaxCluster];
   uint32_t x_tot[kMaxCluster];
-  float x_m[kMaxCluster], x_s[kMaxCluster];   // per-rank (max, sum e^{z - max}) of a row
+  float x_m[kMaxCluster], x_s[kMaxCluster];   // per-rank (max, sum e^{z - max}): of a row's
+                                              // scores, or of a CTA's attention partial state
   uint32_t warp_tot[2 * kSaWarps];
   uint32_t n_sure, n_list;
   int t_bin;
@@ -793,38 +796,38 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   float ew[kSaWarps];
 #pragma unroll
   for (int i = 0; i < kSaWarps; ++i) ew[i] = sm.wm[i] == -INFINITY ? 0.f : expf(sm.wm[i] - M);
+  // this CTA's partial state goes straight into the first CTA's exchange slots (its threshold
+  // list is free during the attention): numerators [rank][D], (m, Z) in x_m / x_s
+  float *xacc0 = reinterpret_cast<float *>(cl.map_shared_rank(sm.list, 0));
   for (int c = tid; c < D; c += kSaThreads) {
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < kSaWarps; ++i) s += ew[i] * sm.wacc[i * D + c];
-    sm.pacc[c] = s;
+    xacc0[rank * D + c] = s;
   }
   if (tid == 0) {
     float zt = 0.f;
 #pragma unroll
     for (int i = 0; i < kSaWarps; ++i) zt += ew[i] * sm.wz[i];
-    sm.pm = M;
-    sm.pz = zt;
+    cl.map_shared_rank(sm.x_m, 0)[rank] = M;
+    cl.map_shared_rank(sm.x_s, 0)[rank] = zt;
   }
-  cl.sync();   // every CTA's partial state is ready
+  cl.sync();   // every CTA's partial state is in the first CTA
   if (rank == 0) {
+    const float *xacc = reinterpret_cast<const float *>(sm.list);
     float Mx = -INFINITY;
-    for (int c = 0; c < ncl; ++c) Mx = fmaxf(Mx, cl.map_shared_rank(&sm.pm, c)[0]);
+    for (int c = 0; c < ncl; ++c) Mx = fmaxf(Mx, sm.x_m[c]);
     float den = 0.f;
-    for (int c = 0; c < ncl; ++c) {
-      const float mc = cl.map_shared_rank(&sm.pm, c)[0];
-      if (mc != -INFINITY) den += expf(mc - Mx) * cl.map_shared_rank(&sm.pz, c)[0];
-    }
+    for (int c = 0; c < ncl; ++c)
+      if (sm.x_m[c] != -INFINITY) den += expf(sm.x_m[c] - Mx) * sm.x_s[c];
     // one cluster: the output; several: this cluster's state for the last one to merge
     constexpr int PS = D + kPartPad;
     float *prow = p.part + static_cast<long long>(row) * kMaxAttnSplit * PS;
     float *mine = prow + static_cast<long long>(blockIdx.z) * PS;
     for (int ch = tid; ch < D; ch += kSaThreads) {
       float num = 0.f;
-      for (int c = 0; c < ncl; ++c) {
-        const float mc = cl.map_shared_rank(&sm.pm, c)[0];
-        if (mc != -INFINITY) num += expf(mc - Mx) * cl.map_shared_rank(sm.pacc, c)[ch];
-      }
+      for (int c = 0; c < ncl; ++c)
+        if (sm.x_m[c] != -INFINITY) num += expf(sm.x_m[c] - Mx) * xacc[c * D + ch];
       if (p.nsplit == 1) p.out[static_cast<long long>(row) * D + ch] = num / den;
       else mine[kPartPad + ch] = num;
     }
@@ -849,7 +852,7 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
       }
     }
   }
-  cl.sync();   // the first CTA has read every partial state
+  // no CTA reads another's shared memory after the exchange barrier: all may leave
 }
 
 template <int D, class Pg>
