@@ -2,10 +2,12 @@
 """Decode-step benchmark of exact top-k retrieval attention on B200.
 
 A step is one pass of the whole hot path for every layer of the workload: append the new
-token's K/V row (ra_append_kv), score all positions (ra_score_gqa), select the top-k per query
-head (ra_topk_select), and attend over sinks + window + top-k (ra_sparse_attn).  The cache
-holds N-1 tokens; each step appends the N-th and decodes over N, then the next step re-appends
-into the same slot, so every step has identical work.  Each step uses its own query.
+token's K/V row and score all positions (ra_score_gqa_append: the append runs inside the
+scan), then select the top-k per query head and attend over sinks + window + top-k
+(ra_select_attend); together they are ra_decode_step_append.  The cache holds N-1 tokens; each
+step appends the N-th and decodes over N, then the next step re-appends into the same slot, so
+every step has identical work.  Each step uses its own query.  (The threshold mode, --eps,
+appends with ra_append_kv and runs ra_decode_step_eps.)
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -319,6 +321,20 @@ def run_ours(args, w, rank, local_rank, world, dist):
         kl = ks[layer]
         if ev is not None:
             ev[0].record(stream)
+        if args.eps <= 0:   # the append runs inside the scan (one launch), then select + attend
+            ra.check(ra.ra_score_gqa_append(kv, qptr, knew[layer].data_ptr(), vnew[layer].data_ptr(),
+                                            Hq, kl, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes,
+                                            sp), "score_append")
+            if ev is not None:
+                ev[1].record(stream)
+                ev[2].record(stream)
+            ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window, idxs[layer].data_ptr(),
+                                         outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp),
+                     "select_attend")
+            if ev is not None:
+                ev[3].record(stream)
+            c.N = N - 1
+            return
         ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
         if ev is not None:
             ev[1].record(stream)
@@ -351,6 +367,18 @@ def run_ours(args, w, rank, local_rank, world, dist):
             kv = c.kv
             kl = ks[layer]
             qptr = qpool[s % P, layer].data_ptr()
+            if args.eps <= 0:   # the scan with the append inside it, timed alone
+                ev[layer][0].record(stream)
+                ra.check(ra.ra_score_gqa_append(kv, qptr, knew[layer].data_ptr(),
+                                                vnew[layer].data_ptr(), Hq, kl, w.n_sink,
+                                                w.n_window, ws.data_ptr(), ws_bytes, sp),
+                         "score_append")
+                ev[layer][1].record(stream)
+                ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window,
+                                             idxs[layer].data_ptr(), outs[layer].data_ptr(),
+                                             ws.data_ptr(), ws_bytes, sp), "select_attend")
+                c.N = N - 1
+                continue
             ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
             if args.eps > 0:   # the score kernel runs inside the one call: time the whole call
                 ev[layer][0].record(stream)
@@ -418,12 +446,18 @@ def run_ours(args, w, rank, local_rank, world, dist):
     for s in range(psteps):
         step(s, evs[s])
     torch.cuda.synchronize()
-    ph = {"append": [], "score": [], "select_attend": []}
+    fused = args.eps <= 0
+    ph = {"score_with_append" if fused else "append": [], "score": [], "select_attend": []}
+    if fused:
+        del ph["score"]
     for s in range(psteps):
         for layer in range(L):
             e = evs[s][layer]
-            ph["append"].append(e[0].elapsed_time(e[1]))
-            ph["score"].append(e[1].elapsed_time(e[2]))
+            if fused:
+                ph["score_with_append"].append(e[0].elapsed_time(e[1]))
+            else:
+                ph["append"].append(e[0].elapsed_time(e[1]))
+                ph["score"].append(e[1].elapsed_time(e[2]))
             ph["select_attend"].append(e[2].elapsed_time(e[3]))
     ph_us = {kk: 1000.0 * statistics.mean(v) for kk, v in ph.items()}
 
@@ -453,7 +487,9 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 "algorithmic_bytes_per_launch": k_bytes,
                 "frac_of_nominal_8tbs": kscan_gbs / NOMINAL_HBM_GBS,
                 "score_kernel_sha": src_hash}
-    launches_per_layer = 3   # append, score, select + attention
+    # the scan with the append inside it, then select + attention (threshold mode: append,
+    # score, select + attention)
+    launches_per_layer = 2 if fused else 3
     result = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -495,7 +531,8 @@ def run_ours(args, w, rank, local_rank, world, dist):
         b.record(stream)
         torch.cuda.synchronize()
         dense_ms = max_over_ranks(dist, a.elapsed_time(b) / dsteps, dev)
-        sparse_decode_ms = ms_per_step - L * ph_us["append"] / 1000.0
+        # the sparse step includes its append (inside the scan); dense decode appends nothing
+        sparse_decode_ms = ms_per_step - (0.0 if fused else L * ph_us["append"] / 1000.0)
         result["dense"] = {"ms_per_step": dense_ms, "steps": dsteps,
                            "hbm_gbs": L * 2 * k_bytes / (dense_ms / 1000.0) / 1e9,
                            "speedup_of_sparse_decode": dense_ms / sparse_decode_ms}
@@ -521,13 +558,15 @@ def run_ours(args, w, rank, local_rank, world, dist):
             for layer in range(L):
                 dk[layer].copy_(hk[layer], non_blocking=True)
                 dv[layer].copy_(hv[layer], non_blocking=True)
-                ra.append_kv(caches[layer], dk[layer], dv[layer])
+                if args.eps <= 0:
+                    ra.decode_step_append(caches[layer], dq[layer], dk[layer], dv[layer], ks[layer],
+                                          w.n_sink, w.n_window, out=outs[layer], idx=idxs[layer],
+                                          ws=ws)
+                else:
+                    ra.append_kv(caches[layer], dk[layer], dv[layer])
                 if args.eps > 0:
                     ra.decode_step_eps(caches[layer], dq[layer], ks[layer], args.eps, w.n_sink,
                                        w.n_window, out=outs[layer], idx=idxs[layer], ws=ws)
-                else:
-                    ra.decode_step(caches[layer], dq[layer], ks[layer], w.n_sink, w.n_window,
-                                   out=outs[layer], idx=idxs[layer], ws=ws)
                 caches[layer].N = N - 1
                 ho[layer].copy_(outs[layer], non_blocking=True)
                 hi[layer].copy_(idxs[layer], non_blocking=True)
@@ -548,7 +587,9 @@ def run_ours(args, w, rank, local_rank, world, dist):
         result["e2e"] = {"value": world * 1000.0 / e2e_ms, "unit": "steps/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": esteps,
                          "ms_per_step": e2e_ms,
-                         "note": "public API (append_kv + decode_step), host sync every step"}
+                         "note": ("public API (decode_step_append" if args.eps <= 0 else
+                                  "public API (append_kv + decode_step_eps") +
+                                 "), host sync every step"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc = oracle_sample(w, args.cpu_seconds)

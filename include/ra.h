@@ -142,6 +142,26 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
                          ra_stream_t stream);
 
 /*
+ * Append one token and run the decode step over the grown cache, with the append done inside
+ * the scan instead of as a launch of its own: ra_append_kv(kv, k_new, v_new, 1) followed by
+ * ra_decode_step, with the same results.  The CTA of the score kernel whose tile holds the new
+ * position writes the token's K and V rows to the cache and scores the key from its staged
+ * tile (Eq. (1) sums over j <= t: the current token is attended, here through the window).
+ *   k_new, v_new : bf16 [B, Hkv, 1, d], device, 16-byte aligned.
+ *   Other arguments as ra_decode_step; the workspace is sized for kv->N + 1 tokens.
+ * On success kv->N has grown by one.  Errors: as ra_decode_step, checked before any launch
+ * (kv unchanged); RA_ERR_CAPACITY when kv->N + 1 > cap.
+ */
+ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, const void *v_new,
+                                int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window,
+                                float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                                ra_stream_t stream);
+/* The scan phase of ra_decode_step_append alone (then ra_select_attend over the grown kv). */
+ra_status ra_score_gqa_append(ra_kv *kv, const void *q, const void *k_new, const void *v_new,
+                              int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window, void *ws,
+                              size_t ws_bytes, ra_stream_t stream);
+
+/*
  * ra_decode_step with the retrieval set cut at a softmax-weight threshold (Eq. (2), slide
  * "Sparse attention renormalizes selected tokens"): Omega = the candidates i of C whose full
  * softmax weight a_i = e^{z_i} / sum_{j < N} e^{z_j} exceeds eps, the k largest of them when

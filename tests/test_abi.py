@@ -134,6 +134,23 @@ def test_append_capacity_and_arguments():
     assert kv.N == 98
 
 
+def test_fused_append_step_validates_before_launch():
+    big = 1 << 30
+    args = (FAKE, 4, 10, 4, 8, FAKE, FAKE, FAKE, big, None)   # Hq, k, sinks, window, out, idx, ws
+    kv = _kv(cap=100, N=100)
+    assert ra.ra_decode_step_append(kv, FAKE, FAKE, FAKE, *args[1:]) == ra.RA_ERR_CAPACITY
+    assert ra.ra_score_gqa_append(kv, FAKE, FAKE, FAKE, 4, 10, 4, 8, FAKE, big, None) == ra.RA_ERR_CAPACITY
+    kv = _kv(cap=100, N=50)
+    assert ra.ra_decode_step_append(kv, FAKE, 0, FAKE, *args[1:]) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step_append(kv, FAKE, FAKE, FAKE + 8, *args[1:]) == ra.RA_ERR_ARG
+    assert ra.ra_decode_step_append(kv, FAKE, FAKE, FAKE, 3, 10, 4, 8, FAKE, FAKE, FAKE, big,
+                                    None) == ra.RA_ERR_SHAPE
+    assert ra.ra_decode_step_append(kv, FAKE, FAKE, FAKE, 4, 10, 4, 8, FAKE, FAKE, FAKE, 16,
+                                    None) == ra.RA_ERR_WORKSPACE
+    assert ra.ra_decode_step_append(kv, 0, FAKE, FAKE, *args[1:]) == ra.RA_ERR_ARG
+    assert kv.N == 50   # no error grows the cache
+
+
 def test_synth_constants_match_host_generator():
     from synth import gen
     a, b = sdev.constants()

@@ -9,5 +9,5 @@ from .ra import (  # noqa: F401
     ra_prefill_workspace_bytes, ra_prefill_topk, ra_prefill_score, ra_prefill_select, prefill_topk,
     ra_decode_step_eps, decode_step_eps, pyramid_budgets, ra_paged_kv, PagedKVCache,
     paged_append_kv, paged_workspace, paged_decode_step, ra_ivf, IvfIndex, ivf_build,
-    ivf_decode_step,
+    ivf_decode_step, ra_decode_step_append, ra_score_gqa_append, decode_step_append,
 )

@@ -43,6 +43,11 @@ struct ScoreParams {
   float scale;
   int do_hist;
   uint32_t *err;            // error word (bit kErrScoreWait: a load never landed)
+  // Appending the step's token inside the scan (dense caches; all null otherwise): position
+  // N - 1 of every head is the new token, whose K / V rows ([B * Hkv, d]) the CTA scanning
+  // that tile writes to the cache and patches into its staged tile before scoring it.
+  const __nv_bfloat16 *k_new, *v_new;
+  __nv_bfloat16 *K_cache, *V_cache;
 };
 
 // Paged KV caches: K and V in pages of kPageSize tokens, [num_pages, Hkv, kPageSize, d]; sequence

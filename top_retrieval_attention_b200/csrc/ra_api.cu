@@ -130,7 +130,8 @@ static ra_status plan_step(const ra_kv *kv, int Hq, int k, int n_sink, int n_win
 static uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
 
 static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void *ws,
-                           cudaStream_t stream, bool hist = true) {
+                           cudaStream_t stream, bool hist = true, const void *k_new = nullptr,
+                           const void *v_new = nullptr) {
   ScoreParams p{};
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -144,6 +145,12 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
   p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
   p.do_hist = hist && st.k_eff > 0 && st.k_eff < st.nC;
   p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
+  if (k_new != nullptr) {   // the step's token is appended inside the scan (position N - 1)
+    p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    p.K_cache = static_cast<__nv_bfloat16 *>(kv->K);
+    p.V_cache = static_cast<__nv_bfloat16 *>(kv->V);
+  }
   const cudaError_t e = launch_score(p, st.d, stream);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
@@ -268,6 +275,49 @@ ra_status ra_score_gqa(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, in
   if (s != RA_OK) return s;
   if (!q || !aligned16(q)) return RA_ERR_ARG;
   return run_score(kv, q, st, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Validation of the fused append + decode entry points: kv grows by one token, which must fit.
+static ra_status plan_append_step(ra_kv *kv, const void *k_new, const void *v_new, int32_t Hq,
+                                  int32_t k, int32_t n_sink, int32_t n_window, void *ws,
+                                  size_t ws_bytes, ra_kv &grown, Step &st) {
+  ra_status s = check_kv(kv);
+  if (s != RA_OK) return s;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return RA_ERR_ARG;
+  if (kv->N + 1 > kv->cap) return RA_ERR_CAPACITY;
+  grown = *kv;
+  grown.N = kv->N + 1;
+  return plan_step(&grown, Hq, k, n_sink, n_window, ws, ws_bytes, st);
+}
+
+ra_status ra_score_gqa_append(ra_kv *kv, const void *q, const void *k_new, const void *v_new,
+                              int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window, void *ws,
+                              size_t ws_bytes, ra_stream_t stream) {
+  ra_kv grown{};
+  Step st{};
+  ra_status s = plan_append_step(kv, k_new, v_new, Hq, k, n_sink, n_window, ws, ws_bytes, grown, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q)) return RA_ERR_ARG;
+  s = run_score(&grown, q, st, ws, reinterpret_cast<cudaStream_t>(stream), true, k_new, v_new);
+  if (s == RA_OK) kv->N = grown.N;
+  return s;
+}
+
+ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, const void *v_new,
+                                int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window,
+                                float *out, int32_t *idx, void *ws, size_t ws_bytes,
+                                ra_stream_t stream) {
+  ra_kv grown{};
+  Step st{};
+  ra_status s = plan_append_step(kv, k_new, v_new, Hq, k, n_sink, n_window, ws, ws_bytes, grown, st);
+  if (s != RA_OK) return s;
+  if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
+  if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  s = run_score(&grown, q, st, ws, cs, true, k_new, v_new);
+  if (s != RA_OK) return s;
+  kv->N = grown.N;   // the token is in the cache once the scan has run
+  return run_select_attend(&grown, st, kSaSelect | kSaAttend, idx, out, ws, cs);
 }
 
 ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,

@@ -13,7 +13,11 @@
 //     fp32 accumulation; each warp scores 16 keys of the tile from ldmatrix fragments;
 //   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram (top
 //     11 bits of the order-preserving key) of the candidate positions in shared memory,
-//     flushed to global once per KV head.
+//     flushed to global once per KV head;
+//   * optionally the step's append is fused in: the CTA whose tile holds the new token writes
+//     its K and V rows to the cache and patches the key row into the staged tile.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tma.cuh"
@@ -195,6 +199,24 @@ __global__ void __launch_bounds__(256, 1)
     }
 
     const uint32_t tbase = tiles + slot * C::kTileBytes;
+    if (std::is_same<Pg, NoPaging>::value && p.k_new != nullptr && c_key <= p.N - 1 &&
+        p.N - 1 < c_key + C::kTile) {
+      // the tile holding the token this step appends (uniform over the CTA): its key row
+      // replaces the stale row in the staged tile, and its K and V rows go to the cache
+      const int r = static_cast<int>(p.N - 1 - c_key);
+      constexpr int kChunks = D / 8;   // 16-byte chunks of a row
+      const long long src = c_bg * D, dst = (c_bg * p.cap + p.N - 1) * D;
+      if (tid < kChunks) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.k_new + src) + tid);
+        st_shared_v4(tbase + (tid >> 3) * C::kBoxBytes + r * 128 + (((tid & 7) ^ (r & 7)) << 4), v);
+        reinterpret_cast<uint4 *>(p.K_cache + dst)[tid] = v;
+        fence_proxy_async_smem();   // before a later TMA load refills this stage
+      } else if (tid >= 32 && tid < 32 + kChunks) {
+        reinterpret_cast<uint4 *>(p.V_cache + dst)[tid - 32] =
+            __ldg(reinterpret_cast<const uint4 *>(p.v_new + src) + (tid - 32));
+      }
+      __syncthreads();
+    }
     float acc0[4] = {0.f, 0.f, 0.f, 0.f};
     float acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

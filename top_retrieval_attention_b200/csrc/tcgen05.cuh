@@ -94,10 +94,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
 
 // ---- TMA tensor store (shared -> global) of an epilogue tile
 
-// Makes this thread's earlier shared-memory writes visible to the tensor-copy (async) proxy.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
+// (fence_proxy_async_smem, which orders the epilogue's shared-memory writes before the store,
+// is in tma.cuh)
 
 // 3-D tiled bulk tensor store of the box at shared address `src` to coordinates (x, y, z);
 // elements outside the tensor are not written.  One thread; completion is tracked per bulk

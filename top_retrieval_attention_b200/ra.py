@@ -25,7 +25,7 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets",
            "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step",
            "ra_ivf_build_workspace_bytes", "ra_ivf_build", "ra_ivf_search_workspace_bytes",
-           "ra_ivf_decode_step")
+           "ra_ivf_decode_step", "ra_decode_step_append", "ra_score_gqa_append")
 
 
 class ra_kv(ctypes.Structure):
@@ -106,6 +106,11 @@ def lib() -> ctypes.CDLL:
                                             c_void_p, c_size_t, c_void_p]),
             "ra_decode_step_static": (c_int32, [P, c_void_p, c_int32, c_int32, c_int32, c_int32,
                                                 c_void_p, c_void_p, c_void_p]),
+            "ra_decode_step_append": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                                c_int32, c_int32, c_void_p, c_void_p, c_void_p,
+                                                c_size_t, c_void_p]),
+            "ra_score_gqa_append": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
+                                              c_int32, c_int32, c_void_p, c_size_t, c_void_p]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -252,6 +257,38 @@ def decode_step(cache: KVCache, q, k: int, n_sink: int, n_window: int, out=None,
     check(ra_decode_step(cache.kv, q.data_ptr(), Hq, k, n_sink, n_window, out.data_ptr(),
                          idx.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
           "ra_decode_step")
+    return out, idx[..., :k]
+
+
+def ra_decode_step_append(kv, q, k_new, v_new, Hq, k, n_sink, n_window, out, idx, ws, ws_bytes,
+                          stream):
+    return lib().ra_decode_step_append(ctypes.byref(kv), q, k_new, v_new, Hq, k, n_sink, n_window,
+                                       out, idx, ws, ws_bytes, stream)
+
+
+def ra_score_gqa_append(kv, q, k_new, v_new, Hq, k, n_sink, n_window, ws, ws_bytes, stream):
+    return lib().ra_score_gqa_append(ctypes.byref(kv), q, k_new, v_new, Hq, k, n_sink, n_window,
+                                     ws, ws_bytes, stream)
+
+
+def decode_step_append(cache: KVCache, q, k_new, v_new, k: int, n_sink: int, n_window: int,
+                       out=None, idx=None, ws=None, stream=None):
+    """Append one token (k_new, v_new: bf16 [B, Hkv, 1, d]) and decode over the grown cache,
+    the append done inside the scan.  Returns (out fp32, idx int32); cache.N grows by one."""
+    import torch
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty((B, Hq, max(k, 1)), dtype=torch.int32, device=q.device)
+    if ws is None:
+        n = ra_decode_workspace_bytes(B, Hq, cache.N + 1, d, k, n_sink, n_window)
+        if n == 0:
+            raise RaError(RA_ERR_SHAPE, "ra_decode_workspace_bytes")
+        ws = torch.zeros(n, dtype=torch.uint8, device=q.device)
+    check(ra_decode_step_append(cache.kv, q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), Hq, k,
+                                n_sink, n_window, out.data_ptr(), idx.data_ptr(), ws.data_ptr(),
+                                ws.numel(), _stream(stream)), "ra_decode_step_append")
     return out, idx[..., :k]
 
 
