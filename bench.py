@@ -76,6 +76,9 @@ def parse():
     ap.add_argument("--paged", action="store_true",
                     help="paged cache (128-token pages, shuffled) with ragged lengths falling "
                          "linearly from N to N/2 over the batch (ra_paged_decode_step)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="every point of the 512K sweep (top-k x group size x head dim), one JSON "
+                         "line each, the dense decode beside it (no e2e / CPU legs)")
     ap.add_argument("--ivf", type=int, default=0, metavar="NLIST",
                     help="decode through a device-built IVF index of NLIST clusters per KV head "
                          "(one layer); reports Recall@k against the exact top-k")
@@ -959,6 +962,17 @@ def main():
         raise SystemExit("bench.py needs a CUDA device (the product has no CPU path)")
     dist = dist_init(world, True)
     try:
+        if args.sweep:
+            import gc
+            args.no_e2e = True
+            args.no_cpu_baseline = True
+            for name in gen.sweep_names():
+                res = run_ours(args, gen.workload(name), rank, local_rank, world, dist)
+                if rank == 0:
+                    print(json.dumps(res), flush=True)
+                gc.collect()
+                torch.cuda.empty_cache()
+            return
         if args.prefill_queries > 0:
             res = run_prefill(args, w, rank, local_rank, world, dist)
         elif args.ivf > 0:
