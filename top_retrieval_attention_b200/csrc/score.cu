@@ -24,15 +24,19 @@
 
 namespace ra {
 
-template <int D>
+// ROWS keys per tile: 128 (d = 128, and every paged tile, which is one page) or 256 (dense
+// d = 64, so that a tile carries as many bytes, and as much fixed per-tile work per byte, as a
+// d = 128 tile).
+template <int D, int ROWS>
 struct ScoreCfg {
   static constexpr int kThreads = 256;
   static constexpr int kWarps = 8;
-  static constexpr int kTile = kScoreTile;                 // keys per tile (16 per warp)
+  static constexpr int kTile = ROWS;                       // keys per tile
+  static constexpr int kGroups = ROWS / 128;               // 16-key MMA row groups per warp
   static constexpr int kBoxes = D / 64;                    // 64-channel boxes per tile
-  static constexpr int kBoxBytes = kTile * 128;            // 16 KB
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;    // 32 KB (d=128) / 16 KB (d=64)
-  static constexpr int kStages = D == 128 ? 5 : 8;
+  static constexpr int kBoxBytes = kTile * 128;            // 16 KB per 128 rows
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;    // 32 KB (d=128 or 256 rows) / 16 KB
+  static constexpr int kStages = kTileBytes == 32768 ? 5 : 8;
   static constexpr size_t smem_bytes(int G) {
     return 1024 + static_cast<size_t>(kStages) * kTileBytes +
            static_cast<size_t>(G) * kHistBins * 4 + kStages * 8;
@@ -48,14 +52,14 @@ __device__ __forceinline__ long long seq_n(const ScoreParams &p, const NoPaging 
 __device__ __forceinline__ long long seq_n(const ScoreParams &p, const PagedInfo &pg, long long bg) {
   return pg.seq_len[bg / p.Hkv];
 }
-// The head and first key of flattened tile t (tiles ordered by head, then key).
+// The head and first key of flattened tile t (tiles ordered by head, then key; rows keys each).
 __device__ __forceinline__ void tile_start(const ScoreParams &p, const NoPaging &, long long t,
-                                           long long &bg, long long &key) {
+                                           long long &bg, long long &key, int rows) {
   bg = t / p.tiles_per_head;
-  key = (t - bg * p.tiles_per_head) * kScoreTile;
+  key = (t - bg * p.tiles_per_head) * rows;
 }
 __device__ __forceinline__ void tile_start(const ScoreParams &p, const PagedInfo &pg, long long t,
-                                           long long &bg, long long &key) {
+                                           long long &bg, long long &key, int) {
   int b = 0;
   while (b + 1 < p.B && pg.tile_off[b + 1] <= t) ++b;   // once per CTA
   const long long per_head = (pg.seq_len[b] + kScoreTile - 1) / kScoreTile;
@@ -92,10 +96,10 @@ __device__ __forceinline__ void cand_range(const ScoreParams &p, const PagedInfo
   hist = p.do_hist != 0 && k_eff > 0 && k_eff < hi - lo;
 }
 
-template <int D, class Pg>
+template <int D, int ROWS, class Pg>
 __global__ void __launch_bounds__(256, 1)
     score_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const ScoreParams p, const Pg pg) {
-  using C = ScoreCfg<D>;
+  using C = ScoreCfg<D, ROWS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t tiles = (raw + 1023u) & ~1023u;          // swizzled boxes need 1024-byte alignment
@@ -125,7 +129,7 @@ __global__ void __launch_bounds__(256, 1)
 
   // load cursor (thread 0 only) and compute cursor (all threads)
   long long bg0, key0;
-  tile_start(p, pg, t_begin, bg0, key0);
+  tile_start(p, pg, t_begin, bg0, key0, C::kTile);
   long long l_bg = bg0, l_key = key0;
   long long c_bg = bg0, c_key = key0;
   const uint64_t pol = policy_evict_first();
@@ -165,7 +169,8 @@ __global__ void __launch_bounds__(256, 1)
   bool cur_hist = false;
   uint32_t bq[D / 16][2];
   const int mat = lane >> 3;
-  const int arow = warp * 16 + (lane & 7) + (mat & 1) * 8;   // ldmatrix source row
+  // ldmatrix source row of group gi: warp * (16 kGroups) + 16 gi + (lane & 7) + 8 (mat & 1)
+  const int arow0 = warp * 16 * C::kGroups + (lane & 7) + (mat & 1) * 8;
   const int g4 = lane >> 2;
   const int t4 = lane & 3;
   int j = 0;
@@ -217,32 +222,36 @@ __global__ void __launch_bounds__(256, 1)
       }
       __syncthreads();
     }
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f};
-    float acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int kk = 0; kk < D / 16; kk += 2) {
-      // logical 16-byte chunk c of row r lives in box c / 8 at swizzled chunk (c % 8) ^ (r % 8)
-      const int c0 = 2 * kk + (mat >> 1);
-      const int c1 = c0 + 2;
-      uint32_t a[4], a2[4];
-      ldmatrix_x4(tbase + (c0 >> 3) * C::kBoxBytes + arow * 128 + (((c0 & 7) ^ (arow & 7)) << 4),
-                  a[0], a[1], a[2], a[3]);
-      ldmatrix_x4(tbase + (c1 >> 3) * C::kBoxBytes + arow * 128 + (((c1 & 7) ^ (arow & 7)) << 4),
-                  a2[0], a2[1], a2[2], a2[3]);
-      mma_bf16_16816(acc0, a, bq[kk][0], bq[kk][1]);
-      mma_bf16_16816(acc1, a2, bq[kk + 1][0], bq[kk + 1][1]);
-    }
+    for (int gi = 0; gi < C::kGroups; ++gi) {
+      const int arow = arow0 + 16 * gi;
+      float acc0[4] = {0.f, 0.f, 0.f, 0.f};
+      float acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kk = 0; kk < D / 16; kk += 2) {
+        // logical 16-byte chunk c of row r lives in box c / 8 at swizzled chunk (c % 8) ^ (r % 8)
+        const int c0 = 2 * kk + (mat >> 1);
+        const int c1 = c0 + 2;
+        uint32_t a[4], a2[4];
+        ldmatrix_x4(tbase + (c0 >> 3) * C::kBoxBytes + arow * 128 + (((c0 & 7) ^ (arow & 7)) << 4),
+                    a[0], a[1], a[2], a[3]);
+        ldmatrix_x4(tbase + (c1 >> 3) * C::kBoxBytes + arow * 128 + (((c1 & 7) ^ (arow & 7)) << 4),
+                    a2[0], a2[1], a2[2], a2[3]);
+        mma_bf16_16816(acc0, a, bq[kk][0], bq[kk][1]);
+        mma_bf16_16816(acc1, a2, bq[kk + 1][0], bq[kk + 1][1]);
+      }
 
-    // C fragment: e = 0,1 -> key g4, heads 2t4, 2t4+1; e = 2,3 -> key g4 + 8
+      // C fragment: e = 0,1 -> key g4, heads 2t4, 2t4+1; e = 2,3 -> key g4 + 8
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int h = 2 * t4 + (e & 1);
-      const long long key = c_key + warp * 16 + g4 + (e >> 1) * 8;
-      if (h < p.G && key < cur_n) {
-        const float z = canon_zero((acc0[e] + acc1[e]) * p.scale);
-        p.S[(rowbase + h) * p.ldS + key] = z;
-        if (cur_hist && key >= cur_lo && key < cur_hi)
-          atomicAdd(&hist_s[h * kHistBins + (order_key(z) >> (32 - kHistBits))], 1u);
+      for (int e = 0; e < 4; ++e) {
+        const int h = 2 * t4 + (e & 1);
+        const long long key = c_key + warp * 16 * C::kGroups + 16 * gi + g4 + (e >> 1) * 8;
+        if (h < p.G && key < cur_n) {
+          const float z = canon_zero((acc0[e] + acc1[e]) * p.scale);
+          p.S[(rowbase + h) * p.ldS + key] = z;
+          if (cur_hist && key >= cur_lo && key < cur_hi)
+            atomicAdd(&hist_s[h * kHistBins + (order_key(z) >> (32 - kHistBits))], 1u);
+        }
       }
     }
     c_key += C::kTile;
@@ -265,12 +274,12 @@ __global__ void __launch_bounds__(256, 1)
   if (cur_bg >= 0 && cur_hist) flush_hist(cur_bg);
 }
 
-template <int D, class Pg>
+template <int D, int ROWS, class Pg>
 static cudaError_t launch_score_t(const ScoreParams &p, const Pg &pg, long long num_pages,
                                   cudaStream_t s) {
-  using C = ScoreCfg<D>;
+  using C = ScoreCfg<D, ROWS>;
   static bool done[64] = {};
-  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D, Pg>),
+  cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(score_gqa_kernel<D, ROWS, Pg>),
                                     static_cast<int>(C::smem_bytes(kMaxGroup)), done);
   if (e != cudaSuccess) return e;
   CUtensorMap tm;
@@ -284,19 +293,26 @@ static cudaError_t launch_score_t(const ScoreParams &p, const Pg &pg, long long 
   long long grid = num_sms();
   if (grid > p.total_tiles) grid = p.total_tiles;
   if (grid < 1) grid = 1;
-  return launch_pdl(score_gqa_kernel<D, Pg>, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads),
-                    C::smem_bytes(p.G), s, tm, p, pg);
+  return launch_pdl(score_gqa_kernel<D, ROWS, Pg>, dim3(static_cast<unsigned>(grid)),
+                    dim3(C::kThreads), C::smem_bytes(p.G), s, tm, p, pg);
 }
+
+int score_tile_rows(int d) { return d == 64 ? 256 : 128; }
 
 cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s) {
   const NoPaging pg{};
-  return d == 128 ? launch_score_t<128>(p, pg, 0, s) : launch_score_t<64>(p, pg, 0, s);
+  // the tile count follows the tile size of this head dimension
+  ScoreParams q = p;
+  const int rows = score_tile_rows(d);
+  q.tiles_per_head = (p.N + rows - 1) / rows;
+  q.total_tiles = q.tiles_per_head * p.B * p.Hkv;
+  return d == 128 ? launch_score_t<128, 128>(q, pg, 0, s) : launch_score_t<64, 256>(q, pg, 0, s);
 }
 
 cudaError_t launch_score_paged(const ScoreParams &p, const PagedInfo &pg, long long num_pages, int d,
                                cudaStream_t s) {
-  return d == 128 ? launch_score_t<128>(p, pg, num_pages, s)
-                  : launch_score_t<64>(p, pg, num_pages, s);
+  return d == 128 ? launch_score_t<128, 128>(p, pg, num_pages, s)
+                  : launch_score_t<64, 128>(p, pg, num_pages, s);
 }
 
 }  // namespace ra
