@@ -45,7 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 # keyed by the sha256 of the score kernel's own sources (score.cu and its TMA helpers) it was
 # taken on, so a changed kernel reports null until it is captured again.  Values are per launch
 # of the named workload (profiles/score_gqa_l8b_128k.md).
-TRAFFIC = {("4854c3ab29ddd3bd", "l8b_128k_k1pct"): 275.59e6}
+TRAFFIC = {("8c722343be687c83", "l8b_128k_k1pct"): 276.25e6}
 
 
 def score_source_hash() -> str:
