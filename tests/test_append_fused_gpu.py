@@ -54,6 +54,8 @@ def _both_paths(q, K, V, k, n_sink, n_window):
     (5000, 64, 100, 16, 64),    # a middle row, d = 64
     (1, 128, 5, 4, 16),         # an empty cache: the token is the whole step
     (4097, 128, 300, 8, 0),     # no window: the token is a candidate
+    (256, 64, 20, 4, 16),       # d = 64 scans 256-key tiles: row 255 of the first tile
+    (257, 64, 20, 4, 16),       # row 0 of the second 256-key tile
 ])
 def test_fused_append_equals_append_then_decode_and_the_oracle(N, d, k, n_sink, n_window):
     B, Hq, Hkv = 2, 8, 2
