@@ -256,7 +256,8 @@ ra_status ra_decode_step_static(const ra_kv *kv, const void *q, int32_t Hq, int3
  * min(k, |C|) largest z_i = q[b,h,m] . K[b,h/G,i] / sqrt(d) over the candidates C = [0,N) \ W,
  * ties to the lower position (the decode step's selection, one query at a time; no causal mask).
  * These are the nearest-key lists the slides build the query-aware index from (slide
- * "Query-aware index construction": prefill queries and their top-k keys).  With G * M query
+ * "Prefill queries teach the key graph what matters": prefill queries and their top-k keys,
+ * found on the GPU).  With G * M query
  * rows per KV head the scores are a dense contraction, computed on the tcgen05 tensor cores
  * (bf16 x bf16 -> fp32 in tensor memory).
  *   q   : bf16 [B, Hq, M, d], device.   M >= 1, B * M <= 65535.

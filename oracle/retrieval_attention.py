@@ -100,8 +100,8 @@ def select_topk(z: np.ndarray, C: np.ndarray, k: int) -> np.ndarray:
 
 # ------------------------------------------------------------------------------------
 # softmax over a selected set, partial states and their merge
-# (slide "Two local softmax outputs need global weights", Eqs. (3)-(5), and the backup
-#  slide "The normalization identity", Appendix B)
+# (slide "Two local softmax outputs need global weights", Eqs. (3)-(5), and the
+#  slide "Backup: the normalization identity", Appendix B)
 
 
 def attend(z: np.ndarray, V: np.ndarray, U: np.ndarray) -> np.ndarray:
@@ -116,7 +116,7 @@ def attend(z: np.ndarray, V: np.ndarray, U: np.ndarray) -> np.ndarray:
 
 def partial_state(z: np.ndarray, V: np.ndarray, S: np.ndarray):
     """(m_S, Z_S, N_S) of one subset S: m_S = max z, Z_S = sum e^{z-m_S},
-    N_S = sum e^{z-m_S} v (backup slide, Appendix B).  o_S = N_S / Z_S."""
+    N_S = sum e^{z-m_S} v (slide "Backup: the normalization identity", Appendix B).  o_S = N_S / Z_S."""
     S = np.asarray(S, dtype=np.int64)
     zs = z[S]
     m = float(np.max(zs))

@@ -1,7 +1,7 @@
 // Merge of split partial softmax states, shared by the sparse and dense attention kernels.
 //
 // A partial state of subset S is (m_S, Z_S, N_S) with m_S = max z, Z_S = sum e^{z - m_S} and
-// N_S = sum e^{z - m_S} v (RetrievalAttention slides, backup slide "The normalization
+// N_S = sum e^{z - m_S} v (RetrievalAttention slides, slide "Backup: the normalization
 // identity", Appendix B).  Disjoint subsets merge to the exact softmax over their union:
 //   o = sum_S e^{m_S - m} N_S / sum_S e^{m_S - m} Z_S,  m = max_S m_S      (Eqs. (3)-(5)).
 // Layout of one state: [m, Z, pad, pad, N[0..D)], stride D + kPartPad floats (16-byte rows).
