@@ -70,9 +70,12 @@ struct __align__(16) SaSmem {
 // The index a selected entry e of row blockIdx.y is reported as in idx: its position in the
 // score row, or, for a candidate list (pos_map set), the cache position the list maps it to (-1:
 // a static-set key).  Read from the parameter block, so it costs the callers no registers.
+template <bool kFull>
 __device__ __forceinline__ int32_t idx_of(const SaParams &p, uint32_t e) {
-  return p.pos_map ? __ldcg(p.pos_map + static_cast<long long>(blockIdx.y) * p.ldS + e)
-                   : static_cast<int32_t>(e);
+  if constexpr (kFull) {
+    if (p.pos_map) return __ldcg(p.pos_map + static_cast<long long>(blockIdx.y) * p.ldS + e);
+  }
+  return static_cast<int32_t>(e);
 }
 
 __device__ __forceinline__ unsigned long long composite(uint32_t key, uint32_t pos) {
@@ -197,7 +200,7 @@ struct ChunkSrc {
 
 // Bitonic finish in the first CTA: the n <= kFinish keys in sm.fin, the `want` largest written
 // to irow[o0 ..].  One warp.
-template <int D>
+template <int D, bool kFull>
 __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm, uint32_t n,
                                                uint32_t want, int32_t *irow, uint32_t o0) {
   const int tid = threadIdx.x, lane = tid & 31;
@@ -207,7 +210,7 @@ __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm,
       uint32_t above = 0;
       for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, x, j) > x ? 1u : 0u;
       if (static_cast<uint32_t>(lane) < n && above < want)
-        irow[o0 + above] = idx_of(p, composite_pos(x));
+        irow[o0 + above] = idx_of<kFull>(p, composite_pos(x));
     }
     return;
   }
@@ -229,7 +232,7 @@ __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm,
         __syncwarp();
       }
     }
-    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = idx_of(p, composite_pos(sm.fin[i]));
+    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = idx_of<kFull>(p, composite_pos(sm.fin[i]));
   }
 }
 
@@ -271,7 +274,7 @@ __device__ int cluster_thresh(SaSmem<D> &sm, cg::cluster_group &cl, int rank, in
 // complete in every CTA's sm.h with the cluster synchronised since, then further 11-bit digits
 // of the composite.  `want` keys are still to be chosen; they go to irow[base ..).  Every CTA of
 // the cluster runs the same rounds (all decisions come from cluster-wide totals).
-template <int D, class Src>
+template <int D, bool kFull, class Src>
 __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank,
                               int ncl, const Src &src, uint32_t b1, uint32_t want, uint32_t base,
                               int32_t *irow, uint32_t k_eff) {
@@ -331,11 +334,11 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
       if ((x >> sh) != prefix) return;
       const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
       if (dg > t) {
-        if (ou < k_eff) irow[ou] = idx_of(p, composite_pos(x));
+        if (ou < k_eff) irow[ou] = idx_of<kFull>(p, composite_pos(x));
         ++ou;
       } else if (dg == t) {
         if (take_eq) {
-          if (base + up + oe < k_eff) irow[base + up + oe] = idx_of(p, composite_pos(x));
+          if (base + up + oe < k_eff) irow[base + up + oe] = idx_of<kFull>(p, composite_pos(x));
         } else if (fin && oe < static_cast<uint32_t>(kFinish)) {
           fin0[oe] = x;
         }
@@ -346,7 +349,8 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
     if (fin) {
       cl.sync();   // the final bucket is complete in the first CTA
       if (rank == 0)
-        bitonic_finish(p, sm, eq, min(want2, k_eff - min(k_eff, base + up)), irow, base + up);
+        bitonic_finish<D, kFull>(p, sm, eq, min(want2, k_eff - min(k_eff, base + up)), irow,
+                                 base + up);
       return;
     }
     // next digit: every remote read of sm.h came before the last barrier
@@ -462,8 +466,9 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
 struct RowGeo {
   long long N, s1, w0, nW, nC, k_eff, cbase, cper;
 };
+template <bool kFull>
 __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const NoPaging &, int row, int ncl) {
-  if (p.row_n) {   // a candidate list of its own length, no static set
+  if (kFull && p.row_n) {   // a candidate list of its own length, no static set
     RowGeo g;
     g.N = p.row_n[row];
     g.s1 = 0;
@@ -477,6 +482,7 @@ __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const NoPaging &, i
   }
   return RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, p.k_eff, p.cbase, p.cper};
 }
+template <bool kFull>
 __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const PagedInfo &pg, int row, int ncl) {
   RowGeo g;
   g.N = pg.seq_len[row / p.Hq];
@@ -492,10 +498,10 @@ __device__ __forceinline__ RowGeo row_geo(const SaParams &p, const PagedInfo &pg
 }
 // The geometry the attention uses: the row's own, except that a candidate list's Omega (the
 // min(k, candidates) entries of idx) is attended together with the cache's static set.
-template <class Pg>
+template <bool kFull, class Pg>
 __device__ __forceinline__ RowGeo attend_geo(const SaParams &p, const Pg &pg, int row, int ncl) {
-  RowGeo g = row_geo(p, pg, row, ncl);
-  if (p.row_n) g = RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, g.k_eff, p.cbase, p.cper};
+  RowGeo g = row_geo<kFull>(p, pg, row, ncl);
+  if (kFull && p.row_n) g = RowGeo{p.N, p.s1, p.w0, p.nW, p.nC, g.k_eff, p.cbase, p.cper};
   return g;
 }
 // Where token `pos` of sequence b, KV head gk, sits in V: v_base(...) + v_index(...) * d.
@@ -570,7 +576,7 @@ __device__ float row_logsumexp(const RowGeo &gm, SaSmem<D> &sm, cg::cluster_grou
 }
 
 // Omega of one query head into irow (cluster-wide; every CTA takes the same branches).
-template <int D>
+template <int D, bool kFull>
 __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
                              cg::cluster_group &cl, int rank, int ncl, int row) {
   const int tid = threadIdx.x;
@@ -589,9 +595,9 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     sm.n_sure = 0u;
     sm.n_list = 0u;
   }
-  const bool build = (p.mode & (kSaBuildHist | kSaEps)) != 0;
+  const bool build = kFull && (p.mode & (kSaBuildHist | kSaEps)) != 0;
   int b1i = -1;
-  if (p.mode & kSaEps) {
+  if (kFull && (p.mode & kSaEps)) {
     // Eq. (2)'s threshold: a_i > eps  <=>  z_i > T = ln(eps) + ln sum_j e^{z_j} (all N)
     const float T = p.log_eps + row_logsumexp(gm, sm, cl, rank, ncl, srow, lo, hi);
     // this CTA's digit-1 histogram of its candidates and its count of z > T
@@ -621,11 +627,11 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   }
   if (k_sel >= gm.nC) {   // every candidate is selected
     for (long long i = lo + tid; i < hi; i += kSaThreads)
-      irow[i - gm.s1] = idx_of(p, static_cast<uint32_t>(i));
+      irow[i - gm.s1] = idx_of<kFull>(p, static_cast<uint32_t>(i));
     return;
   }
   const uint32_t k_eff = static_cast<uint32_t>(k_sel);
-  if (p.mode & kSaEps) {
+  if (kFull && (p.mode & kSaEps)) {
     // b1 found above
   } else if (build) {
     // digit 1 from the scores themselves: this CTA's histogram, then the cluster's threshold
@@ -663,7 +669,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   // the keys above b1 take idx slots [0, above1), CTA by CTA
   if (sm.n_sure <= static_cast<uint32_t>(kSureCap)) {
     for (uint32_t i = tid; i < sm.n_sure; i += kSaThreads)
-      if (off + i < k_eff) irow[off + i] = idx_of(p, sm.sure[i]);
+      if (off + i < k_eff) irow[off + i] = idx_of<kFull>(p, sm.sure[i]);
   } else {   // more sure keys than sm.sure holds: from the chunk again
     uint32_t cu = 0;
     chunk.for_each([&](unsigned long long x) { cu += (x >> (64 - kHistBits)) > b1 ? 1u : 0u; });
@@ -672,13 +678,13 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     uint32_t o = off + inc.x - cu;
     chunk.for_each([&](unsigned long long x) {
       if ((x >> (64 - kHistBits)) > b1) {
-        if (o < k_eff) irow[o] = idx_of(p, composite_pos(x));
+        if (o < k_eff) irow[o] = idx_of<kFull>(p, composite_pos(x));
         ++o;
       }
     });
   }
   // the keys of b1, from the CTAs' lists
-  select_rounds(p, sm, cl, rank, ncl, ListSrc<D>{&sm, spill, sm.n_list}, b1, k_eff - above1,
+  select_rounds<D, kFull>(p, sm, cl, rank, ncl, ListSrc<D>{&sm, spill, sm.n_list}, b1, k_eff - above1,
                 above1, irow, k_eff);
 }
 
@@ -690,7 +696,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
 constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
 constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
 
-template <int D, class Pg>
+template <int D, bool kFull, class Pg>
 __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, SaSmem<D> &sm,
                              cg::cluster_group &cl, int rank, int ncl, int row) {
   constexpr int CPL = D / 32;   // channels per lane
@@ -703,7 +709,7 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   const long long e_hi = min(nU, e_lo + per);
   const int b = row / p.Hq, h = row - b * p.Hq;
   const __nv_bfloat16 *Vb = v_base<D>(p, pg, b, h / p.G);
-  const float *srow = (p.S_att ? p.S_att : p.S) + static_cast<long long>(row) * p.ldS;
+  const float *srow = ((kFull && p.S_att) ? p.S_att : p.S) + static_cast<long long>(row) * p.ldS;
   const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   int *spos = reinterpret_cast<int *>(sm.sure);   // staged: the entry's V row (-1: none)
   float *sz = reinterpret_cast<float *>(sm.sure + kStage);
@@ -855,7 +861,10 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   // no CTA reads another's shared memory after the exchange barrier: all may leave
 }
 
-template <int D, class Pg>
+// kFull = false: the plain decode step (the score kernel's histogram, the cache's own score rows
+// and positions); the threshold budget, the self-built histogram and candidate lists take the
+// kFull = true instantiation, so the plain one carries none of their code.
+template <int D, class Pg, bool kFull>
 __global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaParams p, const Pg pg) {
   __shared__ SaSmem<D> sm;
   cg::cluster_group cl = cg::this_cluster();
@@ -865,10 +874,11 @@ __global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaPa
   pdl_trigger();
   pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
   // each phase computes the row geometry afresh (nothing stays live across the selection)
-  if (p.mode & kSaSelect) select_phase<D>(p, row_geo(p, pg, row, ncl), sm, cl, rank, ncl, row);
+  if (p.mode & kSaSelect)
+    select_phase<D, kFull>(p, row_geo<kFull>(p, pg, row, ncl), sm, cl, rank, ncl, row);
   if (p.mode & kSaAttend) {
     if (p.mode & kSaSelect) cl.sync();   // Omega complete in idx (release/acquire at cluster scope)
-    attend_phase<D>(p, attend_geo(p, pg, row, ncl), pg, sm, cl, rank, ncl, row);
+    attend_phase<D, kFull>(p, attend_geo<kFull>(p, pg, row, ncl), pg, sm, cl, rank, ncl, row);
   } else {
     cl.sync();   // no CTA leaves while the cluster may still use its shared memory
   }
@@ -888,7 +898,7 @@ static int active_clusters_t(int ncl) {
   while ((1 << li) < ncl) ++li;
   if (!done[dev][li]) {
     if (ncl > 8)
-      (void)cudaFuncSetAttribute(select_attend_kernel<D, NoPaging>,
+      (void)cudaFuncSetAttribute(select_attend_kernel<D, NoPaging, false>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(ncl), 1);
@@ -901,7 +911,8 @@ static int active_clusters_t(int ncl) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, select_attend_kernel<D, NoPaging>, &cfg) != cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, select_attend_kernel<D, NoPaging, false>, &cfg) !=
+        cudaSuccess)
       n = 0;
     (void)cudaGetLastError();   // a refused query leaves no error behind
     cache[dev][li] = n;
@@ -924,12 +935,12 @@ int select_cluster_size(long long nC, int R, int d) {
   return n;
 }
 
-template <int D, class Pg>
-static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
+template <int D, class Pg, bool kFull>
+static cudaError_t launch_sa_k(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = 0;
   if (ncl > 8 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !attr_done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg>,
+    const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
                                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
@@ -949,7 +960,14 @@ static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D, Pg>, p, pg);
+  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D, Pg, kFull>, p, pg);
+}
+
+template <int D, class Pg>
+static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
+  const bool full = (p.mode & (kSaEps | kSaBuildHist)) != 0 || p.row_n != nullptr ||
+                    p.pos_map != nullptr || p.S_att != nullptr;
+  return full ? launch_sa_k<D, Pg, true>(p, pg, R, ncl, s) : launch_sa_k<D, Pg, false>(p, pg, R, ncl, s);
 }
 
 int attn_split(long long nU, int R, int ncl, int d) {
