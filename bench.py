@@ -42,17 +42,22 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one score-kernel launch, from an ncu capture,
-# keyed by the sha256 of the score kernel's own sources (score.cu and its TMA helpers) it was
-# taken on, so a changed kernel reports null until it is captured again.  Values are per launch
+# keyed by the hash of the score kernel's own sources (score.cu and its TMA helpers, comments
+# removed) it was taken on, so a changed kernel reports null until it is captured again.  Values are per launch
 # of the named workload (profiles/score_gqa_l8b_128k.md).
-TRAFFIC = {("8c722343be687c83", "l8b_128k_k1pct"): 276.25e6}
+TRAFFIC = {("f5d096058ed5c81b", "l8b_128k_k1pct"): 276.25e6}
 
 
 def score_source_hash() -> str:
+    """sha256 of the score kernel's sources with // comments and blank lines removed, so that
+    a comment edit keeps the key and any code edit changes it."""
     h = hashlib.sha256()
     for f in ("score.cu", "tma.cuh", "tmap.cu"):
-        with open(os.path.join(ROOT, "top_retrieval_attention_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "top_retrieval_attention_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -49,7 +49,7 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// 3-D tiled bulk tensor load global -> shared (no multicast), completion counted in bytes on
+// 3-D tiled bulk tensor load global -> shared (this CTA only), completion counted in bytes on
 // the mbarrier.  x is the innermost coordinate (in elements; x * 2 bytes is a multiple of 16).
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z,
                                             uint32_t bar, uint64_t policy) {
