@@ -21,10 +21,16 @@
 //     sent to the first CTA for a bitonic finish, or become the next round's domain;
 //   * a CTA with more sure keys than its shared array holds (very large k) writes them out from
 //     its chunk of the score row, re-read.
-// Attention: the CTAs split U (W first, then Omega from idx) into ranges; a warp takes 8
+// Attention: the CTAs split U (W first, then Omega from idx) into ranges; a warp takes 16
 // entries at a time (scores from the score row, V rows gathered 8 bytes per lane), keeps an
-// online-softmax state, the CTA combines its warps, and the first CTA merges the cluster's
-// partial states (m_S, Z_S, N_S) with weights e^{m_S - m} into the output.
+// online-softmax state, the CTA combines its warps, every CTA pushes its partial state
+// (m_S, Z_S, N_S) into the first CTA's shared memory, and the first CTA merges them with
+// weights e^{m_S - m} into the output.
+//
+// The same kernel selects from per-row candidate lists (IVF: row_n candidates per row, their
+// cache positions in pos_map) and builds its own digit-1 histogram or applies Eq. (2)'s
+// threshold when asked; those modes run a separate instantiation (kFull), so the decode step's
+// launches carry none of their code.
 #include <cooperative_groups.h>
 #include <math.h>
 
