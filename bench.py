@@ -495,9 +495,11 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 "algorithmic_bytes_per_launch": k_bytes,
                 "frac_of_nominal_8tbs": kscan_gbs / NOMINAL_HBM_GBS,
                 "score_kernel_sha": src_hash}
-    # the scan with the append inside it, then select + attention (threshold mode: append,
-    # score, select + attention)
-    launches_per_layer = 2 if fused else 3
+    # per layer: the scan with the append inside it, then select + attention, and the attention
+    # again as a launch of its own when it is split (the library's own plan); the threshold mode
+    # appends with a launch of its own
+    step_launches = sum(ra.lib().ra_decode_step_launches(B, Hq, Hkv, N, d, kl, w.n_sink, w.n_window)
+                        for kl in ks) + (0 if fused else L)
     result = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -512,7 +514,7 @@ def run_ours(args, w, rank, local_rank, world, dist):
         "step_frac_of_nominal_8tbs": step_gbs / NOMINAL_HBM_GBS,
         "score_kernel_us": 1000.0 * statistics.mean(score_ms),
         "phases_us_breakdown_pass": ph_us,
-        "gpu_launches": launches_per_layer * L * steps,
+        "gpu_launches": step_launches * steps,
         "clocks": clocks,
     }
     if kept is not None:

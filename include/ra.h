@@ -156,6 +156,15 @@ ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, con
                                 int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window,
                                 float *out, int32_t *idx, void *ws, size_t ws_bytes,
                                 ra_stream_t stream);
+/*
+ * Kernel launches that ra_decode_step (or ra_decode_step_append) makes for this shape: 2 (the
+ * scan, then the selection fused with the attention) or 3 (the attention split across several
+ * clusters per head, as a launch of its own).  Host only; it queries the current device's
+ * occupancy like the step itself.  -1 for a shape the step rejects.
+ */
+int32_t ra_decode_step_launches(int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
+                                int32_t k, int32_t n_sink, int32_t n_window);
+
 /* The scan phase of ra_decode_step_append alone (then ra_select_attend over the grown kv). */
 ra_status ra_score_gqa_append(ra_kv *kv, const void *q, const void *k_new, const void *v_new,
                               int32_t Hq, int32_t k, int32_t n_sink, int32_t n_window, void *ws,

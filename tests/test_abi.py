@@ -151,6 +151,14 @@ def test_fused_append_step_validates_before_launch():
     assert kv.N == 50   # no error grows the cache
 
 
+def test_launch_count_query():
+    n = ra.lib().ra_decode_step_launches(1, 32, 8, 131072, 128, 1310, 128, 512)
+    assert n in (2, 3)
+    assert ra.lib().ra_decode_step_launches(1, 32, 8, 131072, 96, 1310, 128, 512) == -1   # d
+    assert ra.lib().ra_decode_step_launches(1, 30, 8, 131072, 128, 1310, 128, 512) == -1  # Hq % Hkv
+    assert ra.lib().ra_decode_step_launches(1, 32, 8, 0, 128, 10, 4, 8) == -1             # N == 0
+
+
 def test_synth_constants_match_host_generator():
     from synth import gen
     a, b = sdev.constants()

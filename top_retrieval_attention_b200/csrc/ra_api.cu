@@ -320,6 +320,16 @@ ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, con
   return run_select_attend(&grown, st, kSaSelect | kSaAttend, idx, out, ws, cs);
 }
 
+int32_t ra_decode_step_launches(int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
+                                int32_t k, int32_t n_sink, int32_t n_window) {
+  Step st{};
+  if (plan_shape(B, Hq, Hkv, N, d, k, n_sink, n_window, st) != RA_OK) return -1;
+  if (N == 0 || st.nW + st.k_eff == 0) return -1;
+  plan_clusters(st);
+  // the scan, then selection + attention in one launch unless the attention is split
+  return attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d) == 1 ? 2 : 3;
+}
+
 ra_status ra_topk_select(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sink,
                          int32_t n_window, int32_t *idx, void *ws, size_t ws_bytes,
                          ra_stream_t stream) {

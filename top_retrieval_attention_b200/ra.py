@@ -25,7 +25,8 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_prefill_score", "ra_prefill_select", "ra_decode_step_eps", "ra_pyramid_budgets",
            "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step",
            "ra_ivf_build_workspace_bytes", "ra_ivf_build", "ra_ivf_search_workspace_bytes",
-           "ra_ivf_decode_step", "ra_decode_step_append", "ra_score_gqa_append")
+           "ra_ivf_decode_step", "ra_decode_step_append", "ra_score_gqa_append",
+           "ra_decode_step_launches")
 
 
 class ra_kv(ctypes.Structure):
@@ -111,6 +112,8 @@ def lib() -> ctypes.CDLL:
                                                 c_size_t, c_void_p]),
             "ra_score_gqa_append": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_int32, c_int32,
                                               c_int32, c_int32, c_void_p, c_size_t, c_void_p]),
+            "ra_decode_step_launches": (c_int32, [c_int32, c_int32, c_int32, c_int64, c_int32,
+                                                  c_int32, c_int32, c_int32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
