@@ -43,25 +43,12 @@ __device__ __forceinline__ float key_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-// ------------------------------------------------------------------ async copies
+// ------------------------------------------------------------------ shared-memory addresses
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// 16-byte global -> shared copy; src_bytes == 0 fills the 16 bytes with zeros.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
 
 // ------------------------------------------------------------------ tensor-core fragments
 
@@ -80,13 +67,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Swizzled byte offset of 16-byte chunk `c` of row `r` in a tile whose rows are `row_bytes`
-// long (128 or 256): the low three chunk bits are XORed with the row's low three bits, so
-// eight consecutive rows at one logical chunk hit eight distinct bank groups.
-__device__ __forceinline__ uint32_t swz(int r, int c, int row_bytes) {
-  return static_cast<uint32_t>(r * row_bytes + ((c ^ (r & 7)) << 4));
 }
 
 // ------------------------------------------------------------------ bf16 pairs
@@ -110,19 +90,6 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
-}
-
-// Warp-aggregated append: every lane with `pred` gets a distinct slot from *counter.
-__device__ __forceinline__ uint32_t warp_append(bool pred, uint32_t *counter, bool &ok) {
-  const uint32_t mask = __ballot_sync(0xffffffffu, pred);
-  ok = pred;
-  if (mask == 0) return 0;
-  const int leader = __ffs(mask) - 1;
-  const int lane = threadIdx.x & 31;
-  uint32_t base = 0;
-  if (lane == leader) base = atomicAdd(counter, static_cast<uint32_t>(__popc(mask)));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  return base + __popc(mask & lanemask_lt());
 }
 
 }  // namespace ra
