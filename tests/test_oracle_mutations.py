@@ -81,3 +81,35 @@ def test_unnormalised_attention_is_caught(monkeypatch):
         return w @ V[U]
     _patch(monkeypatch, "attend", bad)
     assert _fails(pins.test_dense_matches_torch_sdpa_fp64, 7, 128)
+
+
+# ---------------------------------------------------------------- IVF retrieval
+
+
+def test_ivf_probe_of_the_lowest_centroids_is_caught(monkeypatch):
+    def bad(q, centroids, nprobe):
+        zc = centroids @ q
+        return np.lexsort((np.arange(zc.size), zc))[:nprobe]
+    _patch(monkeypatch, "ivf_probe", bad)
+    assert _fails(pins.test_ivf_candidates_are_the_probed_clusters)
+
+
+def test_ivf_probe_ties_to_the_higher_cluster_are_caught(monkeypatch):
+    def bad(q, centroids, nprobe):
+        zc = centroids @ q
+        return np.lexsort((-np.arange(zc.size), -zc))[:nprobe]
+    _patch(monkeypatch, "ivf_probe", bad)
+    assert _fails(pins.test_ivf_candidates_are_the_probed_clusters)
+
+
+def test_ivf_candidates_not_restricted_to_c_are_caught(monkeypatch):
+    def bad(q_bits, K_bits, V_bits, pos, offsets, cent_bits, k, nprobe, n_sink, n_window):
+        q, K, V = ra.bf16_to_f64(q_bits), ra.bf16_to_f64(K_bits), ra.bf16_to_f64(V_bits)
+        z = ra.scores(q, K)
+        probe = ra.ivf_probe(q, ra.bf16_to_f64(cent_bits), nprobe)
+        cand = np.concatenate([pos[offsets[c]:offsets[c + 1]] for c in probe]).astype(np.int64)
+        omega = ra.select_topk(z, cand, k)                 # W keys left among the candidates
+        U = np.union1d(ra.static_set(K.shape[0], n_sink, n_window), omega)
+        return ra.attend(z, V, U), omega, z, probe
+    _patch(monkeypatch, "ivf_decode_head", bad)
+    assert _fails(pins.test_ivf_probing_every_cluster_is_exact_retrieval)
