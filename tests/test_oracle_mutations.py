@@ -113,3 +113,44 @@ def test_ivf_candidates_not_restricted_to_c_are_caught(monkeypatch):
         return ra.attend(z, V, U), omega, z, probe
     _patch(monkeypatch, "ivf_decode_head", bad)
     assert _fails(pins.test_ivf_probing_every_cluster_is_exact_retrieval)
+
+
+# ---------------------------------------------------------------- budgets and paging
+
+
+def test_threshold_weights_over_the_candidates_only_are_caught(monkeypatch):
+    def bad(z, C, k, eps):
+        C = np.asarray(C, dtype=np.int64)
+        a = np.exp(z[C] - z[C].max())
+        a = a / a.sum()                                   # softmax over C instead of all N
+        return ra.select_topk(z, C[a > eps], k)
+    _patch(monkeypatch, "select_threshold", bad)
+    assert _fails(pins.test_threshold_weights_use_the_full_softmax)
+
+
+def test_threshold_not_strict_is_caught(monkeypatch):
+    def bad(z, C, k, eps):
+        a = ra.softmax_weights(z)
+        C = np.asarray(C, dtype=np.int64)
+        return ra.select_topk(z, C[a[C] >= eps], k)      # a_i >= eps instead of a_i > eps
+    _patch(monkeypatch, "select_threshold", bad)
+    assert _fails(pins.test_threshold_two_keys_logistic_closed_form)
+
+
+def test_budgets_growing_with_depth_are_caught(monkeypatch):
+    good = ra.pyramid_budgets
+    _patch(monkeypatch, "pyramid_budgets", lambda L, k, r: good(L, k, r)[::-1].copy())
+    assert _fails(pins.test_pyramid_budgets_shape)
+
+
+def test_paged_gather_off_by_one_page_is_caught(monkeypatch):
+    def bad(pool, table, lens):
+        P = pool.shape[2]
+        out = []
+        for b, n in enumerate(lens):
+            rows = [pool[table[b][min(i // P + 1, table.shape[1] - 1)], :, i % P, :]
+                    for i in range(int(n))]
+            out.append(np.stack(rows, axis=1))
+        return out
+    _patch(monkeypatch, "gather_paged", bad)
+    assert _fails(pins.test_gather_paged_inverts_a_scatter_by_the_definition)
