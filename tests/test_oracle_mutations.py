@@ -154,3 +154,33 @@ def test_paged_gather_off_by_one_page_is_caught(monkeypatch):
         return out
     _patch(monkeypatch, "gather_paged", bad)
     assert _fails(pins.test_gather_paged_inverts_a_scatter_by_the_definition)
+
+
+def test_prefill_with_the_wrong_kv_head_is_caught(monkeypatch):
+    def bad(Q_bits, K_bits, k, n_sink, n_window):
+        B, Hq, M, _ = Q_bits.shape
+        Hkv, N = K_bits.shape[1], K_bits.shape[2]
+        C = ra.candidate_set(N, n_sink, n_window)
+        return [[[ra.select_topk(ra.prefill_score_matrix(Q_bits[b, h], K_bits[b, h % Hkv])[m],
+                                 C, k) for m in range(M)] for h in range(Hq)] for b in range(B)]
+    _patch(monkeypatch, "prefill_topk", bad)    # query head h reading KV head h % Hkv
+    assert any(_fails(pins.test_prefill_topk_brute_force, t) for t in range(6))
+
+
+def test_prefill_with_a_causal_mask_is_caught(monkeypatch):
+    def bad(Q_bits, K_bits, k, n_sink, n_window):
+        B, Hq, M, _ = Q_bits.shape
+        Hkv, N = K_bits.shape[1], K_bits.shape[2]
+        G = Hq // Hkv
+        C = ra.candidate_set(N, n_sink, n_window)
+        out = [[[None] * M for _ in range(Hq)] for _ in range(B)]
+        for b in range(B):
+            for h in range(Hq):
+                Z = ra.prefill_score_matrix(Q_bits[b, h], K_bits[b, h // G])
+                for m in range(M):   # query m of the last M positions sees keys up to N - M + m
+                    out[b][h][m] = ra.select_topk(Z[m], C[C <= N - M + m], k)
+        return out
+    _patch(monkeypatch, "prefill_topk", bad)
+    # (with the window covering the last M positions the mask removes no candidate; the tiny
+    # brute-force cases have windows of 0 or 1 token)
+    assert any(_fails(pins.test_prefill_topk_brute_force, t) for t in range(6))
