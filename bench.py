@@ -43,8 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one score-kernel launch, from an ncu capture,
 # keyed by the hash of the score kernel's own sources (score.cu and its TMA helpers, comments
-# removed) it was taken on, so a changed kernel reports null until it is captured again.  Values are per launch
-# of the named workload (profiles/score_gqa_l8b_128k.md).
+# removed) it was taken on, so a changed kernel reports null until it is captured again.  Values
+# are per launch of the named workload (the score-kernel ncu summary under profiles/).
 TRAFFIC = {("f5d096058ed5c81b", "l8b_128k_k1pct"): 276.25e6}
 
 
@@ -327,9 +327,18 @@ def run_ours(args, w, rank, local_rank, world, dist):
         c = caches[layer]
         kv = c.kv
         kl = ks[layer]
+        if ev is None and args.eps <= 0:
+            # the product call: the scan (with the token's append inside it), and the selection
+            # + attention launched behind it, starting on each KV head as the scan finishes it
+            ra.check(ra.ra_decode_step_append(kv, qptr, knew[layer].data_ptr(), vnew[layer].data_ptr(),
+                                              Hq, kl, w.n_sink, w.n_window, outs[layer].data_ptr(),
+                                              idxs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp),
+                     "decode_step_append")
+            c.N = N - 1
+            return
         if ev is not None:
             ev[0].record(stream)
-        if args.eps <= 0:   # the append runs inside the scan (one launch), then select + attend
+        if args.eps <= 0:   # the phases launched apart: the scan alone, then select + attend
             ra.check(ra.ra_score_gqa_append(kv, qptr, knew[layer].data_ptr(), vnew[layer].data_ptr(),
                                             Hq, kl, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes,
                                             sp), "score_append")
@@ -368,41 +377,6 @@ def run_ours(args, w, rank, local_rank, world, dist):
         for layer in range(L):
             phases(layer, qpool[s % P, layer].data_ptr(), None if evs is None else evs[layer])
 
-    def step_score_probe(s, ev):
-        """One step with events around each score launch only (the dominant kernel)."""
-        for layer in range(L):
-            c = caches[layer]
-            kv = c.kv
-            kl = ks[layer]
-            qptr = qpool[s % P, layer].data_ptr()
-            if args.eps <= 0:   # the scan with the append inside it, timed alone
-                ev[layer][0].record(stream)
-                ra.check(ra.ra_score_gqa_append(kv, qptr, knew[layer].data_ptr(),
-                                                vnew[layer].data_ptr(), Hq, kl, w.n_sink,
-                                                w.n_window, ws.data_ptr(), ws_bytes, sp),
-                         "score_append")
-                ev[layer][1].record(stream)
-                ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window,
-                                             idxs[layer].data_ptr(), outs[layer].data_ptr(),
-                                             ws.data_ptr(), ws_bytes, sp), "select_attend")
-                c.N = N - 1
-                continue
-            ra.check(ra.ra_append_kv(kv, knew[layer].data_ptr(), vnew[layer].data_ptr(), 1, sp), "append")
-            if args.eps > 0:   # the score kernel runs inside the one call: time the whole call
-                ev[layer][0].record(stream)
-                ra.check(ra.ra_decode_step_eps(kv, qptr, Hq, kl, args.eps, w.n_sink, w.n_window,
-                                               outs[layer].data_ptr(), idxs[layer].data_ptr(),
-                                               ws.data_ptr(), ws_bytes, sp), "decode_step_eps")
-                ev[layer][1].record(stream)
-                c.N = N - 1
-                continue
-            ev[layer][0].record(stream)
-            ra.check(ra.ra_score_gqa(kv, qptr, Hq, kl, w.n_sink, w.n_window, ws.data_ptr(), ws_bytes, sp), "score")
-            ev[layer][1].record(stream)
-            ra.check(ra.ra_select_attend(kv, Hq, kl, w.n_sink, w.n_window, idxs[layer].data_ptr(),
-                                         outs[layer].data_ptr(), ws.data_ptr(), ws_bytes, sp), "select_attend")
-            c.N = N - 1
-
     # warm-up, then (for short timed regions) an untimed soak so clocks reach steady state
     for s in range(max(3, args.warmup)):
         step(s)
@@ -413,8 +387,6 @@ def run_ours(args, w, rank, local_rank, world, dist):
     torch.cuda.synchronize()
     est = max((time.perf_counter() - t0) / 5, 1e-6)
     steps = args.steps if args.steps is not None else max(10, min(20000, int(1.0 / est)))
-    sev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(L)]
-           for _ in range(steps)]
     t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = None
     try:
@@ -434,20 +406,20 @@ def run_ours(args, w, rank, local_rank, world, dist):
     torch.cuda.synchronize()
     t_start.record(stream)
     for s in range(steps):
-        step_score_probe(s, sev[s])
+        step(s)
     t_stop.record(stream)
     torch.cuda.synchronize()
     barrier(dist, local_rank)
     clocks = clk.stop()
     elapsed_ms = t_start.elapsed_time(t_stop)
     elapsed_ms = max_over_ranks(dist, elapsed_ms, dev)
-    score_ms = [sev[s][layer][0].elapsed_time(sev[s][layer][1]) for s in range(steps)
-                for layer in range(L)]
     ms_per_step = elapsed_ms / steps
     value = world * steps / (elapsed_ms / 1000.0)
 
-    # phase breakdown (diagnostic, not the timed region): events between every kernel phase,
-    # which also removes the programmatic-launch overlap at each boundary
+    # phase pass right after the timed region: the same launches with events between the
+    # phases, which also removes the overlap of the selection with the scan.  It gives the score
+    # kernel's own duration (the roofline: inside the step the selection runs beside the scan,
+    # so events cannot separate the two there) and the phase breakdown.
     psteps = min(steps, 2000)
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(L)]
            for _ in range(psteps)]
@@ -468,6 +440,7 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 ph["score"].append(e[1].elapsed_time(e[2]))
             ph["select_attend"].append(e[2].elapsed_time(e[3]))
     ph_us = {kk: 1000.0 * statistics.mean(v) for kk, v in ph.items()}
+    score_ms = ph["score_with_append"] if fused else ph["score"]
 
     # algorithmic bytes: K once per KV head, plus the V rows of U per query head
     s1 = min(w.n_sink, N)
@@ -494,7 +467,11 @@ def run_ours(args, w, rank, local_rank, world, dist):
                 "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
                 "algorithmic_bytes_per_launch": k_bytes,
                 "frac_of_nominal_8tbs": kscan_gbs / NOMINAL_HBM_GBS,
-                "score_kernel_sha": src_hash}
+                "score_kernel_sha": src_hash,
+                "duration_from": ("the phase pass after the timed region: CUDA events around "
+                                  "each launch, on the launching stream, in the step's own "
+                                  "launch configuration (in the timed step the selection runs "
+                                  "beside the scan)")}
     # per layer: the scan with the append inside it, then select + attention, and the attention
     # again as a launch of its own when it is split (the library's own plan); the threshold mode
     # appends with a launch of its own

@@ -48,6 +48,11 @@ struct ScoreParams {
   // that tile writes to the cache and patches into its staged tile before scoring it.
   const __nv_bfloat16 *k_new, *v_new;
   __nv_bfloat16 *K_cache, *V_cache;
+  // Completion counters (null: none): when a CTA is done with every tile of the head bg that it
+  // scores, it adds 1 to ready[bg * ready_stride] (after its score and histogram writes of that
+  // head are visible device-wide), so a kernel running concurrently can start on that head.
+  uint32_t *ready;
+  long long ready_stride;
 };
 
 // Paged KV caches: K and V in pages of kPageSize tokens, [num_pages, Hkv, kPageSize, d]; sequence
@@ -78,7 +83,7 @@ constexpr uint32_t kErrSelect = 4u;    // error bit: the selection's counts were
 struct SaParams {
   const float *S;           // [B*Hq, ldS] scores
   uint32_t *hist;           // [B*Hq, kHistBins] digit-1 histogram (left zero by the select)
-  uint2 *list;              // [B*Hq, ldL] (position, order key) of the threshold-bin keys
+  unsigned long long *list; // [B*Hq, ldL] composites (order key << 32 | ~position) of threshold-bin keys
   const __nv_bfloat16 *V;   // [B, Hkv, cap, d]
   int32_t *idx;             // [B*Hq, k]: written (select) or read (attention only)
   float *out;               // [B*Hq, d]
@@ -96,7 +101,14 @@ struct SaParams {
   const int32_t *pos_map;   // with row_n: [B*Hq, ldS] cache position of each candidate (-1: a
                             // static-set key); idx reports these positions
   const float *S_att;       // with row_n: [B*Hq, ldS] full-length score rows for the attention
+  // Overlap with the score kernel (null: none; the kernel waits for its predecessor instead):
+  // the cluster of row r starts once ready[(r / G) * ready_stride] reaches ready_target (every
+  // score CTA is done with that KV head), and the row group's last cluster sets it back to 0.
+  uint32_t *ready;
+  long long ready_stride;
+  uint32_t ready_target;
 };
+constexpr uint32_t kErrReadyWait = 16u;   // error bit: a head's scores never became ready
 
 // Scores of prefill queries (rows (b, h, m) of Q [B, Hq, M, d]) against the keys of their KV
 // head, on the tensor cores.
@@ -172,9 +184,14 @@ size_t counter_block_bytes(size_t rows);
 // including launches inside a stream capture, make no attribute call).
 cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]);
 
-cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s);
+// CTAs of a score launch over `total_tiles` tiles.
+int score_grid(long long total_tiles);
+// Bytes of static shared memory of one selection CTA (a score CTA leaves room for one).
+size_t select_smem_bytes(int d);
+// grid (optional): the launch's CTA count, the value a selection overlapping it waits for.
+cudaError_t launch_score(const ScoreParams &p, int d, cudaStream_t s, int *grid = nullptr);
 cudaError_t launch_score_paged(const ScoreParams &p, const PagedInfo &pg, long long num_pages, int d,
-                               cudaStream_t s);
+                               cudaStream_t s, int *grid = nullptr);
 // Cluster size for one query head: a power of two <= kMaxCluster (16 only where the device
 // schedules 16-CTA clusters of this kernel), chunks of at most 64K scores, grown to fill the GPU.
 int select_cluster_size(long long nC, int R, int d);

@@ -40,6 +40,11 @@ cudaError_t ensure_smem_limit(const void *kernel, int bytes, bool (&done)[64]) {
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // the largest shared-memory carveout, so that an SM running this kernel's CTA keeps room for
+  // a CTA of a kernel launched behind it (the selection beside the scan)
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }
@@ -129,9 +134,18 @@ static ra_status plan_step(const ra_kv *kv, int Hq, int k, int n_sink, int n_win
 
 static uint8_t *at(void *ws, size_t off) { return static_cast<uint8_t *>(ws) + off; }
 
+// Per-KV-head completion counters of an overlapped step: the meta words (slots 0 and 1) of the
+// head group's first query head.
+static uint32_t *ready_counters(void *ws, const Step &st) {
+  return reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
+}
+static long long ready_stride(const Step &st) { return static_cast<long long>(st.G) * kMetaWords; }
+
+// The scan.  With `overlap` set, the score CTAs publish each KV head as they finish it and
+// *overlap receives the count a selection waiting on them needs (the launch's CTA count).
 static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void *ws,
                            cudaStream_t stream, bool hist = true, const void *k_new = nullptr,
-                           const void *v_new = nullptr) {
+                           const void *v_new = nullptr, uint32_t *overlap = nullptr) {
   ScoreParams p{};
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -151,21 +165,29 @@ static ra_status run_score(const ra_kv *kv, const void *q, const Step &st, void 
     p.K_cache = static_cast<__nv_bfloat16 *>(kv->K);
     p.V_cache = static_cast<__nv_bfloat16 *>(kv->V);
   }
-  const cudaError_t e = launch_score(p, st.d, stream);
+  if (overlap != nullptr) {
+    p.ready = ready_counters(ws, st);
+    p.ready_stride = ready_stride(st);
+  }
+  int grid = 0;
+  const cudaError_t e = launch_score(p, st.d, stream, &grid);
+  if (overlap != nullptr) *overlap = static_cast<uint32_t>(grid);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "score");
 }
 
 // Selection (kSaSelect), attention (kSaAttend) or both.  Both run in one launch unless the
 // attention is large enough to want more clusters per head than the selection uses (then it is
 // a second launch with nsplit clusters per head).
+// ready_target > 0: the preceding scan publishes its KV heads (run_score with `overlap`), and
+// the selection launch starts on each head as soon as its counter reaches ready_target.
 static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, int32_t *idx,
                                    float *out, void *ws, cudaStream_t stream,
-                                   float log_eps = 0.f) {
+                                   float log_eps = 0.f, uint32_t ready_target = 0) {
   if (mode == kSaSelect && st.k == 0) return RA_OK;
   SaParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
   p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
-  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
+  p.list = reinterpret_cast<unsigned long long *>(at(ws, st.off_list));
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.idx = idx;
   p.out = out;
@@ -182,10 +204,16 @@ static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, in
     // the attention joins the launch when it can
     p.mode = split == 1 ? mode : (mode & ~kSaAttend);
     p.nsplit = 1;
+    if (ready_target > 0) {
+      p.ready = ready_counters(ws, st);
+      p.ready_stride = ready_stride(st);
+      p.ready_target = ready_target;
+    }
     const cudaError_t e = launch_select_attend(p, st.d, st.R, st.ncl, stream);
     if (e != cudaSuccess) return cuda_fail(e, "select_attend");
     if (p.mode == mode) return RA_OK;
   }
+  p.ready = nullptr;
   p.mode = kSaAttend;
   p.log_eps = 0.f;
   p.nsplit = split;
@@ -314,10 +342,11 @@ ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, con
   if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
   if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  s = run_score(&grown, q, st, ws, cs, true, k_new, v_new);
+  uint32_t target = 0;
+  s = run_score(&grown, q, st, ws, cs, true, k_new, v_new, &target);
   if (s != RA_OK) return s;
   kv->N = grown.N;   // the token is in the cache once the scan has run
-  return run_select_attend(&grown, st, kSaSelect | kSaAttend, idx, out, ws, cs);
+  return run_select_attend(&grown, st, kSaSelect | kSaAttend, idx, out, ws, cs, 0.f, target);
 }
 
 int32_t ra_decode_step_launches(int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
@@ -371,9 +400,10 @@ ra_status ra_decode_step(const ra_kv *kv, const void *q, int32_t Hq, int32_t k, 
   if (!q || !aligned16(q) || !out || !aligned16(out)) return RA_ERR_ARG;
   if (k > 0 && (!idx || !aligned16(idx))) return RA_ERR_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  s = run_score(kv, q, st, ws, cs);
+  uint32_t target = 0;
+  s = run_score(kv, q, st, ws, cs, true, nullptr, nullptr, &target);
   if (s != RA_OK) return s;
-  return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws, cs);
+  return run_select_attend(kv, st, kSaSelect | kSaAttend, idx, out, ws, cs, 0.f, target);
 }
 
 // ---- paged caches
@@ -447,7 +477,7 @@ static ra_status run_prefill_select(const Step &st, int32_t *idx, void *ws, cuda
   SaParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
   p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
-  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
+  p.list = reinterpret_cast<unsigned long long *>(at(ws, st.off_list));
   p.idx = idx;
   p.part = reinterpret_cast<float *>(at(ws, st.off_part));
   p.meta = reinterpret_cast<uint32_t *>(at(ws, st.off_meta));
@@ -654,6 +684,7 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
   PagedInfo pg{};
   fill_paged_info(kv, k, n_sink, n_window, pg);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int grid = 0;
   {
     ScoreParams p{};
     p.K = static_cast<const __nv_bfloat16 *>(kv->K);
@@ -666,13 +697,15 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
     p.scale = 1.0f / sqrtf(static_cast<float>(st.d));
     p.do_hist = k > 0;   // each head decides from its own length
     p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
-    const cudaError_t e = launch_score_paged(p, pg, kv->num_pages, st.d, cs);
+    p.ready = ready_counters(ws, st);   // the selection starts on each head as it is scored
+    p.ready_stride = ready_stride(st);
+    const cudaError_t e = launch_score_paged(p, pg, kv->num_pages, st.d, cs, &grid);
     if (e != cudaSuccess) return cuda_fail(e, "paged_score");
   }
   SaParams p{};
   p.S = reinterpret_cast<const float *>(at(ws, st.off_S));
   p.hist = reinterpret_cast<uint32_t *>(at(ws, st.off_hist));
-  p.list = reinterpret_cast<uint2 *>(at(ws, st.off_list));
+  p.list = reinterpret_cast<unsigned long long *>(at(ws, st.off_list));
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.idx = idx;
   p.out = out;
@@ -684,9 +717,13 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
   const int split = attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d);
   p.mode = split == 1 ? (kSaSelect | kSaAttend) : kSaSelect;
   p.nsplit = 1;
+  p.ready = ready_counters(ws, st);
+  p.ready_stride = ready_stride(st);
+  p.ready_target = static_cast<uint32_t>(grid);
   cudaError_t e = launch_select_attend_paged(p, pg, st.d, st.R, st.ncl, cs);
   if (e != cudaSuccess) return cuda_fail(e, "paged_select_attend");
   if (split > 1) {
+    p.ready = nullptr;
     p.mode = kSaAttend;
     p.nsplit = split;
     e = launch_select_attend_paged(p, pg, st.d, st.R, st.ncl, cs);
@@ -852,7 +889,7 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
   p.pos_map = v.pos_cand;
   p.row_n = v.n_cand;
   p.hist = reinterpret_cast<uint32_t *>(at(ws, L.st.off_hist));
-  p.list = reinterpret_cast<uint2 *>(at(ws, L.st.off_list));
+  p.list = reinterpret_cast<unsigned long long *>(at(ws, L.st.off_list));
   p.V = static_cast<const __nv_bfloat16 *>(kv->V);
   p.idx = idx;
   p.out = out;

@@ -4,16 +4,18 @@
 // U = W u Omega; "Two local softmax outputs need global weights" -- Eqs. (3)-(5)).
 //
 // One thread-block cluster per query head (b, h); the cluster's CTAs split the head's
-// candidate positions C = [s1, w0) into contiguous chunks.
+// candidate positions C = [s1, w0) into contiguous chunks.  During a decode step the kernel is
+// launched behind the score kernel and starts on a head as soon as that head's scores are
+// complete (a per-KV-head counter), so it runs beside the scan of the remaining heads.
 //
 // Selection, a radix select over the 64-bit composite x = order_key(z) << 32 | ~position (all
 // keys distinct: larger z first, equal z to the lower position):
 //   * digit 1 (the top 11 bits of order_key) was histogrammed by the score kernel; every CTA
 //     finds the threshold bin b1 (the bin of the k-th largest key) from it;
 //   * one streaming pass over the CTA's chunk of scores keeps the positions of the keys above
-//     b1 ("sure") in shared memory, keeps the keys in b1 (the "list") in shared memory, past
-//     its capacity in the CTA's slice of a per-head list in the workspace, and histograms
-//     digit 2 of the list;
+//     b1 ("sure") in shared memory, keeps the composites of the keys in b1 (the "list") in
+//     shared memory, past its capacity in the CTA's slice of a per-head list in the workspace,
+//     and histograms digit 2 of the list;
 //   * each later digit is settled across the cluster: every CTA sums one slice of the CTAs'
 //     digit histograms through distributed shared memory, the threshold digit is found from
 //     the slice totals, keys above it are written out at offsets from a cluster-wide prefix
@@ -23,7 +25,7 @@
 //     its chunk of the score row, re-read.
 // Attention: the CTAs split U (W first, then Omega from idx) into ranges; a warp takes 16
 // entries at a time (scores from the score row, V rows gathered 8 bytes per lane), keeps an
-// online-softmax state, the CTA combines its warps, every CTA pushes its partial state
+// online softmax state, the CTA combines its warps, every CTA pushes its partial state
 // (m_S, Z_S, N_S) into the first CTA's shared memory, and the first CTA merges them with
 // weights e^{m_S - m} into the output.
 //
@@ -50,14 +52,14 @@ constexpr int kListSmem = 1536;   // keys in b1 kept in shared memory per CTA (t
 constexpr int kFinish = 64;       // bitonic finish size (one warp)
 constexpr int kStreamVec = 8;     // float4 score loads per thread in flight
 
-// The first CTA's threshold list doubles as the attention's exchange area: one D-float
+// The first CTA's digit histogram doubles as the attention's exchange area: one D-float
 // numerator per CTA of the cluster.
-static_assert(kMaxCluster * 128 * sizeof(float) <= kListSmem * sizeof(uint2), "exchange area");
+static_assert(kMaxCluster * 128 * sizeof(float) <= kHistBins * sizeof(uint32_t), "exchange area");
 
 template <int D>
 struct __align__(16) SaSmem {
-  uint32_t sure[kSureCap];
-  uint2 list[kListSmem];          // (position, order key) of the first keys in b1
+  uint32_t sure[kSureCap];        // positions of the keys above b1
+  unsigned long long list[kListSmem];   // composites of the first keys in b1
   float wacc[kSaWarps * D];       // attention: per-warp numerators
   uint32_t h[kHistBins];          // digit histogram of the current round (slice reduced in place)
   unsigned long long fin[kFinish];  // first CTA: keys of the final bucket
@@ -71,6 +73,7 @@ struct __align__(16) SaSmem {
   uint32_t n_sure, n_list;
   int t_bin;
   uint32_t t_above, t_cnt;
+  uint32_t x_ok;                  // the wait verdict, from the first CTA
 };
 
 // The index a selected entry e of row blockIdx.y is reported as in idx: its position in the
@@ -167,19 +170,17 @@ __device__ __forceinline__ void find_thresh(SaSmem<D> &sm, const uint32_t *src, 
   __syncthreads();
 }
 
-// The CTA's threshold-bin keys (position, order key): the first kListSmem in shared memory,
-// the rest in the CTA's slice of the head's list in the workspace (read back through L2).
+// The CTA's threshold-bin keys (composites): the first kListSmem in shared memory, the rest in
+// the CTA's slice of the head's list in the workspace (read back through L2).
 template <int D>
 struct ListSrc {
   const SaSmem<D> *sm;
-  const uint2 *spill;
+  const unsigned long long *spill;
   uint32_t n;
   template <class F>
   __device__ __forceinline__ void for_each(F f) const {
-    for (uint32_t i = threadIdx.x; i < n; i += kSaThreads) {
-      const uint2 e = i < static_cast<uint32_t>(kListSmem) ? sm->list[i] : __ldcg(spill + i);
-      f(composite(e.y, e.x));
-    }
+    for (uint32_t i = threadIdx.x; i < n; i += kSaThreads)
+      f(i < static_cast<uint32_t>(kListSmem) ? sm->list[i] : __ldcg(spill + i));
   }
 };
 
@@ -204,6 +205,26 @@ struct ChunkSrc {
   }
 };
 
+// Sorts the kFinish keys at f into descending order.  One warp (all 32 lanes).
+__device__ __forceinline__ void bitonic_desc64(unsigned long long *f) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll 1
+  for (int size = 2; size <= kFinish; size <<= 1) {
+#pragma unroll 1
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int i = 2 * stride * (lane / stride) + (lane % stride);
+      const int j = i + stride;
+      const unsigned long long a = f[i], b = f[j];
+      const bool desc = (i & size) == 0;
+      if (desc ? (a < b) : (a > b)) {
+        f[i] = b;
+        f[j] = a;
+      }
+      __syncwarp();
+    }
+  }
+}
+
 // Bitonic finish in the first CTA: the n <= kFinish keys in sm.fin, the `want` largest written
 // to irow[o0 ..].  One warp.
 template <int D, bool kFull>
@@ -223,21 +244,7 @@ __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm,
   for (uint32_t i = n + tid; i < kFinish; i += kSaThreads) sm.fin[i] = 0ull;   // below every key
   __syncthreads();
   if (tid < 32) {
-#pragma unroll 1
-    for (int size = 2; size <= kFinish; size <<= 1) {
-#pragma unroll 1
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const int i = 2 * stride * (lane / stride) + (lane % stride);
-        const int j = i + stride;
-        const unsigned long long a = sm.fin[i], b = sm.fin[j];
-        const bool desc = (i & size) == 0;
-        if (desc ? (a < b) : (a > b)) {
-          sm.fin[i] = b;
-          sm.fin[j] = a;
-        }
-        __syncwarp();
-      }
-    }
+    bitonic_desc64(sm.fin);
     for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = idx_of<kFull>(p, composite_pos(sm.fin[i]));
   }
 }
@@ -370,11 +377,25 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
   if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);   // unreachable for distinct keys
 }
 
-// Appends this lane's hit (if any) to sm.sure / sm.list with one shared atomic per list and
-// warp: all 32 lanes call it together.
+// The score at bit j of a thread's hit mask: element j % 4 of its (j / 4)-th loaded vector,
+// picked from registers (no dynamic indexing).
+__device__ __forceinline__ float pick_score(const float4 (&v)[kStreamVec], int j) {
+  float r = 0.f;
+#pragma unroll
+  for (int u = 0; u < kStreamVec; ++u) {
+    const int e = j - 4 * u;
+    r = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : e == 3 ? v[u].w : r;
+  }
+  return r;
+}
+
+// Appends this lane's hit (if any) with one shared atomic per list and warp: all 32 lanes call
+// it together.  Keys above b1 go to the sure array (positions); keys in b1 go to the list as
+// composites, past its capacity to `spill`, with their digit-2 histogram in sm.h.  The
+// counters keep counting past the capacities.
 template <int D>
-__device__ __forceinline__ void place_hit(SaSmem<D> &sm, uint2 *spill, bool has, uint32_t pos,
-                                          float z, uint32_t b1, uint32_t lt) {
+__device__ __forceinline__ void place_hit(SaSmem<D> &sm, unsigned long long *spill, bool has,
+                                          uint32_t pos, float z, uint32_t b1, uint32_t lt) {
   const uint32_t key = order_key(z);
   const uint32_t d1 = key >> (32 - kHistBits);
   const bool up = has && d1 > b1, eq = has && d1 == b1;
@@ -392,27 +413,23 @@ __device__ __forceinline__ void place_hit(SaSmem<D> &sm, uint2 *spill, bool has,
   }
   if (eq) {
     const uint32_t o = be + __popc(me & lt);
-    const uint2 ent = make_uint2(pos, key);
-    if (o < static_cast<uint32_t>(kListSmem)) sm.list[o] = ent;
-    else spill[o] = ent;
+    const unsigned long long x = composite(key, pos);
+    if (o < static_cast<uint32_t>(kListSmem)) sm.list[o] = x;
+    else spill[o] = x;
     atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
   }
 }
 
-// One pass over the CTA's candidates [lo, hi) of the score row: positions of keys above the
-// digit-1 threshold bin b1 go to sm.sure, keys in b1 to sm.list and, past its capacity, to
-// `spill` (room for hi - lo entries), with their digit-2 histogram in sm.h.  Hits (z >= zlo,
-// the bottom of bin b1) are a few percent of the keys: each thread makes a bit mask of its
-// hits with one compare per score, re-reads its first four hits (L1 or L2) with the loads in
-// flight together, and the warp places them in lock-step rounds; a lane with more hits places
-// the rest alone.  The counters keep counting past the capacities.
+// One pass over the CTA's candidates [lo, hi) of the score row, placing every key at or above
+// the bottom of the digit-1 threshold bin b1 (place_hit).  Hits are a few percent of the keys:
+// each thread makes a bit mask of its hits with one compare per score, and the warp places
+// them in lock-step rounds, each lane's score picked from its registers.
 template <int D>
-__device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, uint2 *spill,
-                                             long long a0, long long lo, long long hi,
-                                             uint32_t b1) {
+__device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
+                                             unsigned long long *spill, long long a0, long long lo,
+                                             long long hi, uint32_t b1) {
   constexpr long long kStep = 4LL * kSaThreads * kStreamVec;
   static_assert(4 * kStreamVec <= 32, "one mask bit per score");
-  constexpr int kPre = 4;
   const float zlo = key_float(b1 << (32 - kHistBits));
   const uint32_t lt = lanemask_lt();
   for (long long it = a0; it < hi; it += kStep) {
@@ -421,7 +438,7 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
 #pragma unroll
     for (int u = 0; u < kStreamVec; ++u) {
       const long long b = b0 + 4LL * kSaThreads * u;
-      v[u] = (b < hi && b + 4 > lo) ? __ldg(reinterpret_cast<const float4 *>(srow + b))
+      v[u] = (b < hi && b + 4 > lo) ? __ldcg(reinterpret_cast<const float4 *>(srow + b))
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const bool interior = it >= lo && it + kStep <= hi;
@@ -438,30 +455,12 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow, u
       }
       m |= bits << (4 * u);
     }
-    if (!__any_sync(0xffffffffu, m != 0u)) continue;
-    uint32_t pp[kPre];
-    float zz[kPre];
-    int np = 0;
-#pragma unroll
-    for (int r = 0; r < kPre; ++r) {
-      const int j = m ? __ffs(m) - 1 : 0;
-      pp[r] = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
-      np += m ? 1 : 0;
-      m &= m ? m - 1 : 0u;
-    }
-#pragma unroll
-    for (int r = 0; r < kPre; ++r) zz[r] = r < np ? __ldg(srow + pp[r]) : 0.f;
-    const int rounds = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(np));
-#pragma unroll
-    for (int r = 0; r < kPre; ++r)
-      if (r < rounds) place_hit(sm, spill, r < np, pp[r], zz[r], b1, lt);
-    // lanes with more than kPre hits (rare): one by one, all lanes in lock-step
     while (__any_sync(0xffffffffu, m != 0u)) {
       const bool has = m != 0u;
       const int j = has ? __ffs(m) - 1 : 0;
       m &= has ? m - 1 : 0u;
       const uint32_t pos = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
-      place_hit(sm, spill, has, pos, has ? __ldg(srow + pos) : 0.f, b1, lt);
+      place_hit<D>(sm, spill, has, pos, has ? pick_score(v, j) : 0.f, b1, lt);
     }
   }
 }
@@ -659,8 +658,8 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   }
   const uint32_t above1 = sm.t_above;
   const uint32_t b1 = b1i < 0 ? 0u : static_cast<uint32_t>(b1i);
-  uint2 *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - gm.s1);
-  if (b1i >= 0) stream_chunk(sm, srow, spill, a0, lo, hi, b1);
+  unsigned long long *spill = p.list + static_cast<long long>(row) * p.ldL + (lo - gm.s1);
+  if (b1i >= 0) stream_chunk<D>(sm, srow, spill, a0, lo, hi, b1);
   __syncthreads();
   if (tid < ncl) cl.map_shared_rank(sm.x_a, tid)[rank] = sm.n_sure;
   cl.sync();   // lists, counts and digit-2 histograms complete; every CTA has read h1
@@ -691,17 +690,150 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   }
   // the keys of b1, from the CTAs' lists
   select_rounds<D, kFull>(p, sm, cl, rank, ncl, ListSrc<D>{&sm, spill, sm.n_list}, b1, k_eff - above1,
-                above1, irow, k_eff);
+                          above1, irow, k_eff);
 }
 
-// Softmax attention of one query head over U = W u Omega (Omega read from idx), split across
-// the nsplit clusters of the head (grid z) and the CTAs of each; the first CTA of a cluster
-// merges the cluster's partial states, and with several clusters the last one to finish merges
-// theirs (Eqs. (3)-(5)).  Each CTA stages its entries' positions and scores in shared memory (in
-// blocks of kStage), then its warps gather 16 V rows at a time and keep online-softmax states.
 constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
 constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
 
+// One warp's online-softmax update over up to 16 entries: lane j < 16 holds entry j's V row
+// index vi (-1: no entry) and score z.  The 16 V rows are gathered together (each lane a D / 32
+// channel slice of every row), then folded into the warp's state (m, zs, acc).
+template <int D>
+__device__ __forceinline__ void attend16(const __nv_bfloat16 *Vb, int vi, float z, float &m,
+                                         float &zs, float (&acc)[D / 32]) {
+  constexpr int CPL = D / 32;   // channels per lane
+  const int lane = threadIdx.x & 31;
+  if (vi < 0) z = -INFINITY;
+  uint32_t wv[kAttnRows][CPL / 2];
+#pragma unroll
+  for (int j = 0; j < kAttnRows; ++j) {
+    const int pj = __shfl_sync(0xffffffffu, vi, j);
+    if (pj >= 0) {
+      const __nv_bfloat16 *vr = Vb + static_cast<long long>(pj) * D;
+      if constexpr (CPL == 4) {
+        const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(vr) + lane);
+        wv[j][0] = v.x;
+        wv[j][1] = v.y;
+      } else {
+        wv[j][0] = __ldcg(reinterpret_cast<const uint32_t *>(vr) + lane);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL / 2; ++c) wv[j][c] = 0u;
+    }
+  }
+  float mg = lane < kAttnRows ? z : -INFINITY;   // the xor partners stay within groups of 16
+#pragma unroll
+  for (int o = kAttnRows / 2; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
+  mg = __shfl_sync(0xffffffffu, mg, 0);
+  if (mg == -INFINITY) return;   // warp-uniform: no entry in this group
+  const float mn = fmaxf(m, mg);
+  const float sc = expf(m - mn);   // 0 while m is -inf
+  const float pe = (lane >= kAttnRows || z == -INFINITY) ? 0.f : expf(z - mn);
+  float ps = pe;
+#pragma unroll
+  for (int o = kAttnRows / 2; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+  ps = __shfl_sync(0xffffffffu, ps, 0);
+  zs = zs * sc + ps;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) acc[c] *= sc;
+#pragma unroll
+  for (int j = 0; j < kAttnRows; ++j) {
+    const float pj = __shfl_sync(0xffffffffu, pe, j);
+#pragma unroll
+    for (int c = 0; c < CPL / 2; ++c) {
+      acc[2 * c] += pj * bf16_lo(wv[j][c]);
+      acc[2 * c + 1] += pj * bf16_hi(wv[j][c]);
+    }
+  }
+  m = mn;
+}
+
+// The CTA's warps' states -> one partial state (m_S, Z_S, N_S), pushed into the first CTA's
+// exchange slots (its digit histogram, free during the attention); after the cluster barrier the
+// first CTA merges the cluster's states into the output, or, with several clusters per head
+// (grid z), into this cluster's state for the head's last cluster to merge (Eqs. (3)-(5)).
+template <int D>
+__device__ void combine_and_merge(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl,
+                                  int rank, int ncl, int row, float m, float zs,
+                                  const float (&acc)[D / 32]) {
+  constexpr int CPL = D / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (lane == 0) {
+    sm.wm[warp] = m;
+    sm.wz[warp] = zs;
+  }
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) sm.wacc[warp * D + lane * CPL + c] = acc[c];
+  __syncthreads();
+  float M = sm.wm[0];
+#pragma unroll
+  for (int i = 1; i < kSaWarps; ++i) M = fmaxf(M, sm.wm[i]);
+  float ew[kSaWarps];
+#pragma unroll
+  for (int i = 0; i < kSaWarps; ++i) ew[i] = sm.wm[i] == -INFINITY ? 0.f : expf(sm.wm[i] - M);
+  float *xacc0 = reinterpret_cast<float *>(cl.map_shared_rank(sm.h, 0));
+  for (int c = tid; c < D; c += kSaThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSaWarps; ++i) s += ew[i] * sm.wacc[i * D + c];
+    xacc0[rank * D + c] = s;
+  }
+  if (tid == 0) {
+    float zt = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSaWarps; ++i) zt += ew[i] * sm.wz[i];
+    cl.map_shared_rank(sm.x_m, 0)[rank] = M;
+    cl.map_shared_rank(sm.x_s, 0)[rank] = zt;
+  }
+  cl.sync();   // every CTA's partial state is in the first CTA
+  if (rank == 0) {
+    const float *xacc = reinterpret_cast<const float *>(sm.h);
+    float Mx = -INFINITY;
+    for (int c = 0; c < ncl; ++c) Mx = fmaxf(Mx, sm.x_m[c]);
+    float den = 0.f;
+    for (int c = 0; c < ncl; ++c)
+      if (sm.x_m[c] != -INFINITY) den += expf(sm.x_m[c] - Mx) * sm.x_s[c];
+    // one cluster: the output; several: this cluster's state for the last one to merge
+    constexpr int PS = D + kPartPad;
+    float *prow = p.part + static_cast<long long>(row) * kMaxAttnSplit * PS;
+    float *mine = prow + static_cast<long long>(blockIdx.z) * PS;
+    for (int ch = tid; ch < D; ch += kSaThreads) {
+      float num = 0.f;
+      for (int c = 0; c < ncl; ++c)
+        if (sm.x_m[c] != -INFINITY) num += expf(sm.x_m[c] - Mx) * xacc[c * D + ch];
+      if (p.nsplit == 1) p.out[static_cast<long long>(row) * D + ch] = num / den;
+      else mine[kPartPad + ch] = num;
+    }
+    if (p.nsplit > 1) {
+      if (tid == 0) {
+        mine[0] = Mx;
+        mine[1] = den;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        const uint32_t prev = atomicAdd(p.meta + static_cast<long long>(row) * kMetaWords + kDone, 1u);
+        sm.t_bin = prev == static_cast<uint32_t>(p.nsplit - 1) ? 1 : 0;
+        if (sm.t_bin) __threadfence();
+      }
+      __syncthreads();
+      if (sm.t_bin) {   // the head's last cluster: merge the nsplit states
+        merge_states<D, kSaThreads>(prow, p.nsplit, p.out + static_cast<long long>(row) * D,
+                                    reinterpret_cast<float *>(sm.warp_tot),
+                                    reinterpret_cast<float *>(sm.sure));
+        if (tid == 0) p.meta[static_cast<long long>(row) * kMetaWords + kDone] = 0u;
+      }
+    }
+  }
+  // no CTA reads another's shared memory after the exchange barrier: all may leave
+}
+
+// Softmax attention of one query head over U = W u Omega (Omega read from idx), split across
+// the nsplit clusters of the head (grid z) and the CTAs of each.  Each CTA stages its entries'
+// positions and scores in shared memory (in blocks of kStage), then its warps gather 16 V rows
+// at a time and keep online-softmax states.
 template <int D, bool kFull, class Pg>
 __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, SaSmem<D> &sm,
                              cg::cluster_group &cl, int rank, int ncl, int row) {
@@ -746,139 +878,68 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
     __syncthreads();
     for (int g = warp * kAttnRows; g < nb; g += kAttnRows * kSaWarps) {
       const bool mine = lane < kAttnRows && g + lane < nb;
-      const int pos = mine ? spos[g + lane] : -1;
-      const float z = mine && pos >= 0 ? sz[g + lane] : -INFINITY;
-      uint32_t wv[kAttnRows][CPL / 2];
-#pragma unroll
-      for (int j = 0; j < kAttnRows; ++j) {
-        const int pj = __shfl_sync(0xffffffffu, pos, j);
-        if (pj >= 0) {
-          const __nv_bfloat16 *vr = Vb + static_cast<long long>(pj) * D;
-          if constexpr (CPL == 4) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(vr) + lane);
-            wv[j][0] = v.x;
-            wv[j][1] = v.y;
-          } else {
-            wv[j][0] = __ldg(reinterpret_cast<const uint32_t *>(vr) + lane);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < CPL / 2; ++c) wv[j][c] = 0u;
-        }
-      }
-      float mg = z;   // lanes >= 16 hold -inf; the xor partners stay within groups of 16
-#pragma unroll
-      for (int o = kAttnRows / 2; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
-      mg = __shfl_sync(0xffffffffu, mg, 0);
-      if (mg == -INFINITY) continue;   // warp-uniform: no entry in this group
-      const float mn = fmaxf(m, mg);
-      const float sc = expf(m - mn);   // 0 while m is -inf
-      const float pe = z == -INFINITY ? 0.f : expf(z - mn);
-      float ps = pe;
-#pragma unroll
-      for (int o = kAttnRows / 2; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-      ps = __shfl_sync(0xffffffffu, ps, 0);
-      zs = zs * sc + ps;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[c] *= sc;
-#pragma unroll
-      for (int j = 0; j < kAttnRows; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, pe, j);
-#pragma unroll
-        for (int c = 0; c < CPL / 2; ++c) {
-          acc[2 * c] += pj * bf16_lo(wv[j][c]);
-          acc[2 * c + 1] += pj * bf16_hi(wv[j][c]);
-        }
-      }
-      m = mn;
+      attend16<D>(Vb, mine ? spos[g + lane] : -1, mine ? sz[g + lane] : -INFINITY, m, zs, acc);
     }
     __syncthreads();   // the staging area is reused by the next block
   }
-  // the CTA's warps -> one partial state (m_S, Z_S, N_S) in this CTA's shared memory
-  if (lane == 0) {
-    sm.wm[warp] = m;
-    sm.wz[warp] = zs;
-  }
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) sm.wacc[warp * D + lane * CPL + c] = acc[c];
-  __syncthreads();
-  float M = sm.wm[0];
-#pragma unroll
-  for (int i = 1; i < kSaWarps; ++i) M = fmaxf(M, sm.wm[i]);
-  float ew[kSaWarps];
-#pragma unroll
-  for (int i = 0; i < kSaWarps; ++i) ew[i] = sm.wm[i] == -INFINITY ? 0.f : expf(sm.wm[i] - M);
-  // this CTA's partial state goes straight into the first CTA's exchange slots (its threshold
-  // list is free during the attention): numerators [rank][D], (m, Z) in x_m / x_s
-  float *xacc0 = reinterpret_cast<float *>(cl.map_shared_rank(sm.list, 0));
-  for (int c = tid; c < D; c += kSaThreads) {
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < kSaWarps; ++i) s += ew[i] * sm.wacc[i * D + c];
-    xacc0[rank * D + c] = s;
-  }
-  if (tid == 0) {
-    float zt = 0.f;
-#pragma unroll
-    for (int i = 0; i < kSaWarps; ++i) zt += ew[i] * sm.wz[i];
-    cl.map_shared_rank(sm.x_m, 0)[rank] = M;
-    cl.map_shared_rank(sm.x_s, 0)[rank] = zt;
-  }
-  cl.sync();   // every CTA's partial state is in the first CTA
-  if (rank == 0) {
-    const float *xacc = reinterpret_cast<const float *>(sm.list);
-    float Mx = -INFINITY;
-    for (int c = 0; c < ncl; ++c) Mx = fmaxf(Mx, sm.x_m[c]);
-    float den = 0.f;
-    for (int c = 0; c < ncl; ++c)
-      if (sm.x_m[c] != -INFINITY) den += expf(sm.x_m[c] - Mx) * sm.x_s[c];
-    // one cluster: the output; several: this cluster's state for the last one to merge
-    constexpr int PS = D + kPartPad;
-    float *prow = p.part + static_cast<long long>(row) * kMaxAttnSplit * PS;
-    float *mine = prow + static_cast<long long>(blockIdx.z) * PS;
-    for (int ch = tid; ch < D; ch += kSaThreads) {
-      float num = 0.f;
-      for (int c = 0; c < ncl; ++c)
-        if (sm.x_m[c] != -INFINITY) num += expf(sm.x_m[c] - Mx) * xacc[c * D + ch];
-      if (p.nsplit == 1) p.out[static_cast<long long>(row) * D + ch] = num / den;
-      else mine[kPartPad + ch] = num;
+  combine_and_merge<D>(p, sm, cl, rank, ncl, row, m, zs, acc);
+}
+
+// Waits (rank 0's first thread, polling with a time limit) until every score CTA is done with
+// this row's KV head, then tells every CTA of the cluster whether it may go on.  The row group's
+// last cluster to get through sets the counter back to zero for the next step (the next score
+// launch adds to it only after this kernel has finished).  Returns false on a timeout (error
+// bit kErrReadyWait); every CTA of the cluster returns the same.
+template <int D>
+__device__ bool wait_ready(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl, int rank, int ncl,
+                           int row) {
+  constexpr unsigned long long kLimitNs = 1000000000ull;   // one second
+  if (rank == 0 && threadIdx.x == 0) {
+    uint32_t *ctr = p.ready + static_cast<long long>(row / p.G) * p.ready_stride;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    uint32_t ok = 1u;
+    for (;;) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= p.ready_target) break;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > kLimitNs) {
+        ok = 0u;
+        atomicOr(p.err, kErrReadyWait);
+        break;
+      }
+      __nanosleep(256);
     }
-    if (p.nsplit > 1) {
-      if (tid == 0) {
-        mine[0] = Mx;
-        mine[1] = den;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        const uint32_t prev = atomicAdd(p.meta + static_cast<long long>(row) * kMetaWords + kDone, 1u);
-        sm.t_bin = prev == static_cast<uint32_t>(p.nsplit - 1) ? 1 : 0;
-        if (sm.t_bin) __threadfence();
-      }
-      __syncthreads();
-      if (sm.t_bin) {   // the head's last cluster: merge the nsplit states
-        merge_states<D, kSaThreads>(prow, p.nsplit, p.out + static_cast<long long>(row) * D,
-                                    reinterpret_cast<float *>(sm.warp_tot),
-                                    reinterpret_cast<float *>(sm.sure));
-        if (tid == 0) p.meta[static_cast<long long>(row) * kMetaWords + kDone] = 0u;
-      }
+    // the G clusters of this KV head pass here once each; the last one resets the counters
+    const uint32_t prev = atomicAdd(ctr + 1, 1u);
+    if (prev == static_cast<uint32_t>(p.G - 1)) {
+      ctr[0] = 0u;
+      ctr[1] = 0u;
     }
+    for (int c = 0; c < ncl; ++c) cl.map_shared_rank(&sm, c)->x_ok = ok;
   }
-  // no CTA reads another's shared memory after the exchange barrier: all may leave
+  cl.sync();   // the verdict is in every CTA (and rank 0's acquire orders the cluster's reads)
+  return sm.x_ok != 0u;
 }
 
 // kFull = false: the plain decode step (the score kernel's histogram, the cache's own score rows
 // and positions); the threshold budget, the self-built histogram and candidate lists take the
 // kFull = true instantiation, so the plain one carries none of their code.
 template <int D, class Pg, bool kFull>
-__global__ void __launch_bounds__(kSaThreads, 4) select_attend_kernel(const SaParams p, const Pg pg) {
+__global__ void __launch_bounds__(kSaThreads, 3) select_attend_kernel(const SaParams p, const Pg pg) {
   __shared__ SaSmem<D> sm;
   cg::cluster_group cl = cg::this_cluster();
   const int ncl = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
   const int row = blockIdx.y;
   pdl_trigger();
-  pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
+  if (p.ready != nullptr) {
+    // the scan is still running: start once this row's KV head is scored
+    if (!wait_ready(p, sm, cl, rank, ncl, row)) return;
+  } else {
+    pdl_wait();   // the scores, histograms and (attention only) idx come from earlier kernels
+  }
   // each phase computes the row geometry afresh (nothing stays live across the selection)
   if (p.mode & kSaSelect)
     select_phase<D, kFull>(p, row_geo<kFull>(p, pg, row, ncl), sm, cl, rank, ncl, row);
@@ -944,12 +1005,22 @@ int select_cluster_size(long long nC, int R, int d) {
 template <int D, class Pg, bool kFull>
 static cudaError_t launch_sa_k(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
   static bool attr_done[64] = {};
+  static bool carve_done[64] = {};
   int dev = 0;
-  if (ncl > 8 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && !attr_done[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
-                                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+    if (ncl > 8 && !attr_done[dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
+                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+      attr_done[dev] = true;
+    }
+    if (!carve_done[dev]) {   // the same carveout as the scan, so both fit on one SM
+      const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
+                                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                 cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
+      carve_done[dev] = true;
+    }
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ncl), static_cast<unsigned>(R),
@@ -975,6 +1046,8 @@ static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, 
                     p.pos_map != nullptr || p.S_att != nullptr;
   return full ? launch_sa_k<D, Pg, true>(p, pg, R, ncl, s) : launch_sa_k<D, Pg, false>(p, pg, R, ncl, s);
 }
+
+size_t select_smem_bytes(int d) { return d == 128 ? sizeof(SaSmem<128>) : sizeof(SaSmem<64>); }
 
 int attn_split(long long nU, int R, int ncl, int d) {
   if (nU <= 1024LL * ncl) return 1;

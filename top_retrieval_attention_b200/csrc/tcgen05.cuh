@@ -7,11 +7,6 @@
 
 namespace ra {
 
-// One arrival (of the count given at init) by this thread on a shared-memory mbarrier.
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-
 // Allocates `ncols` tensor-memory columns (a power of two >= 32) for this CTA; the base address
 // is written to shared memory at `slot`.  Whole warp.
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {

@@ -29,6 +29,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Plain arrival (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+
 // Returns true once the barrier's phase with the given parity has completed, false if the
 // poll budget ran out first.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
@@ -43,6 +48,44 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (done) return true;
   }
   return false;
+}
+
+// As mbar_wait, but also gives up (false) once *abort is non-zero: a CTA whose pipeline broke
+// stops all its waits at once instead of each running out its own budget.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                   const volatile int *abort) {
+  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 15u) == 15u && *abort) return false;
+  }
+  return false;
+}
+
+// 1-D bulk copy global -> shared (this CTA), completion counted in bytes on the mbarrier; both
+// addresses 16-byte aligned and `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Barrier 1 over the first `threads` threads of the CTA (barrier 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int threads) {
+  asm volatile("bar.sync 1, %0;\n" ::"r"(threads) : "memory");
+}
+
+// Adds 1 to a device-wide counter with release semantics: writes this thread has made or
+// observed (a preceding barrier) are visible to any thread that acquires the new value.
+__device__ __forceinline__ void red_release_add1(uint32_t *ctr) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;\n" ::"l"(ctr) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
