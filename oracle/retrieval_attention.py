@@ -321,3 +321,61 @@ def ivf_decode_head(q_bits: np.ndarray, K_bits: np.ndarray, V_bits: np.ndarray,
     omega = select_topk(z, C, k)
     U = np.concatenate([static_set(N, n_sink, n_window), omega])
     return attend(z, V, U), omega, z, probe
+
+
+# ------------------------------------------------------------------------------------
+# IVF index construction (the pages name IVF over the keys as a baseline without fixing a
+# construction; read as spherical k-means): centroids are unit vectors stored in bf16, keys go
+# to the centroid of largest inner product, Lloyd iterations move each centroid to the unit
+# direction of its keys' sum, and the index lists the keys cluster by cluster
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) of the float64 values x, rounded to nearest with ties to
+    even.  The two bf16 neighbours of x are found from a float32 copy truncated to its top 16
+    bits and the next magnitude up, and the nearer one (exact float64 distances) is kept."""
+    x = np.asarray(x, dtype=np.float64)
+    t = x.astype(np.float32).view(np.uint32)
+    sign = t & np.uint32(0x80000000)
+    lo_bits = (t & np.uint32(0x7FFFFFFF)) >> np.uint32(16)
+    hi_bits = lo_bits + np.uint32(1)
+    lo = ((lo_bits << np.uint32(16)) | sign).view(np.float32).astype(np.float64)
+    hi = ((hi_bits << np.uint32(16)) | sign).view(np.float32).astype(np.float64)
+    dlo, dhi = np.abs(x - lo), np.abs(x - hi)
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & ((lo_bits & np.uint32(1)) == 1))
+    mag = np.where(pick_hi, hi_bits, lo_bits)
+    return (mag | (sign >> np.uint32(16))).astype(np.uint16)
+
+
+def unit_bf16(v: np.ndarray) -> np.ndarray:
+    """bf16 bits of v / ||v|| (a zero vector stays zero)."""
+    n = math.sqrt(float(np.sum(v * v)))
+    return round_to_bf16(v / n if n > 0 else np.zeros_like(v))
+
+
+def ivf_build(K_bits: np.ndarray, nlist: int, iters: int):
+    """Spherical k-means index of one KV head's keys K [N, d] (bf16 bits).
+
+    Centroid j starts as the unit key at position floor(j * N / nlist); each of `iters` Lloyd
+    iterations assigns every key to the centroid of largest k . c (ties to the lower centroid)
+    and moves every non-empty cluster's centroid to the unit direction of its keys' sum (an
+    empty cluster keeps its centroid); a final assignment fixes the clusters.  Centroids are
+    held as bf16.  Returns (centroid bits [nlist, d], assignment [N], the positions grouped by
+    cluster in increasing position order [N], cluster offsets [nlist + 1])."""
+    K = bf16_to_f64(K_bits)
+    N = K.shape[0]
+    cent = np.stack([unit_bf16(K[(j * N) // nlist]) for j in range(nlist)])
+    for it in range(iters + 1):
+        S = K @ bf16_to_f64(cent).T
+        assign = np.argmax(S, axis=1)            # the first maximum: ties to the lower centroid
+        if it == iters:
+            break
+        for j in range(nlist):
+            members = assign == j
+            if np.any(members):
+                s = np.sum(K[members], axis=0)
+                if np.sum(s * s) > 0:
+                    cent[j] = unit_bf16(s)
+    pos = np.argsort(assign, kind="stable")
+    offsets = np.concatenate([[0], np.cumsum(np.bincount(assign, minlength=nlist))])
+    return cent, assign, pos, offsets

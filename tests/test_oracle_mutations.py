@@ -184,3 +184,53 @@ def test_prefill_with_a_causal_mask_is_caught(monkeypatch):
     # (with the window covering the last M positions the mask removes no candidate; the tiny
     # brute-force cases have windows of 0 or 1 token)
     assert any(_fails(pins.test_prefill_topk_brute_force, t) for t in range(6))
+
+
+# ---------------------------------------------------------------- IVF index construction
+
+
+def _kmeans(K_bits, nlist, iters, init=None, argmax=None, update=None, empty=None):
+    """The oracle's spherical k-means with one step swapped for a planted mistake."""
+    K = ra.bf16_to_f64(K_bits)
+    N = K.shape[0]
+    starts = init(N, nlist) if init else [(j * N) // nlist for j in range(nlist)]
+    cent = np.stack([ra.unit_bf16(K[i]) for i in starts])
+    for it in range(iters + 1):
+        S = K @ ra.bf16_to_f64(cent).T
+        assign = argmax(S) if argmax else np.argmax(S, axis=1)
+        if it == iters:
+            break
+        for j in range(nlist):
+            members = assign == j
+            if np.any(members):
+                s = np.sum(K[members], axis=0)
+                cent[j] = update(s, members) if update else ra.unit_bf16(s)
+            elif empty:
+                cent[j] = empty(cent[j])
+    pos = np.argsort(assign, kind="stable")
+    offsets = np.concatenate([[0], np.cumsum(np.bincount(assign, minlength=nlist))])
+    return cent, assign, pos, offsets
+
+
+def test_ivf_ties_to_the_higher_centroid_are_caught(monkeypatch):
+    last_max = lambda S: S.shape[1] - 1 - np.argmax(S[:, ::-1], axis=1)
+    _patch(monkeypatch, "ivf_build", lambda K, n, it: _kmeans(K, n, it, argmax=last_max))
+    assert _fails(pins.test_ivf_build_ties_go_to_the_lower_centroid)
+
+
+def test_ivf_unnormalised_mean_is_caught(monkeypatch):
+    mean = lambda s, members: ra.round_to_bf16(s / np.count_nonzero(members))
+    _patch(monkeypatch, "ivf_build", lambda K, n, it: _kmeans(K, n, it, update=mean))
+    assert _fails(pins.test_ivf_build_two_directions_is_a_fixed_point, 1)
+
+
+def test_ivf_empty_cluster_zeroed_is_caught(monkeypatch):
+    zero = lambda c: np.zeros_like(c)
+    _patch(monkeypatch, "ivf_build", lambda K, n, it: _kmeans(K, n, it, empty=zero))
+    assert _fails(pins.test_ivf_build_empty_cluster_keeps_its_centroid)
+
+
+def test_ivf_start_from_the_first_keys_is_caught(monkeypatch):
+    first = lambda N, nlist: list(range(nlist))
+    _patch(monkeypatch, "ivf_build", lambda K, n, it: _kmeans(K, n, it, init=first))
+    assert _fails(pins.test_ivf_build_two_directions_is_a_fixed_point, 0)

@@ -561,3 +561,129 @@ def test_ivf_candidates_are_the_probed_clusters():
     offsets = np.concatenate([[0], np.cumsum(np.bincount(assign, minlength=6))])
     _, om, _, _ = oracle.ivf_decode_head(q, K, V, pos, offsets, cent, 1000, 2, 0, 0)
     assert set(om.tolist()) == {i for i in range(N) if i % 6 in (0, 2)}
+
+
+# ---------------------------------------------------------------- IVF index construction
+
+
+def test_round_to_bf16_known_values():
+    """Round to nearest even, from hand-worked float32 patterns: 0.6 = 0x3F19999A and 0.8 =
+    0x3F4CCCCD round up (low halves above 0x8000); 1 + 2^-8 and 1 + 3 * 2^-8 sit exactly
+    between two bf16 values and go to the even one; 12/13 = 0x3F6C4EC5 rounds down."""
+    x = np.array([0.6, 0.8, 1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 12 / 13, -0.6, 0.0, 1.0])
+    want = [0x3F1A, 0x3F4D, 0x3F80, 0x3F82, 0x3F6C, 0xBF1A, 0x0000, 0x3F80]
+    assert oracle.round_to_bf16(x).tolist() == want
+
+
+def _two_direction_keys():
+    """40 keys in 64 channels: positions 0-19 are multiples of (3, 4) in channels 0-1,
+    positions 20-39 multiples of (5, 12) in channels 2-3 (all exact in bf16)."""
+    K = np.zeros((40, 64))
+    for i in range(20):
+        K[i, :2] = (1 + i % 3) * np.array([3.0, 4.0])
+        K[20 + i, 2:4] = (1 + i % 3) * np.array([5.0, 12.0])
+    return gen.f64_to_bf16_bits(K)
+
+
+@pytest.mark.parametrize("iters", [0, 1, 3])
+def test_ivf_build_two_directions_is_a_fixed_point(iters):
+    """Two orthogonal groups of parallel keys: the evenly spaced start (positions 0 and 20)
+    already points along each group, and the unit direction of a group's sum is that same
+    direction, bf16 (3, 4) / 5 = (0x3F1A, 0x3F4D) and (5, 12) / 13 = (0x3EC5, 0x3F6C)
+    (worked by hand, see test_round_to_bf16_known_values)."""
+    cent, assign, pos, offsets = oracle.ivf_build(_two_direction_keys(), 2, iters)
+    want = np.zeros((2, 64), np.uint16)
+    want[0, :2] = [0x3F1A, 0x3F4D]
+    want[1, 2:4] = [0x3EC5, 0x3F6C]
+    assert np.array_equal(cent, want)
+    assert assign.tolist() == [0] * 20 + [1] * 20
+    assert pos.tolist() == list(range(40)) and offsets.tolist() == [0, 20, 40]
+
+
+def test_ivf_build_ties_go_to_the_lower_centroid():
+    """Keys e_0, e_1 (the two starting centroids) and e_0 + e_1, which scores 1 against both:
+    it joins centroid 0.  One iteration later centroid 0 is the unit direction of (2, 1),
+    bf16 (0x3F65, 0x3EE5), and the assignment is unchanged."""
+    K = np.zeros((3, 64))
+    K[0, 0] = K[1, 1] = 1.0
+    K[2, :2] = 1.0
+    bits = gen.f64_to_bf16_bits(K)
+    cent, assign, _, _ = oracle.ivf_build(bits, 2, 0)
+    assert assign.tolist() == [0, 1, 0]
+    cent, assign, pos, offsets = oracle.ivf_build(bits, 2, 1)
+    assert cent[0, :2].tolist() == [0x3F65, 0x3EE5] and cent[1, :2].tolist() == [0, 0x3F80]
+    assert assign.tolist() == [0, 1, 0]
+    assert pos.tolist() == [0, 2, 1] and offsets.tolist() == [0, 2, 3]
+
+
+def test_ivf_build_empty_cluster_keeps_its_centroid():
+    """Positions 0 and 2 hold the same key e_0, so both centroids start equal; every key ties
+    and joins centroid 0, leaving cluster 1 empty: it keeps e_0 while centroid 0 moves to the
+    unit direction of the sum (5, 2), bf16 (0x3F6E, 0x3EBE).  The final assignment then sends
+    the two e_0 keys to centroid 1 (score 1 against 5 / sqrt(29) = 0.93)."""
+    K = np.zeros((4, 64))
+    K[0, 0] = K[2, 0] = 1.0
+    K[1, :2] = (1.0, 1.0)
+    K[3, :2] = (2.0, 1.0)
+    cent, assign, pos, offsets = oracle.ivf_build(gen.f64_to_bf16_bits(K), 2, 1)
+    assert cent[0, :2].tolist() == [0x3F6E, 0x3EBE] and np.all(cent[0, 2:] == 0)
+    assert cent[1, :2].tolist() == [0x3F80, 0] and np.all(cent[1, 2:] == 0)
+    assert assign.tolist() == [1, 0, 1, 0]
+    assert pos.tolist() == [1, 3, 0, 2] and offsets.tolist() == [0, 2, 4]
+
+
+def _bf16_rne_exact(x):
+    """Nearest bf16 (ties to even) of an exact rational x, by comparing it with the two
+    float32-truncated neighbours as Fractions (struct packing, no numpy)."""
+    import struct
+    xf = float(x)
+    b = struct.unpack(">I", struct.pack(">f", xf))[0]
+    s, lo = b >> 31, (b & 0x7FFFFFFF) >> 16
+
+    def val(m):
+        return Fraction(struct.unpack(">f", struct.pack(">I", (s << 31) | (m << 16)))[0])
+
+    dl, dh = abs(x - val(lo)), abs(x - val(lo + 1))
+    m = lo + 1 if (dh < dl or (dh == dl and lo & 1)) else lo
+    return (s << 15) | m
+
+
+def _unit_bf16_exact(v):
+    from decimal import Decimal, getcontext
+    getcontext().prec = 80
+    n2 = sum(a * a for a in v)
+    if n2 == 0:
+        return [0] * len(v)
+    n = (Decimal(n2.numerator) / Decimal(n2.denominator)).sqrt()
+    return [_bf16_rne_exact(Fraction(Decimal(a.numerator) / Decimal(a.denominator) / n)) for a in v]
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_ivf_build_matches_brute_force_on_tiny_inputs(seed):
+    """Spherical k-means written out with exact rationals (scores, sums), an 80-digit square
+    root and the nearest-even rounding above, on 11 keys of 4 channels into 3 clusters."""
+    rng = np.random.default_rng(100 + seed)
+    N, d, nlist, iters = 11, 4, 3, 2
+    bits = rand_bf16((N, d), rng=rng)
+    Kq = [[Fraction(float(x)) for x in row] for row in oracle.bf16_to_f64(bits)]
+    cent = [_unit_bf16_exact(Kq[(j * N) // nlist]) for j in range(nlist)]
+    for it in range(iters + 1):
+        Cq = [[Fraction(float(x)) for x in oracle.bf16_to_f64(np.array(c, np.uint16))] for c in cent]
+        assign = []
+        for k in Kq:
+            sc = [sum(a * b for a, b in zip(k, c)) for c in Cq]
+            assign.append(max(range(nlist), key=lambda j: (sc[j], -j)))
+        if it == iters:
+            break
+        for j in range(nlist):
+            mem = [Kq[i] for i in range(N) if assign[i] == j]
+            if mem:
+                s = [sum(col) for col in zip(*mem)]
+                if any(x != 0 for x in s):
+                    cent[j] = _unit_bf16_exact(s)
+    got_c, got_a, got_p, got_o = oracle.ivf_build(bits, nlist, iters)
+    assert got_c.tolist() == cent
+    assert got_a.tolist() == assign
+    listing = [i for j in range(nlist) for i in range(N) if assign[i] == j]
+    assert got_p.tolist() == listing
+    assert got_o.tolist() == [0] + list(np.cumsum([assign.count(j) for j in range(nlist)]))
