@@ -314,9 +314,14 @@ typedef struct {
 
 /*
  * Build the index of kv's first ix->N keys (ix->N <= kv->N; B, Hkv, d as kv's): `iters` Lloyd
- * iterations of spherical k-means from centroids at evenly spaced keys (the key-centroid scores
- * on the tcgen05 tensor cores), then the final assignment and the sort by cluster.
- *   ws : at least ra_ivf_build_workspace_bytes(...) bytes, 256-byte aligned.
+ * iterations of spherical k-means from centroids at the unit keys of positions
+ * floor(c * N / nlist) (the key-centroid scores on the tcgen05 tensor cores, an empty cluster
+ * keeping its centroid, each centroid the unit direction of its keys' sum rounded to bf16),
+ * then the final assignment and the sort by cluster, keys of a cluster in increasing position.
+ * Deterministic: the same cache gives the same index bit for bit (integer counts, a stable
+ * sort, sums in position order).  The key-centroid scores are computed over chunks of keys, so
+ * the workspace is about 256 MB plus 4 * B * Hkv * (N + nlist * ceil(N / 1024)) bytes at any N.
+ *   ws : at least ra_ivf_build_workspace_bytes(...) bytes, 256-byte aligned (no zeroing needed).
  * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_WORKSPACE, RA_ERR_CUDA.
  */
 size_t ra_ivf_build_workspace_bytes(int32_t B, int32_t Hkv, int64_t N, int32_t d, int32_t nlist);

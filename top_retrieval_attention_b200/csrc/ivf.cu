@@ -4,12 +4,14 @@
 // searched on the GPU.
 //
 // Build, per KV head: spherical k-means (Lloyd iterations) of the N keys into nlist unit-norm
-// centroids.  The key-centroid scores of an iteration are the tcgen05 prefill score kernel with
-// the keys as its query rows and the centroids as its keys; one warp per key takes the argmax
-// (ties to the lower centroid) and adds the key into its centroid's fp32 sum; the sums are
-// normalised into the next centroids.  A final assignment, a count per cluster, an exclusive
-// scan and a scatter give the keys sorted by cluster (with their positions) and the cluster
-// offsets.
+// bf16 centroids, deterministic from start to end.  The key-centroid scores are the tcgen05
+// prefill score kernel with the keys as its query rows and the centroids as its keys, over
+// chunks of keys (the score workspace is bounded whatever N is); one warp per key takes the
+// argmax (ties to the lower centroid).  A stable counting sort then lists the keys cluster by
+// cluster in increasing position (per-chunk counts, a scan into slots, one warp per chunk
+// placing its keys in order), and one warp per cluster sums its keys in that order into the
+// next centroid (the unit direction of the sum; an empty cluster keeps its centroid).  The
+// final sort also copies the keys into the sorted copy.
 // Search, per query head: the scores of the nlist centroids and the nprobe best, the exact
 // scores of every key of the probed clusters (read contiguously from the sorted copy; static-set
 // positions excluded) and of the static set; the cluster kernel then selects the exact top-k of
@@ -46,12 +48,12 @@ __global__ void __launch_bounds__(128) ivf_init_kernel(const IvfParams p) {
         __float2bfloat16_rn(norm > 0.f ? v / norm : 0.f);
 }
 
-// One warp per key: the argmax of its centroid scores (row of A, ties to the lower centroid),
-// recorded in assign; with sums != nullptr the key is also added into its centroid's sum.
-__global__ void __launch_bounds__(256) ivf_assign_kernel(const IvfParams p, int accumulate) {
+// One warp per key of the chunk [c0, c0 + M): the argmax of its centroid scores (row of A, ties
+// to the lower centroid) into assign.
+__global__ void __launch_bounds__(256) ivf_assign_kernel(const IvfParams p) {
   const long long w = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(p.BH) * p.N;
+  const long long rows = static_cast<long long>(p.BH) * p.M;
   if (w >= rows) return;   // whole warps leave together
   const float *a = p.A + w * p.ldA;
   float best = -INFINITY;
@@ -72,54 +74,53 @@ __global__ void __launch_bounds__(256) ivf_assign_kernel(const IvfParams p, int 
       bi = oi;
     }
   }
-  const long long bg = w / p.N, pos = w - bg * p.N;
   if (lane == 0) {
-    p.assign[w] = bi;
-    atomicAdd(p.count + bg * p.nlist + bi, 1u);
-  }
-  if (accumulate) {
-    const __nv_bfloat16 *k = p.K + (bg * p.cap + pos) * p.d;
-    float *sum = p.sums + (bg * p.nlist + bi) * p.d;
-    for (int c = lane; c < p.d; c += 32) atomicAdd(sum + c, __bfloat162float(k[c]));
+    const long long bg = w / p.M;
+    p.assign[bg * p.N + p.c0 + (w - bg * p.M)] = bi < p.nlist ? bi : 0;   // (a row of NaNs: 0)
   }
 }
 
-// Centroid c of head bg becomes its normalised sum (kept when the cluster is empty); the sums
-// and counts are cleared for the next iteration.
-__global__ void __launch_bounds__(128) ivf_update_kernel(const IvfParams p) {
+// The keys of each cluster in each sort chunk of kIvfSortChunk positions (one CTA per chunk).
+__global__ void __launch_bounds__(256) ivf_chunk_count_kernel(const IvfParams p) {
+  extern __shared__ uint32_t hc[];   // nlist counters
   const long long bg = blockIdx.y;
-  const int c = blockIdx.x;
-  float *sum = p.sums + (bg * p.nlist + c) * p.d;
-  float v = 0.f;
-  if (threadIdx.x < p.d) v = sum[threadIdx.x];
-  __shared__ float red[4];
-  float ss = warp_sum(v * v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  const int ch = blockIdx.x;
+  for (int c = threadIdx.x; c < p.nlist; c += 256) hc[c] = 0u;
   __syncthreads();
-  const float norm = sqrtf(red[0] + red[1] + red[2] + red[3]);
-  const uint32_t n = p.count[bg * p.nlist + c];
-  if (threadIdx.x < p.d) {
-    if (n > 0 && norm > 0.f)
-      p.cent[(bg * p.nlist + c) * p.d + threadIdx.x] = __float2bfloat16_rn(v / norm);
-    sum[threadIdx.x] = 0.f;
-  }
+  const long long lo = static_cast<long long>(ch) * kIvfSortChunk;
+  const long long hi = min(p.N, lo + kIvfSortChunk);
+  for (long long i = lo + threadIdx.x; i < hi; i += 256) atomicAdd(&hc[p.assign[bg * p.N + i]], 1u);
   __syncthreads();
-  if (threadIdx.x == 0) p.count[bg * p.nlist + c] = 0u;
+  uint32_t *out = p.chunk_cnt + (bg * p.nsort + ch) * p.nlist;
+  for (int c = threadIdx.x; c < p.nlist; c += 256) out[c] = hc[c];
 }
 
-// Exclusive scan of one head's cluster counts into offsets[0..nlist] (one CTA per head); the
-// scatter cursors are cleared.
-__global__ void __launch_bounds__(1024) ivf_offsets_kernel(const IvfParams p) {
+// One CTA per head: offsets (an exclusive scan of the cluster totals over the clusters) and,
+// per sort chunk and cluster, the first slot of that chunk's keys of the cluster (the cluster's
+// offset plus the counts of the earlier chunks), in place of the counts.
+__global__ void __launch_bounds__(1024) ivf_slots_kernel(const IvfParams p) {
   const long long bg = blockIdx.x;
+  uint32_t *cc = p.chunk_cnt + bg * p.nsort * p.nlist;
+  int32_t *offs = p.offsets + bg * (p.nlist + 1);
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t carry;
+  // earlier chunks' counts per cluster; the totals go to offs for the scan
+  for (int c = threadIdx.x; c < p.nlist; c += 1024) {
+    uint32_t run = 0;
+    for (int ch = 0; ch < p.nsort; ++ch) {
+      const uint32_t v = cc[static_cast<long long>(ch) * p.nlist + c];
+      cc[static_cast<long long>(ch) * p.nlist + c] = run;
+      run += v;
+    }
+    offs[c] = static_cast<int32_t>(run);
+  }
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int c0 = 0; c0 < p.nlist; c0 += 1024) {
     const int c = c0 + threadIdx.x;
-    const uint32_t v = c < p.nlist ? p.count[bg * p.nlist + c] : 0u;
+    const uint32_t v = c < p.nlist ? static_cast<uint32_t>(offs[c]) : 0u;
     uint32_t x = v;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
@@ -138,33 +139,104 @@ __global__ void __launch_bounds__(1024) ivf_offsets_kernel(const IvfParams p) {
     }
     __syncthreads();
     const uint32_t incl = carry + x + (warp > 0 ? warp_tot[warp - 1] : 0u);
-    if (c < p.nlist) {
-      p.offsets[bg * (p.nlist + 1) + c] = static_cast<int32_t>(incl - v);
-      p.cursor[bg * p.nlist + c] = 0u;
-    }
+    if (c < p.nlist) offs[c] = static_cast<int32_t>(incl - v);
     __syncthreads();
     if (threadIdx.x == 1023) carry = incl;
     __syncthreads();
   }
-  if (threadIdx.x == 0) p.offsets[bg * (p.nlist + 1) + p.nlist] = static_cast<int32_t>(carry);
+  if (threadIdx.x == 0) offs[p.nlist] = static_cast<int32_t>(carry);
+  __syncthreads();
+  for (int c = threadIdx.x; c < p.nlist; c += 1024) {
+    const uint32_t base = static_cast<uint32_t>(offs[c]);
+    for (int ch = 0; ch < p.nsort; ++ch) cc[static_cast<long long>(ch) * p.nlist + c] += base;
+  }
 }
 
-// Every key to its cluster's next free slot of the sorted copy, with its position.
-__global__ void __launch_bounds__(256) ivf_scatter_kernel(const IvfParams p) {
+// Stable scatter: one warp per sort chunk places the chunk's keys, 32 positions at a time in
+// increasing order, at their clusters' next slots: lanes that share a cluster take consecutive
+// slots in lane order and the group's first lane advances the chunk's slot counter (only this
+// warp touches it).  With copy_rows the warp also copies the 32 keys into the sorted copy.
+template <int D>
+__global__ void __launch_bounds__(256) ivf_stable_scatter_kernel(const IvfParams p, int copy_rows) {
   const long long w = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const long long rows = static_cast<long long>(p.BH) * p.N;
-  if (w >= rows) return;
-  const long long bg = w / p.N, pos = w - bg * p.N;
-  const int c = p.assign[w];
-  uint32_t slot = 0;
-  if (lane == 0) slot = atomicAdd(p.cursor + bg * p.nlist + c, 1u);
-  slot = __shfl_sync(0xffffffffu, slot, 0);
-  const long long dst = bg * p.N + p.offsets[bg * (p.nlist + 1) + c] + slot;
-  if (lane == 0) p.pos[dst] = static_cast<int32_t>(pos);
-  const uint32_t *src = reinterpret_cast<const uint32_t *>(p.K + (bg * p.cap + pos) * p.d);
-  uint32_t *out = reinterpret_cast<uint32_t *>(p.Ksorted + dst * p.d);
-  for (int c2 = lane; c2 < p.d / 2; c2 += 32) out[c2] = src[c2];
+  if (w >= static_cast<long long>(p.BH) * p.nsort) return;
+  const long long bg = w / p.nsort;
+  const int ch = static_cast<int>(w - bg * p.nsort);
+  uint32_t *slots = p.chunk_cnt + (bg * p.nsort + ch) * p.nlist;
+  const long long lo = static_cast<long long>(ch) * kIvfSortChunk;
+  const long long hi = min(p.N, lo + kIvfSortChunk);
+  for (long long base = lo; base < hi; base += 32) {
+    const long long i = base + lane;
+    const bool valid = i < hi;
+    const int c = valid ? p.assign[bg * p.N + i] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, c);
+    const int leader = __ffs(peers) - 1;
+    const uint32_t rank = __popc(peers & lanemask_lt());
+    uint32_t first = 0;
+    if (valid && lane == leader) first = atomicAdd(slots + c, static_cast<uint32_t>(__popc(peers)));
+    first = __shfl_sync(0xffffffffu, first, leader);
+    const long long dst = bg * p.N + first + rank;
+    if (valid) p.pos[dst] = static_cast<int32_t>(i);
+    if (copy_rows) {
+      constexpr int W = D / 64;   // 32-bit words of a row per lane
+      for (int j = 0; j < 32 && base + j < hi; ++j) {
+        const long long dj = __shfl_sync(0xffffffffu, dst, j);
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(p.K + (bg * p.cap + base + j) * D);
+        uint32_t *out = reinterpret_cast<uint32_t *>(p.Ksorted + dj * D);
+#pragma unroll
+        for (int u = 0; u < W; ++u) out[lane + 32 * u] = src[lane + 32 * u];
+      }
+    }
+  }
+}
+
+// Centroid c of head bg (one warp): the unit direction of the sum of its keys, added in
+// increasing position (lane l keeps channels [l * D / 32, (l + 1) * D / 32)); an empty cluster,
+// or a zero sum, keeps the centroid.
+template <int D>
+__global__ void __launch_bounds__(256) ivf_update_kernel(const IvfParams p) {
+  constexpr int CPL = D / 32;
+  const long long w = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= static_cast<long long>(p.BH) * p.nlist) return;
+  const long long bg = w / p.nlist;
+  const int c = static_cast<int>(w - bg * p.nlist);
+  const int32_t lo = p.offsets[bg * (p.nlist + 1) + c], hi = p.offsets[bg * (p.nlist + 1) + c + 1];
+  float acc[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) acc[k] = 0.f;
+  const __nv_bfloat16 *Kb = p.K + bg * p.cap * D + lane * CPL;
+  const int32_t *pos = p.pos + bg * p.N;
+  int32_t j = lo;
+  for (; j + 4 <= hi; j += 4) {   // four rows' loads in flight, added in order
+    float x[4][CPL];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const __nv_bfloat16 *row = Kb + static_cast<long long>(__ldg(pos + j + r)) * D;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) x[r][k] = __bfloat162float(row[k]);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) acc[k] += x[r][k];
+  }
+  for (; j < hi; ++j) {
+    const __nv_bfloat16 *row = Kb + static_cast<long long>(__ldg(pos + j)) * D;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) acc[k] += __bfloat162float(row[k]);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) ss += acc[k] * acc[k];
+  ss = warp_sum(ss);
+  const float norm = sqrtf(ss);
+  if (hi > lo && norm > 0.f) {
+    __nv_bfloat16 *out = p.cent + (bg * p.nlist + c) * D + lane * CPL;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) out[k] = __float2bfloat16_rn(acc[k] / norm);
+  }
 }
 
 // ---- search
@@ -440,19 +512,26 @@ cudaError_t launch_ivf_init(const IvfParams &p, cudaStream_t s) {
   ivf_init_kernel<<<dim3(p.nlist, p.BH), 128, 0, s>>>(p);
   return cudaGetLastError();
 }
-cudaError_t launch_ivf_assign(const IvfParams &p, bool accumulate, cudaStream_t s) {
-  const long long warps = static_cast<long long>(p.BH) * p.N;
-  ivf_assign_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(p, accumulate ? 1 : 0);
+cudaError_t launch_ivf_assign(const IvfParams &p, cudaStream_t s) {
+  const long long warps = static_cast<long long>(p.BH) * p.M;
+  ivf_assign_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+cudaError_t launch_ivf_sort(const IvfParams &p, bool copy_rows, cudaStream_t s) {
+  ivf_chunk_count_kernel<<<dim3(static_cast<unsigned>(p.nsort), static_cast<unsigned>(p.BH)), 256,
+                           static_cast<size_t>(p.nlist) * 4, s>>>(p);
+  ivf_slots_kernel<<<p.BH, 1024, 0, s>>>(p);
+  const long long warps = static_cast<long long>(p.BH) * p.nsort;
+  const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
+  if (p.d == 128) ivf_stable_scatter_kernel<128><<<grid, 256, 0, s>>>(p, copy_rows ? 1 : 0);
+  else ivf_stable_scatter_kernel<64><<<grid, 256, 0, s>>>(p, copy_rows ? 1 : 0);
   return cudaGetLastError();
 }
 cudaError_t launch_ivf_update(const IvfParams &p, cudaStream_t s) {
-  ivf_update_kernel<<<dim3(p.nlist, p.BH), 128, 0, s>>>(p);
-  return cudaGetLastError();
-}
-cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s) {
-  ivf_offsets_kernel<<<p.BH, 1024, 0, s>>>(p);
-  const long long warps = static_cast<long long>(p.BH) * p.N;
-  ivf_scatter_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, s>>>(p);
+  const long long warps = static_cast<long long>(p.BH) * p.nlist;
+  const unsigned grid = static_cast<unsigned>((warps + 7) / 8);
+  if (p.d == 128) ivf_update_kernel<128><<<grid, 256, 0, s>>>(p);
+  else ivf_update_kernel<64><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s) {

@@ -124,19 +124,20 @@ struct PfParams {
 };
 constexpr uint32_t kErrPrefillWait = 8u;
 
-// IVF index build over one layer's keys (per KV head, bg = b * Hkv + g).
+// IVF index build over one layer's keys (per KV head, bg = b * Hkv + g).  Every step is
+// deterministic: integer counts, a stable counting sort and fixed-order sums.
+constexpr int kIvfSortChunk = 1024;   // keys one warp places in the stable scatter
 struct IvfParams {
   const __nv_bfloat16 *K;   // cache keys [BH, cap, d]
   __nv_bfloat16 *cent;      // [BH, nlist, d] unit-norm centroids
-  const float *A;           // [BH * N, ldA] key-centroid scores of the current iteration
-  float *sums;              // [BH, nlist, d]
-  uint32_t *count, *cursor; // [BH, nlist]
-  int32_t *assign;          // [BH * N]
+  const float *A;           // [BH * M, ldA] key-centroid scores of the key chunk [c0, c0 + M)
+  int32_t *assign;          // [BH * N] cluster of each key
+  uint32_t *chunk_cnt;      // [BH, nsort, nlist]: per sort chunk, counts, then first slots
   int32_t *offsets;         // [BH, nlist + 1]
   int32_t *pos;             // [BH, N] cache position of each sorted key
-  __nv_bfloat16 *Ksorted;   // [BH, N, d]
-  long long N, cap, ldA;
-  int BH, nlist, d;
+  __nv_bfloat16 *Ksorted;   // [BH, N, d] (written by the final sort)
+  long long N, cap, ldA, c0, M;
+  int BH, nlist, d, nsort;
 };
 
 // IVF search of one decode step (rows = b * Hq + h).
@@ -204,9 +205,9 @@ cudaError_t launch_select_attend_paged(const SaParams &p, const PagedInfo &pg, i
 cudaError_t launch_dense(const DenseParams &p, int d, cudaStream_t s);
 cudaError_t launch_prefill_score(const PfParams &p, int d, cudaStream_t s);
 cudaError_t launch_ivf_init(const IvfParams &p, cudaStream_t s);
-cudaError_t launch_ivf_assign(const IvfParams &p, bool accumulate, cudaStream_t s);
+cudaError_t launch_ivf_assign(const IvfParams &p, cudaStream_t s);   // keys [c0, c0 + M)
+cudaError_t launch_ivf_sort(const IvfParams &p, bool copy_rows, cudaStream_t s);
 cudaError_t launch_ivf_update(const IvfParams &p, cudaStream_t s);
-cudaError_t launch_ivf_sort(const IvfParams &p, cudaStream_t s);
 cudaError_t launch_ivf_probe(const IvfSearchParams &p, cudaStream_t s);
 cudaError_t launch_ivf_cand(const IvfSearchParams &p, int d, cudaStream_t s);
 cudaError_t launch_append(const AppendParams &p, cudaStream_t s);

@@ -734,20 +734,30 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
 
 // ---- IVF index
 
+// Build workspace: the key-centroid scores of one chunk of keys (at most kIvfScoreBytes, so the
+// workspace stays bounded at any N), the assignment, and the sort's per-chunk slot table.
+static constexpr size_t kIvfScoreBytes = size_t(256) << 20;
+
 struct IvfBuildLayout {
-  size_t off_A, off_sums, off_count, off_cursor, off_assign, off_err, total;
-  long long ldA;
+  size_t off_A, off_assign, off_cc, off_err, total;
+  long long ldA, M;   // score row stride, keys scored per chunk
+  int nsort;          // sort chunks per head
 };
 static bool ivf_build_layout(int B, int Hkv, long long N, int d, int nlist, IvfBuildLayout &L) {
   if (B < 1 || Hkv < 1 || N < 1 || (d != 64 && d != 128) || nlist < 1 || nlist > 4096) return false;
+  if (N >= (1LL << 31) - 1) return false;
   const size_t BH = static_cast<size_t>(B) * Hkv;
   L.ldA = round4(nlist);
+  // keys per score chunk: a multiple of the 128-row score tile, at least one tile
+  const long long per_row = static_cast<long long>(BH) * L.ldA * 4;
+  long long M = static_cast<long long>(kIvfScoreBytes) / per_row / 128 * 128;
+  if (M < 128) M = 128;
+  L.M = std::min<long long>(M, N);
+  L.nsort = static_cast<int>((N + kIvfSortChunk - 1) / kIvfSortChunk);
   size_t off = 0;
-  L.off_A = off;      off = align_up(off + BH * N * L.ldA * 4);
-  L.off_sums = off;   off = align_up(off + BH * nlist * d * 4);
-  L.off_count = off;  off = align_up(off + BH * nlist * 4);
-  L.off_cursor = off; off = align_up(off + BH * nlist * 4);
+  L.off_A = off;      off = align_up(off + BH * L.M * L.ldA * 4);
   L.off_assign = off; off = align_up(off + BH * N * 4);
+  L.off_cc = off;     off = align_up(off + BH * L.nsort * nlist * 4);
   L.off_err = off;    off = align_up(off + 4);
   L.total = off;
   return true;
@@ -775,33 +785,37 @@ ra_status ra_ivf_build(const ra_kv *kv, ra_ivf *ix, int32_t iters, void *ws, siz
   p.K = static_cast<const __nv_bfloat16 *>(kv->K);
   p.cent = static_cast<__nv_bfloat16 *>(ix->centroids);
   p.A = reinterpret_cast<const float *>(at(ws, L.off_A));
-  p.sums = reinterpret_cast<float *>(at(ws, L.off_sums));
-  p.count = reinterpret_cast<uint32_t *>(at(ws, L.off_count));
-  p.cursor = reinterpret_cast<uint32_t *>(at(ws, L.off_cursor));
   p.assign = reinterpret_cast<int32_t *>(at(ws, L.off_assign));
+  p.chunk_cnt = reinterpret_cast<uint32_t *>(at(ws, L.off_cc));
   p.offsets = ix->offsets;
   p.pos = ix->pos;
   p.Ksorted = static_cast<__nv_bfloat16 *>(ix->Ksorted);
   p.N = ix->N; p.cap = kv->cap; p.ldA = L.ldA;
-  p.BH = kv->B * kv->Hkv; p.nlist = ix->nlist; p.d = kv->d;
-  // the key-centroid scores: the keys as the query rows of the tensor-core score kernel
+  p.BH = kv->B * kv->Hkv; p.nlist = ix->nlist; p.d = kv->d; p.nsort = L.nsort;
+  // the key-centroid scores of a chunk of keys: those keys as the query rows of the
+  // tensor-core score kernel, the centroids as its keys
   PfParams f{};
-  f.Q = static_cast<const __nv_bfloat16 *>(kv->K);
   f.K = p.cent;
   f.S = reinterpret_cast<float *>(at(ws, L.off_A));
   f.err = reinterpret_cast<uint32_t *>(at(ws, L.off_err));
   f.N = ix->nlist; f.cap = ix->nlist; f.ldS = L.ldA; f.q_plane_rows = kv->cap;
-  f.B = kv->B; f.Hq = kv->Hkv; f.Hkv = kv->Hkv; f.G = 1; f.M = static_cast<int>(ix->N);
+  f.B = kv->B; f.Hq = kv->Hkv; f.Hkv = kv->Hkv; f.G = 1;
   f.scale = 1.0f;
-  cudaError_t e = cudaMemsetAsync(at(ws, L.off_sums), 0, L.off_assign - L.off_sums, cs);
-  if (e == cudaSuccess) e = cudaMemsetAsync(at(ws, L.off_err), 0, 4, cs);
+  cudaError_t e = cudaMemsetAsync(at(ws, L.off_err), 0, 4, cs);
   if (e == cudaSuccess) e = launch_ivf_init(p, cs);
   for (int it = 0; it <= iters && e == cudaSuccess; ++it) {
-    e = launch_prefill_score(f, kv->d, cs);
-    if (e == cudaSuccess) e = launch_ivf_assign(p, it < iters, cs);
+    for (long long c0 = 0; c0 < ix->N && e == cudaSuccess; c0 += L.M) {
+      const long long m = std::min<long long>(L.M, ix->N - c0);
+      f.Q = static_cast<const __nv_bfloat16 *>(kv->K) + c0 * kv->d;
+      f.M = static_cast<int>(m);
+      e = launch_prefill_score(f, kv->d, cs);
+      p.c0 = c0;
+      p.M = m;
+      if (e == cudaSuccess) e = launch_ivf_assign(p, cs);
+    }
+    if (e == cudaSuccess) e = launch_ivf_sort(p, it == iters, cs);
     if (e == cudaSuccess && it < iters) e = launch_ivf_update(p, cs);
   }
-  if (e == cudaSuccess) e = launch_ivf_sort(p, cs);
   return e == cudaSuccess ? RA_OK : cuda_fail(e, "ivf_build");
 }
 
