@@ -96,7 +96,8 @@ const char *ra_status_str(ra_status s);
 /* Library version string (static). */
 const char *ra_version(void);
 
-/* Detail of the last RA_ERR_CUDA on the calling thread (static thread-local string). */
+/* Detail of the last RA_ERR_CUDA on the calling thread, or of a refused first call of
+ * ra_decode_step_static inside a stream capture (static thread-local string). */
 const char *ra_last_error(void);
 
 /*
@@ -251,7 +252,9 @@ ra_status ra_select_attend(const ra_kv *kv, int32_t Hq, int32_t k, int32_t n_sin
  *     ra_decode_workspace_bytes(...) exceeds 64 MiB is rejected with RA_ERR_WORKSPACE before
  *     anything is enqueued (the 128K Llama-3-8B layer, 32 query heads, needs about 48 MiB).
  *   The first call on each device looks up the array's device address (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream capture.
+ *     with that device current); make that first call before any stream capture.  A first
+ *     call on a capturing stream is refused with RA_ERR_ARG (ra_last_error() says why) and
+ *     enqueues nothing.  Host threads may make first calls concurrently.
  *   Each call clears the scratch's counter block with cudaMemsetAsync on `stream`; nothing is
  *     allocated.  All calls on a device share the one array and it keeps the last call's
  *     contents, so calls that overlap on the GPU (other streams, other host threads) race.

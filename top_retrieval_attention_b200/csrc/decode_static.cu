@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/ra.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -25,7 +27,9 @@ __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
 // Device address of g_scratch per device.  In host code `g_scratch` names a host-side stand-in,
 // not device memory, so the address is looked up once per device with that device current.
-void *g_scratch_addr[64] = {};
+// Host threads may make their first calls at the same time: the cache is atomic (two threads
+// may both look the address up; both store the same value).
+std::atomic<void *> g_scratch_addr[64] = {};
 
 }  // namespace
 
@@ -45,12 +49,20 @@ extern "C" ra_status ra_decode_step_static(const ra_kv *kv, const void *q, int32
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RA_ERR_CUDA;
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return RA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void *ws = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (ws == nullptr) {
+    // the look-up is a runtime call that a stream capture may not allow: refuse it there
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(reinterpret_cast<cudaStream_t>(stream), &cap) != cudaSuccess)
+      return RA_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone) {
+      ra::set_last_error("ra_decode_step_static: the first call on a device must come before "
+                         "any stream capture (it looks up the scratch's device address)");
+      return RA_ERR_ARG;
+    }
+    if (cudaGetSymbolAddress(&ws, g_scratch) != cudaSuccess || ws == nullptr) return RA_ERR_CUDA;
+    g_scratch_addr[dev].store(ws, std::memory_order_release);
   }
-  void *ws = g_scratch_addr[dev];
 
   // The counter block at the front of the workspace (per query head: histogram and
   // counters) must start at zero; clear it on every call rather than trusting the last one.

@@ -177,6 +177,9 @@ constexpr int kDenseTile = 128;
 
 int num_sms();
 
+// Sets the calling thread's ra_last_error() text.
+void set_last_error(const char *msg);
+
 // Bytes of the counter block at the front of every workspace for `rows` query heads (the
 // digit-1 histograms, then the per-row counters), 256-byte aligned sections.
 size_t counter_block_bytes(size_t rows);

@@ -15,6 +15,8 @@ namespace ra {
 
 static thread_local char g_last_error[256] = "";
 
+void set_last_error(const char *msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 static ra_status cuda_fail(cudaError_t e, const char *where) {
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e),
            static_cast<int>(e));
