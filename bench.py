@@ -1,10 +1,12 @@
 #!/usr/bin/env python
 """Decode-step benchmark of exact top-k retrieval attention on B200.
 
-A step is one pass of the whole hot path for every layer of the workload: append the new
-token's K/V row and score all positions (ra_score_gqa_append: the append runs inside the
-scan), then select the top-k per query head and attend over sinks + window + top-k
-(ra_select_attend); together they are ra_decode_step_append.  The cache holds N-1 tokens; each
+A step is one pass of the whole hot path for every layer of the workload, one
+ra_decode_step_append call per layer: append the new token's K/V row and score all positions
+(the append runs inside the scan), then select the top-k per query head and attend over sinks +
+window + top-k (the selection launched behind the scan starts on each KV head as the scan
+finishes it).  A phase pass after the timed region runs the scan (ra_score_gqa_append) and the
+selection (ra_select_attend) as separate calls to time each.  The cache holds N-1 tokens; each
 step appends the N-th and decodes over N, then the next step re-appends into the same slot, so
 every step has identical work.  Each step uses its own query.  (The threshold mode, --eps,
 appends with ra_append_kv and runs ra_decode_step_eps.)
@@ -12,11 +14,13 @@ appends with ra_append_kv and runs ra_decode_step_eps.)
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 Rank 0 prints one JSON line.  `value` is whole-job decode steps/s with the caches resident in
-HBM; `e2e` is the same metric through the public Python API with the step's inputs (query,
-new K/V row) copied from pinned host memory and the outputs (out, idx) copied back and waited
-for inside the timed region; `roofline` is the score kernel (the K scan, the dominant kernel)
-against the measured HBM copy bandwidth; `cpu_baseline` is the fp64 oracle on a bounded sample
-timed on the host cores.  `--impl reference` times only the oracle (the reference arm).
+HBM; `e2e` is the same metric through the C ABI's host-buffer step (ra_decode_step_append_host)
+with the step's inputs (query, new K/V row) copied from pinned host memory and the outputs
+(out, idx) copied back and waited for inside the timed region; `roofline` is the score kernel
+(the K scan, the dominant kernel) against the measured HBM copy bandwidth; `cpu_baseline` is the
+fp64 oracle on a bounded sample timed on the host cores; `configs` holds the 32-layer 1M-token
+cache and the batch-16 256K layer, measured the same way in the same run.  `--impl reference`
+times only the oracle (the reference arm).
 Under torchrun each rank runs an independent replica (the step does not shard across GPUs).
 """
 from __future__ import annotations
@@ -72,6 +76,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the 1M x 32-layer and batch-16 workloads the default line also reports")
     ap.add_argument("--eps", type=float, default=0.0,
                     help="threshold budget: keep candidates whose softmax weight exceeds eps "
                          "(at most k per head; ra_decode_step_eps)")
@@ -232,7 +238,7 @@ def oracle_sample(w, seconds: float):
     step_s = statistics.median(times) * scale
     desc = (f"oracle decode of the {w.G} query heads of KV head 0 (layer 0, b 0) over all "
             f"{w.N} keys, median of {len(times)} runs, x{scale} for the whole step")
-    return 1.0 / step_s, _blas_threads(), desc
+    return 1.0 / step_s, _blas_threads(), desc, sum(times)
 
 
 def run_reference(args, w, rank, world):
@@ -256,10 +262,12 @@ def run_reference(args, w, rank, world):
     k_s = w.k if n_keys == w.N else max(1, int(round(w.k * n_keys / w.N)))
     scale = (w.N / n_keys) * w.Hkv * w.B * w.layers
     vals = []
+    timed = 0.0
     for i in range(warm + steps):
         t = _oracle_group_seconds(w, qh, K, V, k_s)
         if i >= warm:
             vals.append(1.0 / (t * scale))
+            timed += t
     value = statistics.median(vals)
     desc = (f"per step: oracle decode of the {w.G} query heads of KV head 0 (layer 0, b 0) over "
             f"keys [0, {n_keys}) of {w.N} with k={k_s}, scaled x{scale:.1f} to one whole step")
@@ -268,8 +276,14 @@ def run_reference(args, w, rank, world):
         "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": 1000.0 / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w),
+        "sampled": True,
+        "steps_note": (f"each of the {steps} timed steps runs the oracle on one sample of the "
+                       f"workload ({desc}); ms_per_step is the scaled whole-step time, not the "
+                       f"time the samples took"),
+        "timed_seconds": timed,
         "cpu_baseline": {"value": value, "unit": "steps/s", "cores": _blas_threads(),
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "sample": desc, "sampled": True,
+                         "timed_seconds": timed},
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -527,7 +541,8 @@ def run_ours(args, w, rank, local_rank, world, dist):
             c.N = N - 1
         del dws
 
-    # end to end through the public Python API, inputs from pinned host memory
+    # end to end through the C ABI's host-buffer step (the threshold mode: the Python API), the
+    # step's inputs from pinned host memory and its outputs back there, waited for every step
     if not args.no_e2e:
         esteps = max(5, min(steps, 1000))
         hq = torch.empty((P, L, B, Hq, d), dtype=torch.bfloat16).pin_memory()
@@ -540,20 +555,29 @@ def run_ours(args, w, rank, local_rank, world, dist):
         ho = torch.empty((L, B, Hq, d), dtype=torch.float32).pin_memory()
         hi = [torch.empty((B, Hq, max(kl, 1)), dtype=torch.int32).pin_memory() for kl in ks]
 
+        ios = [ra.ra_step_io(dq[layer].data_ptr(), dk[layer].data_ptr(), dv[layer].data_ptr(),
+                             outs[layer].data_ptr(), idxs[layer].data_ptr()) for layer in range(L)]
+
         def e2e_step(s):
+            if args.eps <= 0:
+                # one C call per layer: the step's query and token rows from pinned host memory,
+                # the step, and out / idx back to pinned host memory, all on the stream
+                for layer in range(L):
+                    ra.check(ra.ra_decode_step_append_host(
+                        caches[layer].kv, hq[s % P, layer].data_ptr(), hk[layer].data_ptr(),
+                        hv[layer].data_ptr(), Hq, ks[layer], w.n_sink, w.n_window,
+                        ho[layer].data_ptr(), hi[layer].data_ptr(), ios[layer], ws.data_ptr(),
+                        ws_bytes, sp), "decode_step_append_host")
+                    caches[layer].N = N - 1
+                stream.synchronize()
+                return
             dq.copy_(hq[s % P], non_blocking=True)
             for layer in range(L):
                 dk[layer].copy_(hk[layer], non_blocking=True)
                 dv[layer].copy_(hv[layer], non_blocking=True)
-                if args.eps <= 0:
-                    ra.decode_step_append(caches[layer], dq[layer], dk[layer], dv[layer], ks[layer],
-                                          w.n_sink, w.n_window, out=outs[layer], idx=idxs[layer],
-                                          ws=ws)
-                else:
-                    ra.append_kv(caches[layer], dk[layer], dv[layer])
-                if args.eps > 0:
-                    ra.decode_step_eps(caches[layer], dq[layer], ks[layer], args.eps, w.n_sink,
-                                       w.n_window, out=outs[layer], idx=idxs[layer], ws=ws)
+                ra.append_kv(caches[layer], dk[layer], dv[layer])
+                ra.decode_step_eps(caches[layer], dq[layer], ks[layer], args.eps, w.n_sink,
+                                   w.n_window, out=outs[layer], idx=idxs[layer], ws=ws)
                 caches[layer].N = N - 1
                 ho[layer].copy_(outs[layer], non_blocking=True)
                 hi[layer].copy_(idxs[layer], non_blocking=True)
@@ -574,14 +598,15 @@ def run_ours(args, w, rank, local_rank, world, dist):
         result["e2e"] = {"value": world * 1000.0 / e2e_ms, "unit": "steps/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": esteps,
                          "ms_per_step": e2e_ms,
-                         "note": ("public API (decode_step_append" if args.eps <= 0 else
-                                  "public API (append_kv + decode_step_eps") +
-                                 "), host sync every step"}
+                         "note": ("C ABI ra_decode_step_append_host with pinned host buffers (copies in, "
+                                  "step, copies out on the stream)" if args.eps <= 0 else
+                                  "public API (append_kv + decode_step_eps)") +
+                                 ", host sync every step"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc = oracle_sample(w, args.cpu_seconds)
+        v, cores, desc, spent = oracle_sample(w, args.cpu_seconds)
         result["cpu_baseline"] = {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                                  "sample": desc}
+                                  "sample": desc, "sampled": True, "timed_seconds": spent}
     return result
 
 
@@ -935,6 +960,35 @@ def run_prefill(args, w, rank, local_rank, world, dist):
     }
 
 
+# The other workloads of the decode-step suite reported in the default line (the 32-layer 1M
+# cache and the batch-16 256K layer), each measured in this same run the way the headline is.
+EXTRA_CONFIGS = ("l8b_1m_32layer", "l8b_b16_256k")
+
+
+def extra_configs(args, rank, local_rank, world, dist):
+    import copy
+    import gc
+
+    import torch
+
+    from synth import gen
+    out = {}
+    for name in EXTRA_CONFIGS:
+        a = copy.copy(args)
+        a.steps, a.warmup, a.no_e2e, a.no_cpu_baseline = None, 3, True, True
+        r = run_ours(a, gen.workload(name), rank, local_rank, world, dist)
+        out[name] = {k: r[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup",
+                                       "step_frac_of_peak", "step_frac_of_nominal_8tbs",
+                                       "score_kernel_us", "gpu_launches", "clocks", "config")}
+        out[name]["score_kernel_frac_of_peak"] = r["roofline"]["frac"]
+        if "dense" in r:
+            out[name]["dense_ms_per_step"] = r["dense"]["ms_per_step"]
+            out[name]["speedup_over_dense"] = r["dense"]["speedup_of_sparse_decode"]
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     rank, local_rank, world = dist_info()
@@ -967,6 +1021,9 @@ def main():
             res = run_paged(args, w, rank, local_rank, world, dist)
         else:
             res = run_ours(args, w, rank, local_rank, world, dist)
+            if (world == 1 and not args.no_configs and args.workload == DEFAULT_WORKLOAD and
+                    args.eps <= 0 and args.pyramid <= 0):
+                res["configs"] = extra_configs(args, rank, local_rank, world, dist)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -158,6 +158,31 @@ ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, con
                                 float *out, int32_t *idx, void *ws, size_t ws_bytes,
                                 ra_stream_t stream);
 /*
+ * ra_decode_step_append for a caller whose step inputs and outputs live in host memory: the
+ * query and the token's K / V rows are copied from host memory into the caller's device
+ * staging buffers, the step runs, and out and idx are copied back, all enqueued on `stream`
+ * (one cudaMemcpyAsync per buffer); nothing waits on the host, so the caller synchronises
+ * `stream` before reading out_host / idx_host.  Host buffers should be pinned (page-locked)
+ * for the copies to be asynchronous.
+ *   dev : device staging of the step's inputs and outputs (shapes and alignment as
+ *         ra_decode_step_append's q, k_new, v_new, out, idx), caller-owned.
+ *   q_host bf16 [B, Hq, d]; k_new_host, v_new_host bf16 [B, Hkv, 1, d]; out_host fp32
+ *   [B, Hq, d]; idx_host int32 [B, Hq, k] (may be null when k = 0).
+ * Errors: as ra_decode_step_append, checked before anything is enqueued; RA_ERR_ARG for a
+ * null host pointer; RA_ERR_CUDA if a copy cannot be enqueued.
+ */
+typedef struct {
+  void *q, *k_new, *v_new;
+  float *out;
+  int32_t *idx;
+} ra_step_io;
+ra_status ra_decode_step_append_host(ra_kv *kv, const void *q_host, const void *k_new_host,
+                                     const void *v_new_host, int32_t Hq, int32_t k,
+                                     int32_t n_sink, int32_t n_window, float *out_host,
+                                     int32_t *idx_host, const ra_step_io *dev, void *ws,
+                                     size_t ws_bytes, ra_stream_t stream);
+
+/*
  * Kernel launches that ra_decode_step (or ra_decode_step_append) makes for this shape: 2 (the
  * scan, then the selection fused with the attention) or 3 (the attention split across several
  * clusters per head, as a launch of its own).  Host only; it queries the current device's

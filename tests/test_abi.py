@@ -209,3 +209,28 @@ def test_prefill_rejects_bad_arguments():
     assert L.ra_prefill_topk(ctypes.byref(kv), FAKE, 4, 8, 10, 4, 8, FAKE, FAKE, 10, None) == ra.RA_ERR_WORKSPACE
     assert ra.ra_prefill_workspace_bytes(1, 4, 8, 100, 128, 10, 4, 8) > 4 * 8 * 100 * 4
     assert ra.ra_prefill_workspace_bytes(1, 4, 0, 100, 128, 10, 4, 8) == 0
+
+
+def test_host_buffer_step_refuses_before_enqueuing():
+    """ra_decode_step_append_host checks everything ra_decode_step_append checks, plus its
+    host pointers, before the first copy: with a full cache or a null host buffer it returns an
+    error and leaves kv unchanged."""
+    H = (ctypes.c_uint16 * 4096)()
+    O = (ctypes.c_float * 4096)()
+    I = (ctypes.c_int32 * 4096)()
+    dev = ra.ra_step_io(FAKE, FAKE, FAKE, FAKE, FAKE)
+    ws_ok = 1 << 30
+    ws = FAKE << 8   # 256-byte aligned
+    full = _kv(N=100)   # N == cap: no room for the token
+    st = ra.ra_decode_step_append_host(full, H, H, H, 4, 8, 4, 16, O, I, dev, ws, ws_ok, None)
+    assert st == ra.RA_ERR_CAPACITY and full.N == 100
+    kv = _kv(N=50)
+    st = ra.ra_decode_step_append_host(kv, None, H, H, 4, 8, 4, 16, O, I, dev, ws, ws_ok, None)
+    assert st == ra.RA_ERR_ARG and kv.N == 50
+    st = ra.ra_decode_step_append_host(kv, H, H, H, 4, 8, 4, 16, O, None, dev, ws, ws_ok, None)
+    assert st == ra.RA_ERR_ARG and kv.N == 50
+    bad = ra.ra_step_io(FAKE, FAKE + 8, FAKE, FAKE, FAKE)          # misaligned device k_new
+    st = ra.ra_decode_step_append_host(kv, H, H, H, 4, 8, 4, 16, O, I, bad, ws, ws_ok, None)
+    assert st == ra.RA_ERR_ARG and kv.N == 50
+    st = ra.ra_decode_step_append_host(kv, H, H, H, 4, 8, 4, 16, O, I, dev, ws, 256, None)
+    assert st == ra.RA_ERR_WORKSPACE and kv.N == 50

@@ -10,4 +10,5 @@ from .ra import (  # noqa: F401
     ra_decode_step_eps, decode_step_eps, pyramid_budgets, ra_paged_kv, PagedKVCache,
     paged_append_kv, paged_workspace, paged_decode_step, ra_ivf, IvfIndex, ivf_build,
     ivf_decode_step, ra_decode_step_append, ra_score_gqa_append, decode_step_append,
+    ra_decode_step_append_host, ra_step_io,
 )

@@ -351,6 +351,38 @@ ra_status ra_decode_step_append(ra_kv *kv, const void *q, const void *k_new, con
   return run_select_attend(&grown, st, kSaSelect | kSaAttend, idx, out, ws, cs, 0.f, target);
 }
 
+ra_status ra_decode_step_append_host(ra_kv *kv, const void *q_host, const void *k_new_host,
+                                     const void *v_new_host, int32_t Hq, int32_t k,
+                                     int32_t n_sink, int32_t n_window, float *out_host,
+                                     int32_t *idx_host, const ra_step_io *dev, void *ws,
+                                     size_t ws_bytes, ra_stream_t stream) {
+  if (!dev || !q_host || !k_new_host || !v_new_host || !out_host || (k > 0 && !idx_host))
+    return RA_ERR_ARG;
+  // every check of the step first (nothing enqueued, kv unchanged on an error)
+  ra_kv grown{};
+  Step st{};
+  ra_status s = plan_append_step(kv, dev->k_new, dev->v_new, Hq, k, n_sink, n_window, ws, ws_bytes,
+                                 grown, st);
+  if (s != RA_OK) return s;
+  if (!dev->q || !aligned16(dev->q) || !dev->out || !aligned16(dev->out)) return RA_ERR_ARG;
+  if (k > 0 && (!dev->idx || !aligned16(dev->idx))) return RA_ERR_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t qb = static_cast<size_t>(kv->B) * Hq * kv->d * 2;
+  const size_t rowb = static_cast<size_t>(kv->B) * kv->Hkv * kv->d * 2;
+  const size_t ob = static_cast<size_t>(kv->B) * Hq * kv->d * 4;
+  const size_t ib = static_cast<size_t>(kv->B) * Hq * (k > 0 ? k : 0) * 4;
+  cudaError_t e = cudaMemcpyAsync(dev->q, q_host, qb, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->k_new, k_new_host, rowb, cudaMemcpyHostToDevice, cs);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->v_new, v_new_host, rowb, cudaMemcpyHostToDevice, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_step_append_host: copy in");
+  s = ra_decode_step_append(kv, dev->q, dev->k_new, dev->v_new, Hq, k, n_sink, n_window, dev->out,
+                            dev->idx, ws, ws_bytes, stream);
+  if (s != RA_OK) return s;
+  e = cudaMemcpyAsync(out_host, dev->out, ob, cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess && ib > 0) e = cudaMemcpyAsync(idx_host, dev->idx, ib, cudaMemcpyDeviceToHost, cs);
+  return e == cudaSuccess ? RA_OK : cuda_fail(e, "decode_step_append_host: copy out");
+}
+
 int32_t ra_decode_step_launches(int32_t B, int32_t Hq, int32_t Hkv, int64_t N, int32_t d,
                                 int32_t k, int32_t n_sink, int32_t n_window) {
   Step st{};

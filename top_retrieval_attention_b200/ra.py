@@ -26,7 +26,7 @@ EXPORTS = ("ra_status_str", "ra_version", "ra_last_error", "ra_append_kv",
            "ra_paged_append_kv", "ra_paged_workspace_bytes", "ra_paged_decode_step",
            "ra_ivf_build_workspace_bytes", "ra_ivf_build", "ra_ivf_search_workspace_bytes",
            "ra_ivf_decode_step", "ra_decode_step_append", "ra_score_gqa_append",
-           "ra_decode_step_launches")
+           "ra_decode_step_launches", "ra_decode_step_append_host")
 
 
 class ra_kv(ctypes.Structure):
@@ -38,6 +38,11 @@ class ra_paged_kv(ctypes.Structure):
     _fields_ = [("K", c_void_p), ("V", c_void_p), ("block_table", c_void_p),
                 ("seq_len", ctypes.POINTER(c_int32)), ("B", c_int32), ("Hkv", c_int32),
                 ("d", c_int32), ("max_pages", c_int32), ("num_pages", c_int32)]
+
+
+class ra_step_io(ctypes.Structure):
+    _fields_ = [("q", c_void_p), ("k_new", c_void_p), ("v_new", c_void_p), ("out", c_void_p),
+                ("idx", c_void_p)]
 
 
 class ra_ivf(ctypes.Structure):
@@ -114,6 +119,10 @@ def lib() -> ctypes.CDLL:
                                               c_int32, c_int32, c_void_p, c_size_t, c_void_p]),
             "ra_decode_step_launches": (c_int32, [c_int32, c_int32, c_int32, c_int64, c_int32,
                                                   c_int32, c_int32, c_int32]),
+            "ra_decode_step_append_host": (c_int32, [P, c_void_p, c_void_p, c_void_p, c_int32,
+                                                     c_int32, c_int32, c_int32, c_void_p, c_void_p,
+                                                     ctypes.POINTER(ra_step_io), c_void_p, c_size_t,
+                                                     c_void_p]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -267,6 +276,13 @@ def ra_decode_step_append(kv, q, k_new, v_new, Hq, k, n_sink, n_window, out, idx
                           stream):
     return lib().ra_decode_step_append(ctypes.byref(kv), q, k_new, v_new, Hq, k, n_sink, n_window,
                                        out, idx, ws, ws_bytes, stream)
+
+
+def ra_decode_step_append_host(kv, q_host, k_new_host, v_new_host, Hq, k, n_sink, n_window,
+                               out_host, idx_host, dev, ws, ws_bytes, stream):
+    return lib().ra_decode_step_append_host(ctypes.byref(kv), q_host, k_new_host, v_new_host, Hq,
+                                            k, n_sink, n_window, out_host, idx_host,
+                                            ctypes.byref(dev), ws, ws_bytes, stream)
 
 
 def ra_score_gqa_append(kv, q, k_new, v_new, Hq, k, n_sink, n_window, ws, ws_bytes, stream):
