@@ -377,53 +377,28 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
   if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);   // unreachable for distinct keys
 }
 
-// The score at bit j of a thread's hit mask: element j % 4 of its (j / 4)-th loaded vector,
-// picked from registers (no dynamic indexing).
-__device__ __forceinline__ float pick_score(const float4 (&v)[kStreamVec], int j) {
-  float r = 0.f;
+// Inclusive warp prefix sums of two per-lane counts; the warp totals come back in lane 31.
+__device__ __forceinline__ void warp_scan2(uint32_t &a, uint32_t &b) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int u = 0; u < kStreamVec; ++u) {
-    const int e = j - 4 * u;
-    r = e == 0 ? v[u].x : e == 1 ? v[u].y : e == 2 ? v[u].z : e == 3 ? v[u].w : r;
-  }
-  return r;
-}
-
-// Appends this lane's hit (if any) with one shared atomic per list and warp: all 32 lanes call
-// it together.  Keys above b1 go to the sure array (positions); keys in b1 go to the list as
-// composites, past its capacity to `spill`, with their digit-2 histogram in sm.h.  The
-// counters keep counting past the capacities.
-template <int D>
-__device__ __forceinline__ void place_hit(SaSmem<D> &sm, unsigned long long *spill, bool has,
-                                          uint32_t pos, float z, uint32_t b1, uint32_t lt) {
-  const uint32_t key = order_key(z);
-  const uint32_t d1 = key >> (32 - kHistBits);
-  const bool up = has && d1 > b1, eq = has && d1 == b1;
-  const uint32_t mu = __ballot_sync(0xffffffffu, up), me = __ballot_sync(0xffffffffu, eq);
-  uint32_t bu = 0, be = 0;
-  if ((threadIdx.x & 31) == 0) {
-    if (mu) bu = atomicAdd(&sm.n_sure, static_cast<uint32_t>(__popc(mu)));
-    if (me) be = atomicAdd(&sm.n_list, static_cast<uint32_t>(__popc(me)));
-  }
-  bu = __shfl_sync(0xffffffffu, bu, 0);
-  be = __shfl_sync(0xffffffffu, be, 0);
-  if (up) {
-    const uint32_t o = bu + __popc(mu & lt);
-    if (o < static_cast<uint32_t>(kSureCap)) sm.sure[o] = pos;
-  }
-  if (eq) {
-    const uint32_t o = be + __popc(me & lt);
-    const unsigned long long x = composite(key, pos);
-    if (o < static_cast<uint32_t>(kListSmem)) sm.list[o] = x;
-    else spill[o] = x;
-    atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t na = __shfl_up_sync(0xffffffffu, a, o);
+    const uint32_t nb = __shfl_up_sync(0xffffffffu, b, o);
+    if (lane >= o) {
+      a += na;
+      b += nb;
+    }
   }
 }
 
-// One pass over the CTA's candidates [lo, hi) of the score row, placing every key at or above
-// the bottom of the digit-1 threshold bin b1 (place_hit).  Hits are a few percent of the keys:
-// each thread makes a bit mask of its hits with one compare per score, and the warp places
-// them in lock-step rounds, each lane's score picked from its registers.
+// One pass over the CTA's candidates [lo, hi) of the score row.  Keys above the digit-1
+// threshold bin b1 (z >= zhi, the bottom of bin b1 + 1) go to sm.sure as positions; keys in b1
+// (zlo <= z < zhi) go to sm.list as composites, past its capacity to `spill` (room for hi - lo
+// entries), with their digit-2 histogram in sm.h; the counters keep counting past the
+// capacities.  Hits are a few percent of the keys: each thread makes two bit masks with two
+// compares per score, the warp reserves its slots with one shared atomic per list and
+// iteration (offsets from a warp prefix scan of the per-lane counts), and every lane then
+// writes its own hits straight from its registers.
 template <int D>
 __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
                                              unsigned long long *spill, long long a0, long long lo,
@@ -431,7 +406,9 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
   constexpr long long kStep = 4LL * kSaThreads * kStreamVec;
   static_assert(4 * kStreamVec <= 32, "one mask bit per score");
   const float zlo = key_float(b1 << (32 - kHistBits));
-  const uint32_t lt = lanemask_lt();
+  const float zhi = b1 + 1 < static_cast<uint32_t>(kHistBins)
+                        ? key_float((b1 + 1) << (32 - kHistBits)) : INFINITY;
+  const int lane = threadIdx.x & 31;
   for (long long it = a0; it < hi; it += kStep) {
     const long long b0 = it + 4LL * threadIdx.x;
     float4 v[kStreamVec];
@@ -442,25 +419,62 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     const bool interior = it >= lo && it + kStep <= hi;
-    uint32_t m = 0;
+    uint32_t ms = 0, me = 0;   // above b1, in b1
 #pragma unroll
     for (int u = 0; u < kStreamVec; ++u) {
-      uint32_t bits = (v[u].x >= zlo ? 1u : 0u) | (v[u].y >= zlo ? 2u : 0u) |
-                      (v[u].z >= zlo ? 4u : 0u) | (v[u].w >= zlo ? 8u : 0u);
+      const float zz[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t s4 = 0, e4 = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s4 |= (zz[e] >= zhi ? 1u : 0u) << e;
+        e4 |= (zz[e] >= zlo && zz[e] < zhi ? 1u : 0u) << e;
+      }
       if (!interior) {
         const long long b = b0 + 4LL * kSaThreads * u;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (b + e < lo || b + e >= hi) bits &= ~(1u << e);
+          if (b + e < lo || b + e >= hi) {
+            s4 &= ~(1u << e);
+            e4 &= ~(1u << e);
+          }
       }
-      m |= bits << (4 * u);
+      ms |= s4 << (4 * u);
+      me |= e4 << (4 * u);
     }
-    while (__any_sync(0xffffffffu, m != 0u)) {
-      const bool has = m != 0u;
-      const int j = has ? __ffs(m) - 1 : 0;
-      m &= has ? m - 1 : 0u;
-      const uint32_t pos = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
-      place_hit<D>(sm, spill, has, pos, has ? pick_score(v, j) : 0.f, b1, lt);
+    if (!__any_sync(0xffffffffu, (ms | me) != 0u)) continue;
+    const uint32_t ns = __popc(ms), ne = __popc(me);
+    uint32_t ps = ns, pe = ne;
+    warp_scan2(ps, pe);
+    uint32_t bs = 0, be = 0;
+    if (lane == 31) {
+      if (ps) bs = atomicAdd(&sm.n_sure, ps);
+      if (pe) be = atomicAdd(&sm.n_list, pe);
+    }
+    uint32_t os = __shfl_sync(0xffffffffu, bs, 31) + ps - ns;
+    uint32_t oe = __shfl_sync(0xffffffffu, be, 31) + pe - ne;
+    // the lane's hits, vector by vector: every score is read from a register by a
+    // compile-time index (a run-time pick among the 32 would cost a chain of selects per hit)
+#pragma unroll
+    for (int u = 0; u < kStreamVec; ++u) {
+      const uint32_t s4 = (ms >> (4 * u)) & 15u, e4 = (me >> (4 * u)) & 15u;
+      if ((s4 | e4) == 0u) continue;
+      const float zz[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      const uint32_t p0 = static_cast<uint32_t>(b0 + 4LL * kSaThreads * u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (s4 & (1u << e)) {
+          if (os < static_cast<uint32_t>(kSureCap)) sm.sure[os] = p0 + e;
+          ++os;
+        }
+        if (e4 & (1u << e)) {
+          const uint32_t key = order_key(zz[e]);
+          const unsigned long long x = composite(key, p0 + e);
+          if (oe < static_cast<uint32_t>(kListSmem)) sm.list[oe] = x;
+          else spill[oe] = x;
+          atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+          ++oe;
+        }
+      }
     }
   }
 }
