@@ -150,11 +150,11 @@ struct TileWalk {
   }
 };
 
-// At most 112 registers a thread (the bound of two CTAs an SM): registers are allocated per SM
-// sub-partition (16K each), which gets three of this kernel's nine warps, and a selection CTA
-// (eight warps of at most 80 registers, two a sub-partition) must still fit beside them.
+// At most 104 registers a thread: registers are allocated per SM sub-partition (16K each),
+// which gets three of this kernel's nine warps, and a selection CTA (eight warps of at most 96
+// registers, two a sub-partition) must still fit beside them: 3 * 104 + 2 * 96 <= 512 (x 32).
 template <int D, int ROWS, class Pg>
-__global__ void __launch_bounds__(ScoreCfg<D, ROWS>::kThreads, 2)
+__global__ void __maxnreg__(104)
     score_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const ScoreParams p, const Pg pg,
                      const int stages, const int chunk) {
   using C = ScoreCfg<D, ROWS>;

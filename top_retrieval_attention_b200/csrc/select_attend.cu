@@ -377,6 +377,18 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
   if (tid == 0 && rank == 0) atomicOr(p.err, kErrSelect);   // unreachable for distinct keys
 }
 
+// The score at bit j of a thread's hit masks: element j % 4 of its (j / 4)-th loaded vector,
+// chosen from registers by a three-level select on the vector index (no dynamic indexing).
+__device__ __forceinline__ float pick_score(const float4 (&v)[kStreamVec], int j) {
+  static_assert(kStreamVec == 8, "three select levels");
+  const int u = j >> 2, e = j & 3;
+  const float4 a0 = (u & 1) ? v[1] : v[0], a1 = (u & 1) ? v[3] : v[2];
+  const float4 a2 = (u & 1) ? v[5] : v[4], a3 = (u & 1) ? v[7] : v[6];
+  const float4 b0 = (u & 2) ? a1 : a0, b1 = (u & 2) ? a3 : a2;
+  const float4 c = (u & 4) ? b1 : b0;
+  return e == 0 ? c.x : e == 1 ? c.y : e == 2 ? c.z : c.w;
+}
+
 // Inclusive warp prefix sums of two per-lane counts; the warp totals come back in lane 31.
 __device__ __forceinline__ void warp_scan2(uint32_t &a, uint32_t &b) {
   const int lane = threadIdx.x & 31;
@@ -397,8 +409,9 @@ __device__ __forceinline__ void warp_scan2(uint32_t &a, uint32_t &b) {
 // entries), with their digit-2 histogram in sm.h; the counters keep counting past the
 // capacities.  Hits are a few percent of the keys: each thread makes two bit masks with two
 // compares per score, the warp reserves its slots with one shared atomic per list and
-// iteration (offsets from a warp prefix scan of the per-lane counts), and every lane then
-// writes its own hits straight from its registers.
+// iteration (offsets from a warp prefix scan of the per-lane counts), and every lane then walks
+// its own set bits (the warp loops as often as its busiest lane has hits), the score of a key
+// in b1 picked from its registers.
 template <int D>
 __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
                                              unsigned long long *spill, long long a0, long long lo,
@@ -452,29 +465,23 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
     }
     uint32_t os = __shfl_sync(0xffffffffu, bs, 31) + ps - ns;
     uint32_t oe = __shfl_sync(0xffffffffu, be, 31) + pe - ne;
-    // the lane's hits, vector by vector: every score is read from a register by a
-    // compile-time index (a run-time pick among the 32 would cost a chain of selects per hit)
-#pragma unroll
-    for (int u = 0; u < kStreamVec; ++u) {
-      const uint32_t s4 = (ms >> (4 * u)) & 15u, e4 = (me >> (4 * u)) & 15u;
-      if ((s4 | e4) == 0u) continue;
-      const float zz[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      const uint32_t p0 = static_cast<uint32_t>(b0 + 4LL * kSaThreads * u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (s4 & (1u << e)) {
-          if (os < static_cast<uint32_t>(kSureCap)) sm.sure[os] = p0 + e;
-          ++os;
-        }
-        if (e4 & (1u << e)) {
-          const uint32_t key = order_key(zz[e]);
-          const unsigned long long x = composite(key, p0 + e);
-          if (oe < static_cast<uint32_t>(kListSmem)) sm.list[oe] = x;
-          else spill[oe] = x;
-          atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
-          ++oe;
-        }
-      }
+    while (ms) {   // keys above b1: positions only
+      const int j = __ffs(ms) - 1;
+      ms &= ms - 1;
+      if (os < static_cast<uint32_t>(kSureCap))
+        sm.sure[os] = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
+      ++os;
+    }
+    while (me) {   // keys in b1: composites and the digit-2 histogram
+      const int j = __ffs(me) - 1;
+      me &= me - 1;
+      const uint32_t pos = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
+      const uint32_t key = order_key(pick_score(v, j));
+      const unsigned long long x = composite(key, pos);
+      if (oe < static_cast<uint32_t>(kListSmem)) sm.list[oe] = x;
+      else spill[oe] = x;
+      atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+      ++oe;
     }
   }
 }
@@ -708,57 +715,59 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
 }
 
 constexpr int kStage = kSureCap / 2;   // entries staged at a time (the sure array is free here)
-constexpr int kAttnRows = 16;          // V rows a warp gathers at a time
 
-// One warp's online-softmax update over up to 16 entries: lane j < 16 holds entry j's V row
-// index vi (-1: no entry) and score z.  The 16 V rows are gathered together (each lane a D / 32
-// channel slice of every row), then folded into the warp's state (m, zs, acc).
+// The attention gathers V rows with 16-byte loads: a row of D bf16 is D / 8 lanes, so one load
+// instruction of the warp fetches 256 / D rows (2 at d = 128, 4 at d = 64), and a warp takes
+// kLoads instructions' worth of rows at a time (16 at d = 128, 32 at d = 64).  Lane l keeps the
+// channels [8 (l mod D/8), + 8) of the rows of its lane group.
 template <int D>
-__device__ __forceinline__ void attend16(const __nv_bfloat16 *Vb, int vi, float z, float &m,
-                                         float &zs, float (&acc)[D / 32]) {
-  constexpr int CPL = D / 32;   // channels per lane
+struct AttnCfg {
+  static constexpr int kLanesPerRow = D / 8;
+  static constexpr int kRowsPerLoad = 32 / kLanesPerRow;
+  static constexpr int kLoads = 8;
+  static constexpr int kRows = kLoads * kRowsPerLoad;
+  static_assert(kRows <= 32, "one entry per lane");
+};
+
+// One warp's online-softmax update over up to AttnCfg<D>::kRows entries: lane j < kRows holds
+// entry j's V row index vi (-1: no entry) and score z.  All the rows' loads are issued together,
+// then folded into the warp's state (m, zs) and the lane's eight channel numerators acc.
+template <int D>
+__device__ __forceinline__ void attend_rows(const __nv_bfloat16 *Vb, int vi, float z, float &m,
+                                            float &zs, float (&acc)[8]) {
+  using A = AttnCfg<D>;
   const int lane = threadIdx.x & 31;
+  const int grp = lane / A::kLanesPerRow;
+  const int c0 = (lane % A::kLanesPerRow) * 8;
   if (vi < 0) z = -INFINITY;
-  uint32_t wv[kAttnRows][CPL / 2];
+  uint4 wv[A::kLoads];
 #pragma unroll
-  for (int j = 0; j < kAttnRows; ++j) {
-    const int pj = __shfl_sync(0xffffffffu, vi, j);
-    if (pj >= 0) {
-      const __nv_bfloat16 *vr = Vb + static_cast<long long>(pj) * D;
-      if constexpr (CPL == 4) {
-        const uint2 v = __ldcg(reinterpret_cast<const uint2 *>(vr) + lane);
-        wv[j][0] = v.x;
-        wv[j][1] = v.y;
-      } else {
-        wv[j][0] = __ldcg(reinterpret_cast<const uint32_t *>(vr) + lane);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < CPL / 2; ++c) wv[j][c] = 0u;
-    }
+  for (int i = 0; i < A::kLoads; ++i) {
+    const int pj = __shfl_sync(0xffffffffu, vi, i * A::kRowsPerLoad + grp);
+    wv[i] = pj >= 0 ? __ldcg(reinterpret_cast<const uint4 *>(Vb + static_cast<long long>(pj) * D + c0))
+                    : make_uint4(0u, 0u, 0u, 0u);
   }
-  float mg = lane < kAttnRows ? z : -INFINITY;   // the xor partners stay within groups of 16
+  float mg = lane < A::kRows ? z : -INFINITY;
 #pragma unroll
-  for (int o = kAttnRows / 2; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
-  mg = __shfl_sync(0xffffffffu, mg, 0);
+  for (int o = 16; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
   if (mg == -INFINITY) return;   // warp-uniform: no entry in this group
   const float mn = fmaxf(m, mg);
   const float sc = expf(m - mn);   // 0 while m is -inf
-  const float pe = (lane >= kAttnRows || z == -INFINITY) ? 0.f : expf(z - mn);
+  const float pe = (lane >= A::kRows || z == -INFINITY) ? 0.f : expf(z - mn);
   float ps = pe;
 #pragma unroll
-  for (int o = kAttnRows / 2; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-  ps = __shfl_sync(0xffffffffu, ps, 0);
+  for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
   zs = zs * sc + ps;
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] *= sc;
+  for (int c = 0; c < 8; ++c) acc[c] *= sc;
 #pragma unroll
-  for (int j = 0; j < kAttnRows; ++j) {
-    const float pj = __shfl_sync(0xffffffffu, pe, j);
+  for (int i = 0; i < A::kLoads; ++i) {
+    const float pj = __shfl_sync(0xffffffffu, pe, i * A::kRowsPerLoad + grp);
+    const uint32_t w[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
 #pragma unroll
-    for (int c = 0; c < CPL / 2; ++c) {
-      acc[2 * c] += pj * bf16_lo(wv[j][c]);
-      acc[2 * c + 1] += pj * bf16_hi(wv[j][c]);
+    for (int c = 0; c < 4; ++c) {
+      acc[2 * c] += pj * bf16_lo(w[c]);
+      acc[2 * c + 1] += pj * bf16_hi(w[c]);
     }
   }
   m = mn;
@@ -770,16 +779,21 @@ __device__ __forceinline__ void attend16(const __nv_bfloat16 *Vb, int vi, float 
 // (grid z), into this cluster's state for the head's last cluster to merge (Eqs. (3)-(5)).
 template <int D>
 __device__ void combine_and_merge(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &cl,
-                                  int rank, int ncl, int row, float m, float zs,
-                                  const float (&acc)[D / 32]) {
-  constexpr int CPL = D / 32;
+                                  int rank, int ncl, int row, float m, float zs, float (&acc)[8]) {
+  using A = AttnCfg<D>;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (lane == 0) {
     sm.wm[warp] = m;
     sm.wz[warp] = zs;
   }
+  // the lane groups' numerators of the same channels add up
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) sm.wacc[warp * D + lane * CPL + c] = acc[c];
+  for (int o = A::kLanesPerRow; o < 32; o <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+  if (lane < A::kLanesPerRow)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) sm.wacc[warp * D + lane * 8 + c] = acc[c];
   __syncthreads();
   float M = sm.wm[0];
 #pragma unroll
@@ -846,12 +860,11 @@ __device__ void combine_and_merge(const SaParams &p, SaSmem<D> &sm, cg::cluster_
 
 // Softmax attention of one query head over U = W u Omega (Omega read from idx), split across
 // the nsplit clusters of the head (grid z) and the CTAs of each.  Each CTA stages its entries'
-// positions and scores in shared memory (in blocks of kStage), then its warps gather 16 V rows
-// at a time and keep online-softmax states.
+// positions and scores in shared memory (in blocks of kStage), then its warps gather V rows
+// (attend_rows) and keep online-softmax states.
 template <int D, bool kFull, class Pg>
 __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, SaSmem<D> &sm,
                              cg::cluster_group &cl, int rank, int ncl, int row) {
-  constexpr int CPL = D / 32;   // channels per lane
   constexpr int kPer = kStage / kSaThreads;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long nU = gm.nW + gm.k_eff;
@@ -865,9 +878,10 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
   int *spos = reinterpret_cast<int *>(sm.sure);   // staged: the entry's V row (-1: none)
   float *sz = reinterpret_cast<float *>(sm.sure + kStage);
-  float m = -INFINITY, zs = 0.f, acc[CPL];
+  constexpr int kRows = AttnCfg<D>::kRows;
+  float m = -INFINITY, zs = 0.f, acc[8];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
   for (long long blk = e_lo; blk < e_hi; blk += kStage) {
     const int nb = static_cast<int>(min(static_cast<long long>(kStage), e_hi - blk));
     // positions (W computed, Omega from idx), then their scores: two rounds of loads in flight
@@ -890,9 +904,9 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
       }
     }
     __syncthreads();
-    for (int g = warp * kAttnRows; g < nb; g += kAttnRows * kSaWarps) {
-      const bool mine = lane < kAttnRows && g + lane < nb;
-      attend16<D>(Vb, mine ? spos[g + lane] : -1, mine ? sz[g + lane] : -INFINITY, m, zs, acc);
+    for (int g = warp * kRows; g < nb; g += kRows * kSaWarps) {
+      const bool mine = lane < kRows && g + lane < nb;
+      attend_rows<D>(Vb, mine ? spos[g + lane] : -1, mine ? sz[g + lane] : -INFINITY, m, zs, acc);
     }
     __syncthreads();   // the staging area is reused by the next block
   }
@@ -940,8 +954,10 @@ __device__ bool wait_ready(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &
 // kFull = false: the plain decode step (the score kernel's histogram, the cache's own score rows
 // and positions); the threshold budget, the self-built histogram and candidate lists take the
 // kFull = true instantiation, so the plain one carries none of their code.
+// At most 96 registers a thread, so that a CTA fits on an SM sub-partition beside a score CTA
+// (the score kernel's bound states the sum).
 template <int D, class Pg, bool kFull>
-__global__ void __launch_bounds__(kSaThreads, 3) select_attend_kernel(const SaParams p, const Pg pg) {
+__global__ void __maxnreg__(96) select_attend_kernel(const SaParams p, const Pg pg) {
   __shared__ SaSmem<D> sm;
   cg::cluster_group cl = cg::this_cluster();
   const int ncl = static_cast<int>(cl.num_blocks());
