@@ -101,6 +101,8 @@ struct SaParams {
   const int32_t *pos_map;   // with row_n: [B*Hq, ldS] cache position of each candidate (-1: a
                             // static-set key); idx reports these positions
   const float *S_att;       // with row_n: [B*Hq, ldS] full-length score rows for the attention
+  float *sel_z;             // if set: [B*Hq, k] the score of each selected entry, beside idx (the
+                            // selection writes it; the attention reads it instead of the rows)
   // Overlap with the score kernel (null: none; the kernel waits for its predecessor instead):
   // the cluster of row r starts once ready[(r / G) * ready_stride] reaches ready_target (every
   // score CTA is done with that KV head), and the row group's last cluster sets it back to 0.

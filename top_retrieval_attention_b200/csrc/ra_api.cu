@@ -67,7 +67,7 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 struct Step {
   int B, Hq, Hkv, G, d, k, n_sink, n_window, R, ncl;
   long long N, cap, s1, w0, nW, nC, k_eff, ldS, ldL, cbase, cper;
-  size_t off_S, off_hist, off_meta, off_list, off_part, total;
+  size_t off_S, off_hist, off_meta, off_list, off_selz, off_part, total;
 };
 
 static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, int n_sink,
@@ -94,9 +94,14 @@ static ra_status plan_shape(int B, int Hq, int Hkv, long long N, int d, int k, i
   st.off_hist = off;  off = align_up(off + static_cast<size_t>(st.R) * kHistBins * 4);
   st.off_meta = off;  off = align_up(off + static_cast<size_t>(st.R) * kMetaWords * 4);
   st.off_S = off;     off = align_up(off + static_cast<size_t>(st.R) * st.ldS * 4);
-  // the threshold-bin lists are needed only when the selection is a proper subset of C
+  // the threshold-bin lists (and the scores of the keys above the bin), whenever a selection
+  // may stream over C: with a budget under |C|, and under a threshold budget, which can keep
+  // fewer keys than a budget of |C| or more
   st.off_list = off;
-  if (st.k_eff > 0 && st.k_eff < st.nC) off = align_up(off + static_cast<size_t>(st.R) * st.ldL * 8);
+  if (st.k_eff > 0) off = align_up(off + static_cast<size_t>(st.R) * st.ldL * 8);
+  // the score of each selected entry, beside idx
+  st.off_selz = off;
+  if (st.k > 0) off = align_up(off + static_cast<size_t>(st.R) * st.k * 4);
   st.off_part = off;  off = align_up(off + static_cast<size_t>(st.R) * kMaxAttnSplit * (d + 4) * 4);
   st.total = off;
   return RA_OK;
@@ -201,6 +206,9 @@ static ra_status run_select_attend(const ra_kv *kv, const Step &st, int mode, in
   p.cbase = st.cbase; p.cper = st.cper;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
   p.log_eps = log_eps;
+  // a selection in this call keeps the selected scores beside idx for the attention; an
+  // attention over a caller's idx (ra_sparse_attn) reads the score rows
+  if ((mode & kSaSelect) && st.k > 0) p.sel_z = reinterpret_cast<float *>(at(ws, st.off_selz));
   const int split = (mode & kSaAttend) ? attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d) : 1;
   if (mode & kSaSelect) {
     // the attention joins the launch when it can
@@ -748,6 +756,7 @@ ra_status ra_paged_decode_step(const ra_paged_kv *kv, const void *q, int32_t Hq,
   p.err = reinterpret_cast<uint32_t *>(at(ws, st.off_meta)) + kError;
   p.ldS = st.ldS; p.ldL = st.ldL; p.cap = 0; p.N = st.N;
   p.k = st.k; p.Hq = st.Hq; p.G = st.G; p.Hkv = st.Hkv;
+  if (k > 0) p.sel_z = reinterpret_cast<float *>(at(ws, st.off_selz));
   const int split = attn_split(st.nW + st.k_eff, st.R, st.ncl, st.d);
   p.mode = split == 1 ? (kSaSelect | kSaAttend) : kSaSelect;
   p.nsplit = 1;
@@ -948,6 +957,7 @@ ra_status ra_ivf_decode_step(const ra_kv *kv, const ra_ivf *ix, const void *q, i
   p.s1 = dec.s1; p.w0 = dec.w0; p.nW = dec.nW; p.nC = dec.nC; p.k_eff = dec.k_eff;
   p.cbase = dec.cbase; p.cper = dec.cper;
   p.k = k; p.Hq = Hq; p.G = dec.G; p.Hkv = dec.Hkv;
+  if (k > 0) p.sel_z = reinterpret_cast<float *>(at(ws, L.st.off_selz));
   const int split = attn_split(nU, dec.R, ncl, dec.d);
   if (k > 0) {
     p.mode = kSaSelect | kSaBuildHist | (split == 1 ? kSaAttend : 0);

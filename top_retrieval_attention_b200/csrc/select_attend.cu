@@ -93,6 +93,18 @@ __device__ __forceinline__ unsigned long long composite(uint32_t key, uint32_t p
 __device__ __forceinline__ uint32_t composite_pos(unsigned long long x) {
   return 0xFFFFFFFFu - static_cast<uint32_t>(x);
 }
+__device__ __forceinline__ float composite_z(unsigned long long x) {
+  return key_float(static_cast<uint32_t>(x >> 32));
+}
+
+// Selected entry o of row blockIdx.y: its index into idx and, when the launch keeps them, its
+// score into sel_z.
+template <bool kFull>
+__device__ __forceinline__ void put_sel(const SaParams &p, int32_t *irow, uint32_t o, uint32_t e,
+                                        float z) {
+  irow[o] = idx_of<kFull>(p, e);
+  if (p.sel_z) p.sel_z[static_cast<long long>(blockIdx.y) * p.k + o] = z;
+}
 
 // Block-wide inclusive prefix sums of two counters at once; warp_tot holds 2 * kSaWarps words.
 // Returns the inclusive sums; the block totals are left in tot_a / tot_b.
@@ -237,7 +249,7 @@ __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm,
       uint32_t above = 0;
       for (int j = 0; j < 32; ++j) above += __shfl_sync(0xffffffffu, x, j) > x ? 1u : 0u;
       if (static_cast<uint32_t>(lane) < n && above < want)
-        irow[o0 + above] = idx_of<kFull>(p, composite_pos(x));
+        put_sel<kFull>(p, irow, o0 + above, composite_pos(x), composite_z(x));
     }
     return;
   }
@@ -245,7 +257,8 @@ __device__ __forceinline__ void bitonic_finish(const SaParams &p, SaSmem<D> &sm,
   __syncthreads();
   if (tid < 32) {
     bitonic_desc64(sm.fin);
-    for (uint32_t i = lane; i < want; i += 32) irow[o0 + i] = idx_of<kFull>(p, composite_pos(sm.fin[i]));
+    for (uint32_t i = lane; i < want; i += 32)
+      put_sel<kFull>(p, irow, o0 + i, composite_pos(sm.fin[i]), composite_z(sm.fin[i]));
   }
 }
 
@@ -347,11 +360,12 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
       if ((x >> sh) != prefix) return;
       const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
       if (dg > t) {
-        if (ou < k_eff) irow[ou] = idx_of<kFull>(p, composite_pos(x));
+        if (ou < k_eff) put_sel<kFull>(p, irow, ou, composite_pos(x), composite_z(x));
         ++ou;
       } else if (dg == t) {
         if (take_eq) {
-          if (base + up + oe < k_eff) irow[base + up + oe] = idx_of<kFull>(p, composite_pos(x));
+          if (base + up + oe < k_eff)
+            put_sel<kFull>(p, irow, base + up + oe, composite_pos(x), composite_z(x));
         } else if (fin && oe < static_cast<uint32_t>(kFinish)) {
           fin0[oe] = x;
         }
@@ -404,10 +418,11 @@ __device__ __forceinline__ void warp_scan2(uint32_t &a, uint32_t &b) {
 }
 
 // One pass over the CTA's candidates [lo, hi) of the score row.  Keys above the digit-1
-// threshold bin b1 (z >= zhi, the bottom of bin b1 + 1) go to sm.sure as positions; keys in b1
+// threshold bin b1 (z >= zhi, the bottom of bin b1 + 1) go to sm.sure as positions, their
+// scores to the top of `spill` (entry i at spill[hi - lo - 1 - i]); keys in b1
 // (zlo <= z < zhi) go to sm.list as composites, past its capacity to `spill` (room for hi - lo
-// entries), with their digit-2 histogram in sm.h; the counters keep counting past the
-// capacities.  Hits are a few percent of the keys: each thread makes two bit masks with two
+// entries: the two never meet, a candidate being one or the other), with their digit-2
+// histogram in sm.h; the counters keep counting past the capacities.  Hits are a few percent of the keys: each thread makes two bit masks with two
 // compares per score, the warp reserves its slots with one shared atomic per list and
 // iteration (offsets from a warp prefix scan of the per-lane counts), and every lane then walks
 // its own set bits (the warp loops as often as its busiest lane has hits), the score of a key
@@ -465,11 +480,13 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
     }
     uint32_t os = __shfl_sync(0xffffffffu, bs, 31) + ps - ns;
     uint32_t oe = __shfl_sync(0xffffffffu, be, 31) + pe - ne;
-    while (ms) {   // keys above b1: positions only
+    while (ms) {   // keys above b1: positions, their scores at the slice's top
       const int j = __ffs(ms) - 1;
       ms &= ms - 1;
-      if (os < static_cast<uint32_t>(kSureCap))
+      if (os < static_cast<uint32_t>(kSureCap)) {
         sm.sure[os] = static_cast<uint32_t>(b0 + 4LL * kSaThreads * (j >> 2) + (j & 3));
+        spill[hi - lo - 1 - os] = __float_as_uint(pick_score(v, j));
+      }
       ++os;
     }
     while (me) {   // keys in b1: composites and the digit-2 histogram
@@ -653,7 +670,8 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   }
   if (k_sel >= gm.nC) {   // every candidate is selected
     for (long long i = lo + tid; i < hi; i += kSaThreads)
-      irow[i - gm.s1] = idx_of<kFull>(p, static_cast<uint32_t>(i));
+      put_sel<kFull>(p, irow, static_cast<uint32_t>(i - gm.s1), static_cast<uint32_t>(i),
+                     p.sel_z ? __ldcg(srow + i) : 0.f);
     return;
   }
   const uint32_t k_eff = static_cast<uint32_t>(k_sel);
@@ -694,8 +712,11 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
   for (int c = 0; c < rank; ++c) off += sm.x_a[c];
   // the keys above b1 take idx slots [0, above1), CTA by CTA
   if (sm.n_sure <= static_cast<uint32_t>(kSureCap)) {
+    // their scores sit at the top of the CTA's spill slice (stream_chunk)
+    const unsigned long long *ztop = spill + (hi - lo - 1);
     for (uint32_t i = tid; i < sm.n_sure; i += kSaThreads)
-      if (off + i < k_eff) irow[off + i] = idx_of<kFull>(p, sm.sure[i]);
+      if (off + i < k_eff)
+        put_sel<kFull>(p, irow, off + i, sm.sure[i], __uint_as_float(static_cast<uint32_t>(__ldcg(ztop - i))));
   } else {   // more sure keys than sm.sure holds: from the chunk again
     uint32_t cu = 0;
     chunk.for_each([&](unsigned long long x) { cu += (x >> (64 - kHistBits)) > b1 ? 1u : 0u; });
@@ -704,7 +725,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     uint32_t o = off + inc.x - cu;
     chunk.for_each([&](unsigned long long x) {
       if ((x >> (64 - kHistBits)) > b1) {
-        if (o < k_eff) irow[o] = idx_of<kFull>(p, composite_pos(x));
+        if (o < k_eff) put_sel<kFull>(p, irow, o, composite_pos(x), composite_z(x));
         ++o;
       }
     });
@@ -876,6 +897,7 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   const __nv_bfloat16 *Vb = v_base<D>(p, pg, b, h / p.G);
   const float *srow = ((kFull && p.S_att) ? p.S_att : p.S) + static_cast<long long>(row) * p.ldS;
   const int32_t *irow = p.idx + static_cast<long long>(row) * p.k;
+  const float *zrow = p.sel_z ? p.sel_z + static_cast<long long>(row) * p.k : nullptr;
   int *spos = reinterpret_cast<int *>(sm.sure);   // staged: the entry's V row (-1: none)
   float *sz = reinterpret_cast<float *>(sm.sure + kStage);
   constexpr int kRows = AttnCfg<D>::kRows;
@@ -885,19 +907,30 @@ __device__ void attend_phase(const SaParams &p, const RowGeo &gm, const Pg &pg, 
   for (long long blk = e_lo; blk < e_hi; blk += kStage) {
     const int nb = static_cast<int>(min(static_cast<long long>(kStage), e_hi - blk));
     // positions (W computed, Omega from idx), then their scores: two rounds of loads in flight
+    // positions (W computed, Omega from idx) and, for Omega, the scores the selection kept
+    // beside idx, loaded together; the other scores from the score row
     int pp[kPer];
+    float zk[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int i = tid + j * kSaThreads;
       const long long e = blk + i;
       long long pos = -1;
-      if (i < nb) pos = e < gm.nW ? (e < gm.s1 ? e : gm.w0 + (e - gm.s1)) : __ldcg(irow + (e - gm.nW));
+      zk[j] = NAN;
+      if (i < nb) {
+        if (e < gm.nW) {
+          pos = e < gm.s1 ? e : gm.w0 + (e - gm.s1);
+        } else {
+          pos = __ldcg(irow + (e - gm.nW));
+          if (zrow) zk[j] = __ldcg(zrow + (e - gm.nW));
+        }
+      }
       pp[j] = (pos >= 0 && pos < gm.N) ? static_cast<int>(pos) : -1;   // always, for a complete idx
     }
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int i = tid + j * kSaThreads;
-      const float z = pp[j] >= 0 ? __ldcg(srow + pp[j]) : -INFINITY;
+      const float z = pp[j] < 0 ? -INFINITY : (zk[j] == zk[j] ? zk[j] : __ldcg(srow + pp[j]));
       if (i < nb) {
         spos[i] = pp[j] >= 0 ? v_index(p, pg, b, h / p.G, pp[j]) : -1;
         sz[i] = z;
