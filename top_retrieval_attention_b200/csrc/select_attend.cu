@@ -987,10 +987,8 @@ __device__ bool wait_ready(const SaParams &p, SaSmem<D> &sm, cg::cluster_group &
 // kFull = false: the plain decode step (the score kernel's histogram, the cache's own score rows
 // and positions); the threshold budget, the self-built histogram and candidate lists take the
 // kFull = true instantiation, so the plain one carries none of their code.
-// At most 96 registers a thread, so that a CTA fits on an SM sub-partition beside a score CTA
-// (the score kernel's bound states the sum).
 template <int D, class Pg, bool kFull>
-__global__ void __maxnreg__(96) select_attend_kernel(const SaParams p, const Pg pg) {
+__device__ __forceinline__ void select_attend_body(const SaParams &p, const Pg &pg) {
   __shared__ SaSmem<D> sm;
   cg::cluster_group cl = cg::this_cluster();
   const int ncl = static_cast<int>(cl.num_blocks());
@@ -1013,6 +1011,31 @@ __global__ void __maxnreg__(96) select_attend_kernel(const SaParams p, const Pg 
     cl.sync();   // no CTA leaves while the cluster may still use its shared memory
   }
 }
+
+// Two register bounds over the same body.  A launch whose clusters all run at once (one wave)
+// is latency-bound: it takes 96 registers a thread and spills nothing, and a CTA of it still
+// fits on an SM sub-partition beside a score CTA (the score kernel's bound states the sum).
+// A launch of more clusters than that is throughput-bound: it keeps three CTAs an SM (at most
+// 80 registers a thread, a few spilled words).
+template <int D, class Pg, bool kFull>
+__global__ void __maxnreg__(96) select_attend_kernel(const SaParams p, const Pg pg) {
+  select_attend_body<D, Pg, kFull>(p, pg);
+}
+
+template <int D, class Pg, bool kFull>
+__global__ void __launch_bounds__(kSaThreads, 3) select_attend_wide_kernel(const SaParams p,
+                                                                           const Pg pg) {
+  select_attend_body<D, Pg, kFull>(p, pg);
+}
+
+template <int D, class Pg, bool kFull, bool kWide>
+struct SaKernel {
+  static constexpr auto fn = select_attend_kernel<D, Pg, kFull>;
+};
+template <int D, class Pg, bool kFull>
+struct SaKernel<D, Pg, kFull, true> {
+  static constexpr auto fn = select_attend_wide_kernel<D, Pg, kFull>;
+};
 
 // ------------------------------------------------------------------ host
 
@@ -1065,20 +1088,20 @@ int select_cluster_size(long long nC, int R, int d) {
   return n;
 }
 
-template <int D, class Pg, bool kFull>
+template <int D, class Pg, bool kFull, bool kWide>
 static cudaError_t launch_sa_k(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
   static bool attr_done[64] = {};
   static bool carve_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
     if (ncl > 8 && !attr_done[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
+      const cudaError_t e = cudaFuncSetAttribute(SaKernel<D, Pg, kFull, kWide>::fn,
                                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
       attr_done[dev] = true;
     }
     if (!carve_done[dev]) {   // the same carveout as the scan, so both fit on one SM
-      const cudaError_t e = cudaFuncSetAttribute(select_attend_kernel<D, Pg, kFull>,
+      const cudaError_t e = cudaFuncSetAttribute(SaKernel<D, Pg, kFull, kWide>::fn,
                                                  cudaFuncAttributePreferredSharedMemoryCarveout,
                                                  cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return e;
@@ -1100,14 +1123,21 @@ static cudaError_t launch_sa_k(const SaParams &p, const Pg &pg, int R, int ncl, 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, select_attend_kernel<D, Pg, kFull>, p, pg);
+  return cudaLaunchKernelEx(&cfg, SaKernel<D, Pg, kFull, kWide>::fn, p, pg);
 }
 
 template <int D, class Pg>
 static cudaError_t launch_sa_t(const SaParams &p, const Pg &pg, int R, int ncl, cudaStream_t s) {
   const bool full = (p.mode & (kSaEps | kSaBuildHist)) != 0 || p.row_n != nullptr ||
                     p.pos_map != nullptr || p.S_att != nullptr;
-  return full ? launch_sa_k<D, Pg, true>(p, pg, R, ncl, s) : launch_sa_k<D, Pg, false>(p, pg, R, ncl, s);
+  // more clusters than the 96-register kernel runs at once: the three-CTA bound
+  const long long clusters = static_cast<long long>(R) * (p.nsplit < 1 ? 1 : p.nsplit);
+  const bool wide = clusters > active_clusters_t<D>(ncl);
+  if (full)
+    return wide ? launch_sa_k<D, Pg, true, true>(p, pg, R, ncl, s)
+                : launch_sa_k<D, Pg, true, false>(p, pg, R, ncl, s);
+  return wide ? launch_sa_k<D, Pg, false, true>(p, pg, R, ncl, s)
+              : launch_sa_k<D, Pg, false, false>(p, pg, R, ncl, s);
 }
 
 size_t select_smem_bytes(int d) { return d == 128 ? sizeof(SaSmem<128>) : sizeof(SaSmem<64>); }
