@@ -43,6 +43,49 @@ __device__ __forceinline__ float key_float(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
+// ------------------------------------------------------------------ digit 1 of the top-k select
+//
+// The first digit of the selection's radix select is a bin of the score that is fine where top-k
+// thresholds lie.  Let a = bits [17, 31) of |z| (its exponent and top 6 mantissa bits) and
+// m = clamp(a - kD1A0, 0, 1023): m = 1 .. 1022 cover |z| in [2^-8, 2^8) at 64 steps an octave,
+// m = 0 holds |z| < 2^-8 and m = 1023 holds |z| >= 2^8 (less the top two steps).  The bin is
+// 1024 + m for z >= +0 and 1023 - m for z < 0, so bins rise with z; a bin with 1 <= m <= 1022
+// is one value of the order key's top 15 bits (sign and a), the four others (0, 1023, 1024,
+// 2047) share no key prefix.  (A plain top-11-bit digit has 4 bins an octave: at 1 % of 128K
+// keys its threshold bin holds thousands of a head's keys.)
+constexpr uint32_t kD1A0 = (127u - 8u) * 64u - 1u;   // a of 2^-8, less one
+constexpr uint32_t kD1PrefixBits = 15;
+
+// From the score itself (canonical zero): two float clamps, a shift, a subtraction, a sign flip.
+__device__ __forceinline__ uint32_t digit1_bin_z(float z) {
+  const float c = fminf(fmaxf(fabsf(z), __uint_as_float(kD1A0 << 17)),
+                        __uint_as_float((kD1A0 + 1023u) << 17));
+  const int m = static_cast<int>(__float_as_uint(c) >> 17) - static_cast<int>(kD1A0);
+  const int s = static_cast<int>(__float_as_uint(z)) >> 31;   // 0, or -1 for z < 0
+  return static_cast<uint32_t>(1024 + (m ^ s));
+}
+// The same bin from an order key (the inverse of order_key, then the rule above).
+__host__ __device__ __forceinline__ uint32_t digit1_bin(uint32_t key) {
+  const uint32_t u = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;   // the float's bits
+  const uint32_t a = (u >> 17) & 0x3FFFu;
+  const uint32_t m = a <= kD1A0 ? 0u : (a - kD1A0 > 1023u ? 1023u : a - kD1A0);
+  return (u & 0x80000000u) ? 1023u - m : 1024u + m;
+}
+// The smallest key of bin b (b = 2048: 2^32, past every key).
+__host__ __device__ __forceinline__ unsigned long long digit1_floor(uint32_t b) {
+  if (b >= 2048u) return 1ull << 32;
+  if (b >= 1024u) {   // z >= +0: the smallest |z| of its m
+    const uint32_t m = b - 1024u;
+    return m == 0u ? 0x80000000ull : (0x80000000ull | (static_cast<unsigned long long>(kD1A0 + m) << 17));
+  }
+  const uint32_t m = 1023u - b;   // z < 0: the largest |z| of its m
+  return m == 1023u ? 0ull : static_cast<unsigned long long>(0x3FFFu - (kD1A0 + m)) << 17;
+}
+// Key bits every key of bin b shares from the top: 15, or 0 for the four catch-all bins.
+__host__ __device__ __forceinline__ int digit1_prefix_bits(uint32_t b) {
+  return (b == 0u || b == 1023u || b == 1024u || b >= 2047u) ? 0 : static_cast<int>(kD1PrefixBits);
+}
+
 // ------------------------------------------------------------------ shared-memory addresses
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

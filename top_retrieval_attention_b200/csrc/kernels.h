@@ -77,7 +77,6 @@ constexpr int kSaBuildHist = 4;        // with kSaSelect: build the digit-1 hist
 constexpr int kSaEps = 8;              // with kSaSelect: keep only keys whose softmax weight > eps
 constexpr int kMaxCluster = 16;        // CTAs per query head at most
 constexpr int kMaxAttnSplit = 4;       // clusters per query head in the attention-only launch
-constexpr int kDigit2Shift = 10;       // digit 2 = bits [10, 21) of the order key
 constexpr uint32_t kErrSelect = 4u;    // error bit: the selection's counts were inconsistent
 
 struct SaParams {

@@ -17,9 +17,10 @@
 //     no CTA-wide barrier per tile; every wait is bounded;
 //   * the G query vectors are the n = 8 operand of bf16 m16n8k16 tensor-core products with
 //     fp32 accumulation, read from the stage's query copy when the KV head changes;
-//   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram (top
-//     11 bits of the order-preserving key) of the candidate positions in shared memory (16-bit
-//     counts, two bins a word), flushed to global when the CTA moves to another KV head;
+//   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram (the
+//     2048 bins of digit1_bin over the order-preserving key) of the candidate positions in
+//     shared memory (16-bit counts, two bins a word), flushed to global when the CTA moves to
+//     another KV head;
 //   * optionally the step's append is fused in: the CTA whose tile holds the new token writes
 //     its K and V rows to the cache and patches the key row into the staged tile.
 #include <type_traits>
@@ -289,8 +290,12 @@ __global__ void __maxnreg__(104)
   TileWalk<ROWS> w;
   w.start(p, pg, chunk);
   long long cur_bg = -1;
-  long long rowbase = 0;
   long long cur_lo = 0, cur_hi = 0, cur_n = 0;
+  // this lane's two query heads of the group (C fragment columns 2 t4 and 2 t4 + 1): their score
+  // rows and shared histograms, set at each head change
+  float *srow0 = nullptr, *srow1 = nullptr;
+  uint32_t *hrow0 = hist_s, *hrow1 = hist_s;
+  bool hv0 = false, hv1 = false;
   bool cur_hist = false;
   int since_flush = 0;
   uint32_t bq[D / 16][2];
@@ -323,7 +328,13 @@ __global__ void __maxnreg__(104)
         cur_n = w.n;
         const long long b = cur_bg / p.Hkv;
         const long long g = cur_bg - b * p.Hkv;
-        rowbase = b * p.Hq + g * p.G;
+        const long long rowbase = b * p.Hq + g * p.G;
+        hv0 = 2 * t4 < p.G;
+        hv1 = 2 * t4 + 1 < p.G;
+        srow0 = p.S + (rowbase + (hv0 ? 2 * t4 : 0)) * p.ldS;
+        srow1 = p.S + (rowbase + (hv1 ? 2 * t4 + 1 : 0)) * p.ldS;
+        hrow0 = hist_s + (hv0 ? 2 * t4 : 0) * C::kHistWords;
+        hrow1 = hist_s + (hv1 ? 2 * t4 + 1 : 0) * C::kHistWords;
         if (ok) {
           // B operand (col-major k x n): element (k = channel, n = query head g4), from the
           // stage's copy of the group's queries
@@ -361,6 +372,8 @@ __global__ void __maxnreg__(104)
       named_bar_sync(kCons);   // the patched row is in place for every consumer warp
     }
     if (ok) {
+      // the whole tile holds cached candidates: no per-key range checks
+      const bool tile_in = w.key >= cur_lo && w.key + C::kTile <= cur_hi && w.key + C::kTile <= cur_n;
 #pragma unroll
       for (int gi = 0; gi < C::kGroups; ++gi) {
         const int arow = arow0 + 16 * gi;
@@ -379,17 +392,33 @@ __global__ void __maxnreg__(104)
           mma_bf16_16816(acc0, a, bq[kk][0], bq[kk][1]);
           mma_bf16_16816(acc1, a2, bq[kk + 1][0], bq[kk + 1][1]);
         }
-        // C fragment: e = 0,1 -> key g4, heads 2t4, 2t4+1; e = 2,3 -> key g4 + 8
+        // C fragment: e = 0,1 -> key g4, heads 2t4, 2t4+1; e = 2,3 -> key g4 + 8.  The
+        // zero of a product is made +0 by the fused add of +0.
+        const long long k0 = w.key + warp * 16 * C::kGroups + 16 * gi + g4;
+        float *s0 = srow0 + k0, *s1 = srow1 + k0;
+        if (tile_in) {   // every key of the tile is cached and a candidate
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int h = 2 * t4 + (e & 1);
-          const long long key = w.key + warp * 16 * C::kGroups + 16 * gi + g4 + (e >> 1) * 8;
-          if (h < p.G && key < cur_n) {
-            const float z = canon_zero((acc0[e] + acc1[e]) * p.scale);
-            p.S[(rowbase + h) * p.ldS + key] = z;
+          for (int e = 0; e < 4; ++e) {
+            const bool hv = (e & 1) ? hv1 : hv0;
+            if (!hv) continue;
+            const float z = fmaf(acc0[e] + acc1[e], p.scale, 0.0f);
+            ((e & 1) ? s1 : s0)[(e >> 1) * 8] = z;
+            if (cur_hist) {
+              const uint32_t bin = digit1_bin_z(z);
+              atomicAdd(((e & 1) ? hrow1 : hrow0) + (bin >> 1), 1u << ((bin & 1u) << 4));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool hv = (e & 1) ? hv1 : hv0;
+            const long long key = k0 + (e >> 1) * 8;
+            if (!hv || key >= cur_n) continue;
+            const float z = fmaf(acc0[e] + acc1[e], p.scale, 0.0f);
+            ((e & 1) ? s1 : s0)[(e >> 1) * 8] = z;
             if (cur_hist && key >= cur_lo && key < cur_hi) {
-              const uint32_t bin = order_key(z) >> (32 - kHistBits);
-              atomicAdd(&hist_s[h * C::kHistWords + (bin >> 1)], 1u << ((bin & 1u) << 4));
+              const uint32_t bin = digit1_bin_z(z);
+              atomicAdd(((e & 1) ? hrow1 : hrow0) + (bin >> 1), 1u << ((bin & 1u) << 4));
             }
           }
         }

@@ -10,8 +10,9 @@
 //
 // Selection, a radix select over the 64-bit composite x = order_key(z) << 32 | ~position (all
 // keys distinct: larger z first, equal z to the lower position):
-//   * digit 1 (the top 11 bits of order_key) was histogrammed by the score kernel; every CTA
-//     finds the threshold bin b1 (the bin of the k-th largest key) from it;
+//   * digit 1 (digit1_bin of order_key: 64 bins per octave where thresholds lie, a 15-bit key
+//     prefix each) was histogrammed by the score kernel; every CTA finds the threshold bin b1
+//     (the bin of the k-th largest key) from it;
 //   * one streaming pass over the CTA's chunk of scores keeps the positions of the keys above
 //     b1 ("sure") in shared memory, keeps the composites of the keys in b1 (the "list") in
 //     shared memory, past its capacity in the CTA's slice of a per-head list in the workspace,
@@ -23,11 +24,13 @@
 //     sent to the first CTA for a bitonic finish, or become the next round's domain;
 //   * a CTA with more sure keys than its shared array holds (very large k) writes them out from
 //     its chunk of the score row, re-read.
-// Attention: the CTAs split U (W first, then Omega from idx) into ranges; a warp takes 16
-// entries at a time (scores from the score row, V rows gathered 8 bytes per lane), keeps an
-// online softmax state, the CTA combines its warps, every CTA pushes its partial state
-// (m_S, Z_S, N_S) into the first CTA's shared memory, and the first CTA merges them with
-// weights e^{m_S - m} into the output.
+// Attention: the CTAs split U (W first, then Omega from idx) into ranges and stage their range's
+// positions and scores in shared memory (W's scores from the score row, Omega's from the scores
+// the selection wrote beside idx); a warp takes 16 entries at a time at d = 128 (32 at d = 64),
+// gathers their V rows 16 bytes per lane with all loads in flight together, keeps an online
+// softmax state, the CTA combines its warps, every CTA pushes its partial state (m_S, Z_S,
+// N_S) into the first CTA's shared memory, and the first CTA merges them with weights
+// e^{m_S - m} into the output.
 //
 // The same kernel selects from per-row candidate lists (IVF: row_n candidates per row, their
 // cache positions in pos_map) and builds its own digit-1 histogram or applies Eq. (2)'s
@@ -305,8 +308,11 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
                               int ncl, const Src &src, uint32_t b1, uint32_t want, uint32_t base,
                               int32_t *irow, uint32_t k_eff) {
   const int tid = threadIdx.x;
-  unsigned long long prefix = b1;
-  int sh = 64 - kHistBits;   // composite bits below digit 1
+  // the composite bits the keys of b1 share (none for a catch-all bin) and the bits below them
+  const int pbits = digit1_prefix_bits(b1);
+  unsigned long long prefix = pbits ? digit1_floor(b1) >> (32 - pbits) : 0ull;
+  int sh = 64 - pbits;
+  const auto top = [&sh](unsigned long long x) { return sh >= 64 ? 0ull : x >> sh; };
   bool have_hist = true;
 #pragma unroll 1
   for (int round = 0; round < 6 && sh > 0; ++round) {
@@ -316,7 +322,7 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
     const int nb = 1 << w;
     if (!have_hist) {
       src.for_each([&](unsigned long long x) {
-        if ((x >> sh) == prefix) atomicAdd(&sm.h[static_cast<uint32_t>(x >> nsh) & mask], 1u);
+        if (top(x) == prefix) atomicAdd(&sm.h[static_cast<uint32_t>(x >> nsh) & mask], 1u);
       });
       __syncthreads();
       cl.sync();   // every CTA's digit histogram is complete
@@ -335,7 +341,7 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
     const bool fin = !take_eq && eq <= static_cast<uint32_t>(kFinish);
     uint32_t cu = 0, ce = 0;
     src.for_each([&](unsigned long long x) {
-      if ((x >> sh) == prefix) {
+      if (top(x) == prefix) {
         const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
         cu += dg > t ? 1u : 0u;
         ce += dg == t ? 1u : 0u;
@@ -357,7 +363,7 @@ __device__ void select_rounds(const SaParams &p, SaSmem<D> &sm, cg::cluster_grou
     uint32_t oe = off_e + inc.y - ce;
     unsigned long long *fin0 = cl.map_shared_rank(sm.fin, 0);
     src.for_each([&](unsigned long long x) {
-      if ((x >> sh) != prefix) return;
+      if (top(x) != prefix) return;
       const uint32_t dg = static_cast<uint32_t>(x >> nsh) & mask;
       if (dg > t) {
         if (ou < k_eff) put_sel<kFull>(p, irow, ou, composite_pos(x), composite_z(x));
@@ -433,9 +439,11 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
                                              long long hi, uint32_t b1) {
   constexpr long long kStep = 4LL * kSaThreads * kStreamVec;
   static_assert(4 * kStreamVec <= 32, "one mask bit per score");
-  const float zlo = key_float(b1 << (32 - kHistBits));
+  // b1 is [zlo, zhi) in score order; digit 2 is the 11 key bits below those its keys share
+  const float zlo = b1 == 0u ? -INFINITY : key_float(static_cast<uint32_t>(digit1_floor(b1)));
   const float zhi = b1 + 1 < static_cast<uint32_t>(kHistBins)
-                        ? key_float((b1 + 1) << (32 - kHistBits)) : INFINITY;
+                        ? key_float(static_cast<uint32_t>(digit1_floor(b1 + 1))) : INFINITY;
+  const int d2sh = 32 - digit1_prefix_bits(b1) - kHistBits;   // digit 2 within the order key
   const int lane = threadIdx.x & 31;
   for (long long it = a0; it < hi; it += kStep) {
     const long long b0 = it + 4LL * threadIdx.x;
@@ -497,7 +505,7 @@ __device__ __forceinline__ void stream_chunk(SaSmem<D> &sm, const float *srow,
       const unsigned long long x = composite(key, pos);
       if (oe < static_cast<uint32_t>(kListSmem)) sm.list[oe] = x;
       else spill[oe] = x;
-      atomicAdd(&sm.h[(key >> kDigit2Shift) & (kHistBins - 1)], 1u);
+      atomicAdd(&sm.h[(key >> d2sh) & (kHistBins - 1)], 1u);
       ++oe;
     }
   }
@@ -646,7 +654,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     // this CTA's digit-1 histogram of its candidates and its count of z > T
     uint32_t cnt = 0;
     chunk.for_each([&](unsigned long long x) {
-      atomicAdd(&sm.h[static_cast<uint32_t>(x >> (64 - kHistBits))], 1u);
+      atomicAdd(&sm.h[digit1_bin(static_cast<uint32_t>(x >> 32))], 1u);
       cnt += key_float(static_cast<uint32_t>(x >> 32)) > T ? 1u : 0u;
     });
     uint32_t tot, unused;
@@ -681,7 +689,7 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
     // digit 1 from the scores themselves: this CTA's histogram, then the cluster's threshold
     __syncthreads();
     chunk.for_each([&](unsigned long long x) {
-      atomicAdd(&sm.h[static_cast<uint32_t>(x >> (64 - kHistBits))], 1u);
+      atomicAdd(&sm.h[digit1_bin(static_cast<uint32_t>(x >> 32))], 1u);
     });
     __syncthreads();
     cl.sync();   // every CTA's digit-1 histogram is complete
@@ -719,12 +727,14 @@ __device__ void select_phase(const SaParams &p, const RowGeo &gm, SaSmem<D> &sm,
         put_sel<kFull>(p, irow, off + i, sm.sure[i], __uint_as_float(static_cast<uint32_t>(__ldcg(ztop - i))));
   } else {   // more sure keys than sm.sure holds: from the chunk again
     uint32_t cu = 0;
-    chunk.for_each([&](unsigned long long x) { cu += (x >> (64 - kHistBits)) > b1 ? 1u : 0u; });
+    chunk.for_each([&](unsigned long long x) {
+      cu += digit1_bin(static_cast<uint32_t>(x >> 32)) > b1 ? 1u : 0u;
+    });
     uint32_t tu, unused;
     const uint2 inc = block_scan2(cu, 0u, sm.warp_tot, tu, unused);
     uint32_t o = off + inc.x - cu;
     chunk.for_each([&](unsigned long long x) {
-      if ((x >> (64 - kHistBits)) > b1) {
+      if (digit1_bin(static_cast<uint32_t>(x >> 32)) > b1) {
         if (o < k_eff) put_sel<kFull>(p, irow, o, composite_pos(x), composite_z(x));
         ++o;
       }
