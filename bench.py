@@ -49,14 +49,15 @@ FALLBACK_HBM_GBS = 6650.0
 # keyed by the hash of the score kernel's own sources (score.cu and its TMA helpers, comments
 # removed) it was taken on, so a changed kernel reports null until it is captured again.  Values
 # are per launch of the named workload (the score-kernel ncu summary under profiles/).
-TRAFFIC = {("462c81b3d31dbdfb", "l8b_128k_k1pct"): 274.11e6}
+TRAFFIC = {("3c7ba5e51d427bb6", "l8b_128k_k1pct"): 274.11e6}
 
 
 def score_source_hash() -> str:
-    """sha256 of the score kernel's sources with // comments and blank lines removed, so that
-    a comment edit keeps the key and any code edit changes it."""
+    """sha256 of the score kernel's sources (its own file, the TMA helpers and tensor maps, and
+    the shared header with the digit-1 bin and the parameter structs) with // comments and blank
+    lines removed, so that a comment edit keeps the key and any code edit changes it."""
     h = hashlib.sha256()
-    for f in ("score.cu", "tma.cuh", "tmap.cu"):
+    for f in ("score.cu", "tma.cuh", "tmap.cu", "common.cuh", "kernels.h"):
         with open(os.path.join(ROOT, "top_retrieval_attention_b200", "csrc", f)) as fh:
             for line in fh:
                 code = line.split("//", 1)[0].rstrip()

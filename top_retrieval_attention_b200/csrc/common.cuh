@@ -7,7 +7,7 @@
 
 namespace ra {
 
-constexpr int kHistBits = 11;                 // first radix digit: top 11 bits of the key
+constexpr int kHistBits = 11;                 // radix digits of 11 bits (digit 1: digit1_bin)
 constexpr int kHistBins = 1 << kHistBits;     // 2048 bins per query head
 constexpr int kMaxGroup = 8;                  // query heads per KV head (one n8 MMA tile)
 constexpr int kMetaWords = 8;                 // per-row counters in the workspace

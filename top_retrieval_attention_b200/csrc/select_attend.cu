@@ -428,8 +428,9 @@ __device__ __forceinline__ void warp_scan2(uint32_t &a, uint32_t &b) {
 // scores to the top of `spill` (entry i at spill[hi - lo - 1 - i]); keys in b1
 // (zlo <= z < zhi) go to sm.list as composites, past its capacity to `spill` (room for hi - lo
 // entries: the two never meet, a candidate being one or the other), with their digit-2
-// histogram in sm.h; the counters keep counting past the capacities.  Hits are a few percent of the keys: each thread makes two bit masks with two
-// compares per score, the warp reserves its slots with one shared atomic per list and
+// histogram in sm.h; the counters keep counting past the capacities.  Hits are a small
+// fraction of the keys (about k / |C| plus the bin's share): each thread makes two bit masks
+// with two compares per score, the warp reserves its slots with one shared atomic per list and
 // iteration (offsets from a warp prefix scan of the per-lane counts), and every lane then walks
 // its own set bits (the warp loops as often as its busiest lane has hits), the score of a key
 // in b1 picked from its registers.
