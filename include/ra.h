@@ -52,7 +52,7 @@ typedef enum {
   RA_ERR_CAPACITY = 3,   /* append would exceed the cache capacity                         */
   RA_ERR_WORKSPACE = 4,  /* ws is NULL or ws_bytes is below the required size              */
   RA_ERR_CUDA = 5,       /* a CUDA call or kernel launch failed                            */
-  RA_ERR_EMPTY = 6       /* N == 0: nothing to attend to                                   */
+  RA_ERR_EMPTY = 6       /* empty selected union (N == 0, or W empty and k == 0)           */
 } ra_status;
 
 /*
