@@ -184,14 +184,18 @@ def _scaled_case(N, d, zs, seed):
     return gen.f64_to_bf16_bits(q), K, V
 
 
-@pytest.mark.parametrize("where", ["above_256", "below_m256", "tiny_pos", "tiny_neg", "window_edge"])
-def test_selection_when_the_threshold_is_in_a_catch_all_bin(where):
+@pytest.mark.parametrize("where,seed", [("above_256", 11), ("below_m256", 12), ("tiny_pos", 13),
+                                        ("tiny_neg", 14), ("window_edge", 15),
+                                        ("near_zero_wide", 16)])
+def test_selection_when_the_threshold_is_in_a_catch_all_bin(where, seed):
     """Scores laid out so that the k-th largest candidate falls in each bin that shares no key
-    prefix (z >= 256, z <= -256, 0 <= z < 2^-8, -2^-8 < z < 0) and at the window's lower edge:
-    Omega and out against the oracle."""
+    prefix (z >= 256, z <= -256, 0 <= z < 2^-8, -2^-8 < z < 0, the last from two ranges), and in
+    the first window bin just above 2^-8 with the bin below it crowded and about 270 keys equal
+    to the k-th score (bf16 keys leave some 20 distinct scores): Omega and out against the
+    oracle, and Omega against the exact top-k of the scan's own scores."""
     from parity import check_head
     N, d, k = 6000, 128, 300
-    rng = np.random.default_rng(hash(where) % 1000)
+    rng = np.random.default_rng(seed)
     if where == "above_256":
         zs = rng.uniform(200.0, 400.0, N)
     elif where == "below_m256":
@@ -200,6 +204,8 @@ def test_selection_when_the_threshold_is_in_a_catch_all_bin(where):
         zs = rng.uniform(-0.01, 0.0042, N)
     elif where == "tiny_neg":
         zs = rng.uniform(-0.0045, 0.00005, N)
+    elif where == "window_edge":
+        zs = rng.uniform(0.0035, 0.00395, N)
     else:
         zs = rng.uniform(-0.1, 2 ** -8 * 1.05, N)
     q, K, V = _scaled_case(N, d, zs, 77)
