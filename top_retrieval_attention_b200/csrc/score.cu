@@ -17,10 +17,11 @@
 //     no CTA-wide barrier per tile; every wait is bounded;
 //   * the G query vectors are the n = 8 operand of bf16 m16n8k16 tensor-core products with
 //     fp32 accumulation, read from the stage's query copy when the KV head changes;
-//   * the epilogue scales, writes fp32 z, and builds the first radix digit's histogram (the
-//     2048 bins of digit1_bin over the order-preserving key) of the candidate positions in
+//   * the epilogue scales, writes fp32 z, and builds the histogram of the selection's first
+//     radix digit (digit1_bin_z, computed from the float) over the candidate positions in
 //     shared memory (16-bit counts, two bins a word), flushed to global when the CTA moves to
-//     another KV head;
+//     another KV head; score-row and histogram pointers are set per head and key ranges are
+//     checked per tile, since the consumer warps' issue rate bounds the scan at G = 4-8;
 //   * optionally the step's append is fused in: the CTA whose tile holds the new token writes
 //     its K and V rows to the cache and patches the key row into the staged tile.
 #include <type_traits>
