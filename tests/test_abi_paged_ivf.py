@@ -6,6 +6,8 @@ to and that the caller's structs are left unchanged.
 """
 import ctypes
 
+import pytest
+
 import top_retrieval_attention_b200 as ra
 
 FAKE = 1 << 20   # a 16-byte aligned non-null address; never dereferenced on these paths
@@ -92,3 +94,23 @@ def test_ivf_decode_checks_before_launch():
     assert call(ix, 16, Hq=7) == ra.RA_ERR_SHAPE                 # Hq % Hkv != 0
     assert call(ix, 16, ws_bytes=need - 1) == ra.RA_ERR_WORKSPACE
     assert kv.N == 1010
+
+
+def _ivf_build_bound(B, Hkv, N, nlist):
+    """The build workspace the header states: a key-centroid score block of at most 256 MB (or
+    one 128-key tile's scores when a tile alone is larger), the assignments and the per-1024-key
+    cluster counts, each section 256-byte aligned."""
+    BH = B * Hkv
+    ld = (nlist + 3) // 4 * 4
+    block = max(256 << 20, BH * ld * 4 * 128)
+    return block + 4 * BH * (N + nlist * ((N + 1023) // 1024)) + 4 * 256
+
+
+@pytest.mark.parametrize("B,Hkv,N,d,nlist", [(1, 8, 1 << 20, 128, 1024), (1, 8, 131071, 128, 1024),
+                                             (2, 8, 262144, 64, 256), (64, 8, 4096, 128, 4096)])
+def test_ivf_build_workspace_is_bounded(B, Hkv, N, d, nlist):
+    need = ra.lib().ra_ivf_build_workspace_bytes(B, Hkv, N, d, nlist)
+    assert 4 * B * Hkv * N < need <= _ivf_build_bound(B, Hkv, N, nlist)
+    # far below the whole key-centroid score matrix once N is large
+    if N >= 1 << 20:
+        assert need < B * Hkv * N * nlist * 4 // 50
