@@ -348,7 +348,8 @@ typedef struct {
  * then the final assignment and the sort by cluster, keys of a cluster in increasing position.
  * Deterministic: the same cache gives the same index bit for bit (integer counts, a stable
  * sort, sums in position order).  The key-centroid scores are computed over chunks of keys, so
- * the workspace is about 256 MB plus 4 * B * Hkv * (N + nlist * ceil(N / 1024)) bytes at any N.
+ * the workspace is about 256 MB plus 4 * B * Hkv * (N + nlist * ceil(N / 1024)) bytes at any N
+ * (the 256 MB score block grows to one 128-key tile, B * Hkv * nlist * 512 bytes, if that is larger).
  *   ws : at least ra_ivf_build_workspace_bytes(...) bytes, 256-byte aligned (no zeroing needed).
  * Errors: RA_ERR_ARG, RA_ERR_SHAPE, RA_ERR_WORKSPACE, RA_ERR_CUDA.
  */
